@@ -1,0 +1,206 @@
+"""ctypes binding of the CPU oracle (``lamp_oracle.c``).
+
+Test infrastructure only: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference legs use it; the CUDA library and its
+Python binding never import it. The C library is single threaded; callers that
+want several cores run disjoint row lists from Python threads (ctypes releases
+the GIL during the call).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lamp_oracle.c")
+_LIB = os.path.join(_HERE, "liblamp_oracle.so")
+_CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c99"]
+
+STRICT, RELAXED, GIVEN_MASK = 0, 1, 2
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain C, no contraction of a*b+c)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            L.lamp_oracle_round_ps.restype = ctypes.c_float
+            L.lamp_oracle_round_ps.argtypes = [ctypes.c_float, ctypes.c_int]
+            L.lamp_oracle_round_ps_array.restype = None
+            L.lamp_oracle_round_ps_array.argtypes = [P, P, ctypes.c_int64, ctypes.c_int]
+            L.lamp_oracle_ps_dot.restype = ctypes.c_float
+            L.lamp_oracle_ps_dot.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_float]
+            L.lamp_oracle_fp32_dot.restype = ctypes.c_float
+            L.lamp_oracle_fp32_dot.argtypes = [P, P, ctypes.c_int, ctypes.c_float]
+            L.lamp_oracle_strict_criterion.restype = None
+            L.lamp_oracle_strict_criterion.argtypes = [P, ctypes.c_int, P]
+            L.lamp_oracle_relaxed_criterion.restype = None
+            L.lamp_oracle_relaxed_criterion.argtypes = [P, ctypes.c_int, P]
+            L.lamp_oracle_softmax_pv.restype = None
+            L.lamp_oracle_softmax_pv.argtypes = [P, ctypes.c_int, P, ctypes.c_int, P, P, P]
+            L.lamp_oracle_rows.restype = ctypes.c_int
+            L.lamp_oracle_rows.argtypes = [P, ctypes.c_int, P, P, P, ctypes.c_float, ctypes.c_int,
+                                           ctypes.c_double, ctypes.c_int, P, P, ctypes.c_int64,
+                                           P, P, P, P, P, P, P, P]
+            L.lamp_oracle_row_kl.restype = ctypes.c_double
+            L.lamp_oracle_row_kl.argtypes = [P, P, ctypes.c_int]
+            L.lamp_oracle_kl_rows.restype = None
+            L.lamp_oracle_kl_rows.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64, P]
+            _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_scale(d: int) -> float:
+    """fl32(1/sqrt(d)): 1/sqrt(d) in double, rounded once to binary32."""
+    return float(np.float32(1.0 / np.sqrt(np.float64(d))))
+
+
+def round_ps(x, mu: int) -> np.ndarray:
+    """Elementwise PS(mu) rounding of a float32 array."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(x)
+    lib().lamp_oracle_round_ps_array(_ptr(x), _ptr(out), x.size, int(mu))
+    return out
+
+
+def ps_dot(q_bits, k_bits, mu: int, scale: float) -> np.float32:
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    return np.float32(lib().lamp_oracle_ps_dot(_ptr(q), _ptr(k), q.size, mu, scale))
+
+
+def fp32_dot(q_bits, k_bits, scale: float) -> np.float32:
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    return np.float32(lib().lamp_oracle_fp32_dot(_ptr(q), _ptr(k), q.size, scale))
+
+
+def strict_criterion(ps) -> np.ndarray:
+    ps = np.ascontiguousarray(ps, dtype=np.float32)
+    c = np.zeros(ps.size, dtype=np.float64)
+    lib().lamp_oracle_strict_criterion(_ptr(ps), ps.size, _ptr(c))
+    return c
+
+
+def relaxed_criterion(ps) -> np.ndarray:
+    ps = np.ascontiguousarray(ps, dtype=np.float32)
+    c = np.zeros(ps.size, dtype=np.float64)
+    lib().lamp_oracle_relaxed_criterion(_ptr(ps), ps.size, _ptr(c))
+    return c
+
+
+def softmax_pv(y, V_bits):
+    """Softmax of a score row and P.V (double). Returns (out[d], lse, P[n])."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    V = np.ascontiguousarray(V_bits, dtype=np.uint16)
+    n, d = V.shape
+    out = np.zeros(d, dtype=np.float64)
+    lse = np.zeros(1, dtype=np.float64)
+    P = np.zeros(n, dtype=np.float64)
+    lib().lamp_oracle_softmax_pv(_ptr(y), n, _ptr(V), d, _ptr(out), _ptr(lse), _ptr(P))
+    return out, float(lse[0]), P
+
+
+class RowResult:
+    """Per-row oracle outputs for a list of query rows."""
+
+    def __init__(self, nrows, n_k, d, want_scores=True, want_crit=False):
+        nw = (n_k + 31) // 32
+        self.ps = np.empty((nrows, n_k), np.float32) if want_scores else None
+        self.y32 = np.empty((nrows, n_k), np.float32) if want_scores else None
+        self.mixed = np.empty((nrows, n_k), np.float32) if want_scores else None
+        self.mask = np.zeros((nrows, nw), np.uint32)
+        self.crit = np.empty((nrows, n_k), np.float64) if want_crit else None
+        self.out = np.empty((nrows, d), np.float64)
+        self.lse = np.empty(nrows, np.float64)
+        self.nsel = np.zeros(nrows, np.int64)
+
+
+def attention_rows(Q, K, V, *, causal=True, scale=None, mu=4, tau=0.0, variant=STRICT,
+                   mask_in=None, rows=None, want_scores=True, want_crit=False,
+                   threads: int = 1) -> RowResult:
+    """Oracle LAMP attention for selected query rows.
+
+    Q: uint16 [B, H, n_q, d]; K, V: uint16 [B, H, n_k, d] (bf16 bit patterns).
+    rows: flat row ids (b*H + h)*n_q + i, or None for every row.
+    """
+    Q = np.ascontiguousarray(Q, dtype=np.uint16)
+    K = np.ascontiguousarray(K, dtype=np.uint16)
+    V = np.ascontiguousarray(V, dtype=np.uint16)
+    B, H, n_q, d = Q.shape
+    n_k = K.shape[2]
+    if scale is None:
+        scale = default_scale(d)
+    if rows is None:
+        rows = np.arange(B * H * n_q, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    res = RowResult(rows.size, n_k, d, want_scores, want_crit)
+    dims = np.array([B, H, n_q, n_k, d], dtype=np.int64)
+    if mask_in is not None:
+        mask_in = np.ascontiguousarray(mask_in, dtype=np.uint32)
+    L = lib()
+
+    def run(lo, hi):
+        sub = slice(lo, hi)
+        rc = L.lamp_oracle_rows(
+            _ptr(dims), int(causal), _ptr(Q), _ptr(K), _ptr(V), float(scale), int(mu), float(tau),
+            int(variant), _ptr(mask_in), _ptr(rows[sub]), hi - lo,
+            None if res.ps is None else _ptr(res.ps[sub]),
+            None if res.y32 is None else _ptr(res.y32[sub]),
+            None if res.mixed is None else _ptr(res.mixed[sub]),
+            _ptr(res.mask[sub]), None if res.crit is None else _ptr(res.crit[sub]),
+            _ptr(res.out[sub]), _ptr(res.lse[sub]), _ptr(res.nsel[sub]))
+        if rc != 0:
+            raise ValueError(f"oracle rejected its arguments (rc={rc})")
+
+    n = rows.size
+    if threads <= 1 or n < 2 * threads:
+        run(0, n)
+    else:
+        # interleaved chunks so that causal rows of different lengths spread evenly
+        chunk = max(1, n // (threads * 8))
+        bounds = [(lo, min(n, lo + chunk)) for lo in range(0, n, chunk)]
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda b: run(*b), bounds))
+    return res
+
+
+def kl_rows(y_ref, y_x, n_valid) -> np.ndarray:
+    y_ref = np.ascontiguousarray(y_ref, dtype=np.float32)
+    y_x = np.ascontiguousarray(y_x, dtype=np.float32)
+    nv = np.ascontiguousarray(n_valid, dtype=np.int32)
+    nrows, n_k = y_ref.shape
+    kl = np.zeros(nrows, dtype=np.float64)
+    lib().lamp_oracle_kl_rows(_ptr(y_ref), _ptr(y_x), _ptr(nv), nrows, n_k, _ptr(kl))
+    return kl
+
+
+def calibrate_tau(crit: np.ndarray, n_valid_per_row, rate: float) -> float:
+    """tau giving round(rate * valid) selections: the (k+1)-th largest criterion
+    value among valid entries (entries strictly above it are selected)."""
+    vals = np.concatenate([crit[r, :n] for r, n in enumerate(n_valid_per_row)])
+    k = int(round(rate * vals.size))
+    if k >= vals.size:
+        return -1.0
+    return float(np.partition(vals, vals.size - 1 - k)[vals.size - 1 - k])
