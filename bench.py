@@ -1,0 +1,433 @@
+"""Benchmark of LAMP attention on B200: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--mu MU] [--rate R]
+
+A step is one LAMP attention call over one batch of synthetic inputs: PS(mu)
+scores, look-ahead selection, FP32 recompute of the selected scores, softmax
+and P.V. The default workload is the GPT-2 XL attention shape (batch 1, 25
+heads, 1024 causal tokens, d = 64), strict LAMP, mu = 4, tau from
+tests/golden/tau.json for a 1.6 % recompute rate (computed by the oracle).
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch
+(seed = rank): the (batch, head) units are independent, so there is no
+collective on the data path and the scaling is weak. Timing: per step, CUDA
+events around the call on the launching stream, L2 flushed (256 MB write)
+between steps outside the events; the max over ranks is reported.
+
+--impl reference times the CPU oracle (the plain C definition of the method)
+on this host's cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "LAMP attention G-scores/s at 1x25x1024x64 mu=4; % of roofline; KL vs FP32"
+UNIT = "G-scores/s"
+TAU_FILE = os.path.join(ROOT, "tests", "golden", "tau.json")
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["lamp_strict.cu", "lamp_device.cuh"]
+L2_FLUSH_BYTES = 256 << 20
+N_SM = 148
+FP32_LANES_PER_SM_CLK = 128
+VARIANT_NAMES = {0: "strict", 1: "relaxed", 2: "given_mask"}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gpt2xl_1x25x1024x64", choices=sorted(S.WORKLOADS))
+    ap.add_argument("--variant", type=int, default=None, help="0 strict, 1 relaxed (default: per workload)")
+    ap.add_argument("--mu", type=int, default=4)
+    ap.add_argument("--rate", type=float, default=None, help="target recompute rate (tau from tau.json)")
+    ap.add_argument("--no-kl", action="store_true", help="skip the accuracy evaluation")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+DEFAULTS = {  # workload -> (variant, rate)
+    "gpt2xl_1x25x1024x64": (0, 0.016),
+    "batch8_8x25x1024x64": (1, 0.016),
+    "long_1x32x16384x128": (1, 0.01),
+    "outlier_4x25x4096x64": (0, 0.003),
+    "single_head_128": (0, None),
+}
+
+
+def lookup_tau(workload: str, variant: int, mu: int, rate: float | None) -> tuple[float, float | None]:
+    if workload == "single_head_128" and rate is None:
+        return 0.05, None
+    doc = json.load(open(TAU_FILE))
+    for e in doc["entries"]:
+        if e["workload"] == workload and e["variant"] == variant and e["mu"] == mu and abs(e["rate"] - rate) < 1e-12:
+            return float(e["tau"]), float(e["rate"])
+    raise SystemExit(f"no tau for {workload} variant={variant} mu={mu} rate={rate} in {TAU_FILE}")
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+# ----------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.lines: list[str] = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        mhz, mx, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for (t, line) in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10 or (self.uuid and f[1] != self.uuid):
+                continue
+            if self.t0 and t < self.t0 - 0.05:
+                continue
+            if self.t1 and t > self.t1 + 0.25:
+                continue
+            n += 1
+            try:
+                mhz.append(float(f[2]))
+                mx = float(f[3])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": n}
+
+
+# ----------------------------------------------------------------------------------------
+# reference arm: the CPU oracle on the host cores
+# ----------------------------------------------------------------------------------------
+def sample_rows_for(w: S.Workload, frac: float) -> np.ndarray:
+    """Every m-th query row of every head (a bounded, evenly spread sample)."""
+    total = w.B * w.H * w.n_q
+    m = max(1, int(round(1.0 / frac)))
+    return np.arange(0, total, m, dtype=np.int64)
+
+
+def valid_in_rows(w: S.Workload, rows: np.ndarray) -> int:
+    return int(sum(w.valid_keys(int(r) % w.n_q) for r in rows))
+
+
+def oracle_rate(w, Q, K, V, mu, tau, variant, rows, threads) -> tuple[float, float]:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attention_rows(Q, K, V, causal=w.causal, mu=mu, tau=tau, variant=variant, rows=rows,
+                          want_scores=False, threads=threads)
+    dt = time.perf_counter() - t0
+    return valid_in_rows(w, rows) / dt / 1e9, dt
+
+
+def run_reference(a, w, variant, mu, tau, cfg):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    Q, K, V = S.make_qkv(w)
+    # each step: a fixed sample of rows sized to about 0.1-0.5 s on the host's cores
+    frac = min(1.0, 2.0e6 / max(1, w.valid_scores()))
+    rows = sample_rows_for(w, frac)
+    for _ in range(a.warmup):
+        oracle_rate(w, Q, K, V, mu, tau, variant, rows, threads)
+    times = []
+    for _ in range(a.steps):
+        _, dt = oracle_rate(w, Q, K, V, mu, tau, variant, rows, threads)
+        times.append(dt)
+    per = valid_in_rows(w, rows)
+    ms = 1e3 * statistics.mean(times)
+    value = per / (ms * 1e-3) / 1e9
+    sample = f"{rows.size} of {w.B * w.H * w.n_q} query rows (every {int(round(1 / frac))}th), {per} scores per step"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": cfg, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "mixed_precision_attention_ps_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_bytes(workload: str, variant: int, mu: int) -> float | None:
+    """DRAM bytes per launch of the row kernel from the committed ncu summary, or
+    None when the kernel sources changed since that capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    doc = json.load(open(TRAFFIC_FILE))
+    if doc.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    for e in doc.get("entries", []):
+        if e["workload"] == workload and e["variant"] == variant and e["mu"] == mu:
+            return float(e["dram_bytes_per_launch"])
+    return None
+
+
+def kl_eval(lamp, torch, w, Qd, Kd, Vd, mu, tau, variant, stream):
+    """Mean row KL(P_fp32 || P_x) for no recompute, LAMP at tau, and a random
+    selection of the same per-row count (evaluation only, outside the timed region)."""
+    def run(**kw):
+        r = lamp.attention(Qd, Kd, Vd, mu=mu, causal=w.causal, want_scores=True, want_count=True, stream=stream, **kw)
+        torch.cuda.synchronize()
+        return r
+
+    def mean_kl(ref, x):
+        lp = torch.log_softmax(ref.double(), dim=-1)
+        lq = torch.log_softmax(x.double(), dim=-1)
+        p = lp.exp()
+        t = torch.where(p > 0, p * (lp - lq), torch.zeros_like(p))
+        kl = t.sum(-1)
+        valid = torch.isfinite(ref).any(-1)
+        return float(kl[valid].mean().item())
+
+    ref = run(tau=-1.0, variant=0).mixed_scores
+    base = run(tau=float("inf"), variant=0).mixed_scores
+    lr = run(tau=tau, variant=variant)
+    kl0 = mean_kl(ref, base)
+    kl_l = mean_kl(ref, lr.mixed_scores)
+    counts = lr.mask.view(torch.int32).cpu().numpy().view(np.uint32)
+    per_row = np.unpackbits(counts.view(np.uint8), axis=-1).sum(-1).reshape(w.B * w.H, w.n_q)
+    rmask = S.random_control_mask(w, per_row).reshape(w.B, w.H, w.n_q, -1)
+    rr = run(tau=0.0, variant=2, mask_in=torch.from_numpy(rmask.view(np.int32)).cuda())
+    kl_r = mean_kl(ref, rr.mixed_scores)
+    rate = lr.n_selected.item() / w.valid_scores()
+    return {"recompute_rate": rate, "kl_ps_only": kl0, "kl_lamp": kl_l, "kl_random_same_count": kl_r,
+            "kl_reduction_lamp": kl0 / kl_l if kl_l > 0 else None,
+            "kl_reduction_random": kl0 / kl_r if kl_r > 0 else None,
+            "pages_mu4_context": "GPT-2 XL model-output KL reductions 12x @0.3%, 83x @1.6%, 385x @7.6% "
+                                 "(simulation; a different quantity)"}
+
+
+def run_ours(a, w, variant, mu, tau, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import mixed_precision_attention_ps_b200 as lamp
+
+    rank, local, world = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lamp.load()
+    wr = S.Workload(w.B, w.H, w.n_q, w.n_k, w.d, w.causal, w.outlier_frac, w.outlier_scale, seed=w.seed + rank)
+    Q, K, V = S.make_qkv(wr)
+
+    def dev_t(x):
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    Qd, Kd, Vd = dev_t(Q), dev_t(K), dev_t(V)
+    dims = (w.B, w.H, w.n_q, w.n_k, w.d)
+    nwords = (w.n_k + 31) // 32
+    out = torch.empty_like(Qd)
+    mask = torch.empty((w.B, w.H, w.n_q, nwords), dtype=torch.int32, device=dev)
+    ws_bytes = lamp.lamp_workspace_size(dims, variant)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    args = lamp.make_args(dims, Qd, Kd, Vd, out, mask_out=mask, mu=mu, tau=tau, variant=variant,
+                          causal=int(w.causal), stream=stream, workspace=ws, workspace_bytes=ws_bytes)
+    call = lambda: lamp.lamp_attention_ex(args)  # noqa: E731
+    valid = wr.valid_scores()
+
+    # ---- device-resident timing --------------------------------------------------------
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(getattr(props, "uuid", None) and ("GPU-" + str(props.uuid)))
+    clocks.start()
+    for _ in range(a.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    for s, e in evs:
+        flush.zero_()
+        s.record(stream)
+        call()
+        e.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    times = [s.elapsed_time(e) for s, e in evs]
+    ms = statistics.mean(times)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    launches_per_step = 2  # exponent-statistics kernel + row kernel
+
+    # ---- end to end through the C ABI with host buffers ---------------------------------
+    hQ, hK, hV = (torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).pin_memory() for x in (Q, K, V))
+    hout = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+    hmask = torch.empty(mask.shape, dtype=torch.int32).pin_memory()
+    Qi, Ki, Vi = Qd.view(torch.int16), Kd.view(torch.int16), Vd.view(torch.int16)
+    e2e_steps = max(3, min(a.steps, 500))
+    for _ in range(3):
+        Qi.copy_(hQ, non_blocking=True); Ki.copy_(hK, non_blocking=True); Vi.copy_(hV, non_blocking=True)
+        call()
+        hout.copy_(out.view(torch.int16), non_blocking=True); hmask.copy_(mask, non_blocking=True)
+    torch.cuda.synchronize()
+    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s, e in evs2:
+        flush.zero_()
+        s.record(stream)
+        Qi.copy_(hQ, non_blocking=True); Ki.copy_(hK, non_blocking=True); Vi.copy_(hV, non_blocking=True)
+        call()
+        hout.copy_(out.view(torch.int16), non_blocking=True); hmask.copy_(mask, non_blocking=True)
+        e.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = statistics.mean(s.elapsed_time(e) for s, e in evs2)
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+        dist.barrier()
+    h2d = 3 * Q.nbytes
+    d2h = out.numel() * 2 + mask.numel() * 4
+
+    result = None
+    if rank == 0:
+        value = world * valid / (ms * 1e-3) / 1e9
+        value_e2e = world * valid / (ms_e2e * 1e-3) / 1e9
+        # roofline: ALU issue. 4 d lane-ops per valid score (1 multiply-add + 3 integer
+        # ops of the round-to-nearest-even to mu bits, per accumulation step), against
+        # 128 FP32/INT32 lanes per SM per clock x 148 SMs x the maximum SM clock.
+        peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
+        f_max = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+        peak = N_SM * FP32_LANES_PER_SM_CLK * f_max / 1e12
+        achieved = 4.0 * w.d * valid / (ms * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s",
+                "frac": achieved / peak, "traffic": traffic_bytes(a.workload, variant, mu),
+                "kernel": "lamp row kernel (timed with its exponent-statistics kernel: the whole call)",
+                "peak_basis": f"148 SMs x 128 lanes/clk x {f_max / 1e6:.0f} MHz (max SM clock)"}
+        result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+                  "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                  "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+                  "clocks": clk, "roofline": roof, "gpu_launches": launches_per_step * a.steps,
+                  "e2e": {"value": value_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                          "ms_per_step": ms_e2e},
+                  "attention_gflops": 4.0 * w.d * valid / (ms * 1e-3) / 1e9 * world,
+                  "ms_p10_p90": [float(np.percentile(times, 10)), float(np.percentile(times, 90))]}
+    # accuracy evaluation (rank 0, outside the timed region)
+    if rank == 0 and not a.no_kl:
+        result["accuracy"] = kl_eval(lamp, torch, wr, Qd, Kd, Vd, mu, tau, variant, stream)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not a.no_cpu_baseline and world == 1:
+            result["cpu_baseline"] = cpu_baseline(wr, Q, K, V, mu, tau, variant)
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def cpu_baseline(w, Q, K, V, mu, tau, variant) -> dict:
+    """The oracle as it stands, on the host's cores, over whole-workload passes
+    (or row samples of it) until about 10 s of work have run."""
+    threads = os.cpu_count() or 1
+    total = w.valid_scores()
+    frac = min(1.0, 1.5e8 / total)
+    rows = sample_rows_for(w, frac)
+    per = valid_in_rows(w, rows)
+    t_all, n_scores, passes = 0.0, 0, 0
+    while t_all < 10.0 and passes < 20:
+        _, dt = oracle_rate(w, Q, K, V, mu, tau, variant, rows, threads)
+        t_all += dt
+        n_scores += per
+        passes += 1
+    sample = (f"{passes} pass(es) over {rows.size} of {w.B * w.H * w.n_q} query rows"
+              f" ({per} scores each), {t_all:.1f} s")
+    return {"value": n_scores / t_all / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+
+
+def main():
+    a = parse()
+    w = S.WORKLOADS[a.workload]
+    dv, drate = DEFAULTS[a.workload]
+    variant = dv if a.variant is None else a.variant
+    rate = drate if a.rate is None else a.rate
+    tau, rate = lookup_tau(a.workload, variant, a.mu, rate)
+    cfg = {"workload": a.workload, "B": w.B, "H": w.H, "n_q": w.n_q, "n_k": w.n_k, "d": w.d, "causal": w.causal,
+           "variant": VARIANT_NAMES[variant], "mu": a.mu, "tau": tau, "target_recompute_rate": rate,
+           "inputs": "bf16 N(0,1) (SplitMix64 + Box-Muller), seed = rank", "l2": "flushed between steps (256 MB write)",
+           "valid_scores_per_step_per_gpu": w.valid_scores()}
+    if a.impl == "reference":
+        return run_reference(a, w, variant, a.mu, tau, cfg)
+    return run_ours(a, w, variant, a.mu, tau, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,172 @@
+/*
+ * lamp.h -- C ABI of the B200 (sm_100a) LAMP attention library (liblamp.so).
+ *
+ * LAMP = look-ahead mixed-precision inference ("LAMP: Look-Ahead Mixed-Precision
+ * Inference of Large Language Models", technical summary on gist.science,
+ * paper 2601.21623). The library computes attention in which every key-query
+ * product is first accumulated in a simulated low-precision float PS(mu), a
+ * look-ahead test picks the few products whose rounding error the softmax would
+ * amplify most, only those are recomputed in FP32, and softmax and P.V follow:
+ *   - section "Implementation strategy", steps 1-3: low-precision baseline of g,
+ *     look-ahead selection from that baseline, recompute of the selection in
+ *     higher precision before f;
+ *   - section "Theoretical basis", item 3 (softmax bullet): the strict test
+ *     2 z_j (1 - z_j) |y_j| > tau, z the softmax probabilities of the row;
+ *   - section "Experimental results": PS(mu) (mu mantissa bits), the relaxed
+ *     relative-threshold variant that needs no normalising constant and so fits
+ *     a one-pass softmax, and the random-selection control.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller. Q is
+ *     [B, H, n_q, d], K and V are [B, H, n_k, d], out is [B, H, n_q, d]; all
+ *     contiguous row-major bfloat16 given as raw 16-bit patterns, 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream). Outputs
+ *     are valid once the stream has reached the end of the call.
+ *   - The library keeps no state between calls. It never traps on the device;
+ *     errors are return codes (below), with a message from lamp_last_error().
+ *   - Arguments are checked on the host before anything is launched; a rejected
+ *     call launches nothing and writes nothing.
+ *   - Key j is valid for query row i when causal == 0, or when
+ *     j <= i + (n_k - n_q) (bottom-right aligned causal mask). A row with no
+ *     valid key produces out = 0, lse = -inf and no mask bits.
+ *
+ * Numerical contract (fixed by this library's reading of the pages, which give
+ * no kernel; see the oracle tests for the pins):
+ *   - PS(mu), mu in [1, 23]: binary32 exponent range and subnormals, mu explicit
+ *     fraction bits, round to nearest with ties to even. Score accumulation:
+ *     acc = +0; for k = 0..d-1: acc = round_PS(fl32(acc + fl32(q_k * k_k)));
+ *     y_hat = fl32(scale * acc). mu = 23 is plain binary32.
+ *   - FP32 recompute: the same sequential binary32 sum without rounding, then
+ *     the same scaling.
+ *   - Strict (variant 0): the criterion c_j = 2 z_j (1 - z_j) |y_hat_j| over the
+ *     valid keys of the row, with z = softmax(y_hat); select when c_j > tau.
+ *   - Relaxed (variant 1): c_j = 2 exp(y_hat_j - M_t) |y_hat_j|, M_t the running
+ *     maximum of y_hat over 64-key tiles counted from key 0 up to and including
+ *     the tile of key j; select when c_j > tau. It selects a superset of strict.
+ *   - Given mask (variant 2): select exactly the bits of mask_in (the random
+ *     control of the experiments).
+ *   - Mixed row y_j = FP32 value if selected, else y_hat_j; then P = softmax(y)
+ *     and out = P.V with fp32 accumulation, stored as bf16 (round to nearest even).
+ *   - The selection of an entry whose criterion lies within about 1e-6 relative
+ *     of tau may differ from an exact double-precision evaluation; everything
+ *     else in the scores and the mask is bit-exact with the definition above.
+ */
+#ifndef LAMP_H
+#define LAMP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point is exported from liblamp.so with default visibility. */
+#if defined(__GNUC__)
+#define LAMP_API __attribute__((visibility("default")))
+#else
+#define LAMP_API
+#endif
+
+/* Same handle as cudaStream_t; declared here so that this header needs no CUDA headers. */
+typedef struct CUstream_st *lamp_stream_t;
+
+enum lamp_variant { LAMP_STRICT = 0, LAMP_RELAXED = 1, LAMP_GIVEN_MASK = 2 };
+
+enum lamp_status {
+  LAMP_OK = 0,
+  LAMP_ERR_ARG = -1,          /* null required pointer, mu outside [1,23], tau NaN,
+                                 unknown variant, a dimension <= 0, scale <= 0 or NaN */
+  LAMP_ERR_UNSUPPORTED = -2,  /* d not in {64, 128}; pointer not 16-byte aligned;
+                                 strict/given-mask with n_k > LAMP_MAX_STRICT_NK;
+                                 B * H > 65535 */
+  LAMP_ERR_WORKSPACE = -3,    /* workspace given but smaller than lamp_workspace_size() */
+  LAMP_ERR_CUDA = -4,         /* a CUDA call failed (allocation, launch); see lamp_last_error() */
+  LAMP_ERR_TIMEOUT = -5,      /* reserved: a bounded device wait gave up (none in this version) */
+  LAMP_ERR_CHECK = -6         /* reserved: a device-side check failed (reported via status_out) */
+};
+
+/* Largest n_k accepted by the strict and given-mask variants (their softmax
+ * needs the whole row of scores before any probability is known). */
+#define LAMP_MAX_STRICT_NK 65536
+
+typedef struct {
+  int B, H, n_q, n_k, d;
+} lamp_dims;
+
+/*
+ * lamp_attention -- LAMP attention, basic form.
+ *   dims      shapes (see conventions); d must be 64 or 128.
+ *   Q, K, V   bf16 inputs; out bf16 [B, H, n_q, d].
+ *   mask_out  nullable. uint32 words [B, H, n_q, ceil(n_k/32)]: bit (j % 32) of
+ *             word j / 32 is 1 when score j of the row was recomputed in FP32.
+ *             Bits of invalid keys and of the padding past n_k are 0.
+ *   mu        PS(mu) mantissa bits, 1..23.
+ *   tau       selection threshold (strict and relaxed); tau < 0 recomputes every
+ *             valid score; tau = +inf recomputes none. Ignored for variant 2.
+ *   variant   LAMP_STRICT or LAMP_RELAXED (LAMP_GIVEN_MASK needs lamp_attention_ex).
+ *   causal    0 or 1.
+ * Scratch memory is taken from the stream-ordered allocator and returned before
+ * the call completes on the stream. Returns LAMP_OK or a negative lamp_status.
+ */
+LAMP_API int lamp_attention(const lamp_dims *dims, const void *Q, const void *K, const void *V,
+                   void *out, uint32_t *mask_out, int mu, float tau, int variant,
+                   int causal, lamp_stream_t stream);
+
+/* Extended call. Every field after `stream` is optional (NULL / 0 = off). */
+typedef struct {
+  lamp_dims dims;
+  const void *Q, *K, *V;
+  void *out;
+  uint32_t *mask_out;
+  int mu;
+  float tau;
+  int variant;
+  int causal;
+  lamp_stream_t stream;
+  float scale;                 /* score scale; 0 = fl32(1/sqrt(d)) */
+  const uint32_t *mask_in;     /* LAMP_GIVEN_MASK: words in the mask_out layout; bits of
+                                  invalid keys are ignored */
+  float *out_f32;              /* fp32 copy of out [B, H, n_q, d] before bf16 rounding */
+  float *ps_scores_out;        /* fp32 [B, H, n_q, n_k]: y_hat (invalid keys: -inf) */
+  float *mixed_scores_out;     /* fp32 [B, H, n_q, n_k]: y after recompute (invalid: -inf) */
+  float *lse_out;              /* fp32 [B, H, n_q]: log-sum-exp of the mixed row */
+  unsigned long long *n_selected_out; /* device word: set to the number of recomputed
+                                         scores of this call */
+  void *workspace;             /* device scratch; NULL = stream-ordered allocation */
+  size_t workspace_bytes;
+  int *status_out;             /* reserved (device status word); may be NULL */
+} lamp_args;
+
+LAMP_API int lamp_attention_ex(const lamp_args *args);
+
+/* Bytes of device scratch lamp_attention_ex needs for these shapes and variant
+ * (0 when dims is NULL or invalid). The content need not be initialised. */
+LAMP_API size_t lamp_workspace_size(const lamp_dims *dims, int variant);
+
+/* Message for the last non-zero return on the calling thread ("" if none). */
+LAMP_API const char *lamp_last_error(void);
+
+/*
+ * lamp_ps_round -- elementwise PS(mu) rounding of n binary32 values on the
+ * device (the rounding the score kernels apply after every add). x and y are
+ * device pointers to n floats (may alias). path: 0 = the exact integer
+ * sequence, 1 = the two-instruction floating-point sequence the score kernels
+ * use when the inputs' magnitude range allows it (valid for mu <= 10 and
+ * |x| in {0} U [2^-126, 2^(127 - (23 - mu)))); outside that domain path 1
+ * returns what the hardware sequence computes, which is what the tests check.
+ */
+LAMP_API int lamp_ps_round(const float *x, float *y, size_t n, int mu, int path, lamp_stream_t stream);
+
+/* Library version string. */
+LAMP_API const char *lamp_version(void);
+
+/* sizeof(lamp_args) as compiled into the library, so that a binding can check
+ * that its copy of the struct has the same layout. */
+LAMP_API size_t lamp_args_size(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAMP_H */

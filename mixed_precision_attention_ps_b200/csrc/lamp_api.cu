@@ -1,0 +1,230 @@
+// C ABI of the LAMP attention library: argument checks, workspace planning and
+// the launch sequence (preparation kernel, then the strict or relaxed kernel).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "lamp.h"
+#include "lamp_kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = '\0';
+  return LAMP_OK;
+}
+
+struct DeviceInfo {
+  int num_sms = 0;
+  size_t smem_optin = 0;
+};
+
+// Per-device attributes, queried once per device.
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+cudaError_t device_info(DeviceInfo& out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaError_t qe = cudaSuccess;
+  std::call_once(g_dev_once[dev], [&]() {
+    int sms = 0, optin = 0;
+    qe = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (qe == cudaSuccess) qe = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    g_dev[dev].num_sms = sms;
+    g_dev[dev].smem_optin = (size_t)optin;
+  });
+  if (qe != cudaSuccess) return qe;
+  out = g_dev[dev];
+  if (out.num_sms <= 0) return cudaErrorInvalidDevice;
+  return cudaSuccess;
+}
+
+bool aligned(const void* ptr, size_t a) { return ((uintptr_t)ptr % a) == 0; }
+
+// Largest e_q + e_k (unbiased exponents of the largest |q| and |k| of a head)
+// for which every partial sum x of every PS(mu) score stays below
+// 2^(127 - s): |x| <= d * 2^(e_q + 1) * 2^(e_k + 1) * ((1 + 2^-24)(1 + 2^-(mu+1)))^d.
+int emax_sum_limit(int mu, int d) {
+  const int s = 23 - mu;
+  const double growth = (double)d * std::log2((1.0 + std::ldexp(1.0, -24)) * (1.0 + std::ldexp(1.0, -(mu + 1))));
+  const double lim = 127.0 - s - 2.0 - std::log2((double)d) - growth;
+  return (int)std::floor(lim) - 1;
+}
+
+int check_args(const lamp_args* a) {
+  if (!a) return fail(LAMP_ERR_ARG, "args is NULL");
+  const lamp_dims& d = a->dims;
+  if (d.B <= 0 || d.H <= 0 || d.n_q <= 0 || d.n_k <= 0 || d.d <= 0)
+    return fail(LAMP_ERR_ARG, "dimensions must be positive (B=%d H=%d n_q=%d n_k=%d d=%d)", d.B, d.H,
+                d.n_q, d.n_k, d.d);
+  if (!a->Q || !a->K || !a->V || !a->out) return fail(LAMP_ERR_ARG, "Q, K, V and out must be non-NULL");
+  if (a->mu < 1 || a->mu > 23) return fail(LAMP_ERR_ARG, "mu must be in [1, 23] (got %d)", a->mu);
+  if (a->variant < 0 || a->variant > 2) return fail(LAMP_ERR_ARG, "unknown variant %d", a->variant);
+  if (a->variant != LAMP_GIVEN_MASK && std::isnan(a->tau)) return fail(LAMP_ERR_ARG, "tau is NaN");
+  if (a->variant == LAMP_GIVEN_MASK && !a->mask_in)
+    return fail(LAMP_ERR_ARG, "LAMP_GIVEN_MASK needs mask_in");
+  if (a->causal != 0 && a->causal != 1) return fail(LAMP_ERR_ARG, "causal must be 0 or 1");
+  if (std::isnan(a->scale) || a->scale < 0.f || std::isinf(a->scale))
+    return fail(LAMP_ERR_ARG, "scale must be 0 (default) or a positive finite value");
+  if (d.d != 64 && d.d != 128) return fail(LAMP_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d.d);
+  if (a->variant != LAMP_RELAXED && d.n_k > LAMP_MAX_STRICT_NK)
+    return fail(LAMP_ERR_UNSUPPORTED, "strict/given-mask variants support n_k <= %d", LAMP_MAX_STRICT_NK);
+  const long long rows = (long long)d.B * d.H * d.n_q;
+  if ((long long)d.B * d.H > 65535 || rows > (1LL << 40))
+    return fail(LAMP_ERR_UNSUPPORTED, "problem too large for the index space");
+  if (!aligned(a->Q, 16) || !aligned(a->K, 16) || !aligned(a->V, 16) || !aligned(a->out, 16))
+    return fail(LAMP_ERR_UNSUPPORTED, "Q, K, V and out must be 16-byte aligned");
+  if ((a->mask_out && !aligned(a->mask_out, 4)) || (a->mask_in && !aligned(a->mask_in, 4)) ||
+      (a->out_f32 && !aligned(a->out_f32, 8)) || (a->ps_scores_out && !aligned(a->ps_scores_out, 4)) ||
+      (a->mixed_scores_out && !aligned(a->mixed_scores_out, 4)) || (a->lse_out && !aligned(a->lse_out, 4)) ||
+      (a->n_selected_out && !aligned(a->n_selected_out, 8)))
+    return fail(LAMP_ERR_UNSUPPORTED, "optional outputs must be naturally aligned (out_f32: 8 bytes)");
+  return LAMP_OK;
+}
+
+lamp::Problem make_problem(const lamp_args* a) {
+  lamp::Problem p;
+  p.B = a->dims.B; p.H = a->dims.H; p.n_q = a->dims.n_q; p.n_k = a->dims.n_k; p.d = a->dims.d;
+  p.causal = a->causal;
+  p.mu = a->mu;
+  p.tau = a->tau;
+  p.scale = a->scale > 0.f ? a->scale : (float)(1.0 / std::sqrt((double)a->dims.d));
+  p.variant = a->variant;
+  p.Q = static_cast<const uint16_t*>(a->Q);
+  p.K = static_cast<const uint16_t*>(a->K);
+  p.V = static_cast<const uint16_t*>(a->V);
+  p.out = static_cast<uint16_t*>(a->out);
+  p.mask_out = a->mask_out;
+  p.mask_in = a->mask_in;
+  p.out_f32 = a->out_f32;
+  p.ps_out = a->ps_scores_out;
+  p.mixed_out = a->mixed_scores_out;
+  p.lse_out = a->lse_out;
+  p.nsel_out = a->n_selected_out;
+  p.emax_sum_limit = emax_sum_limit(a->mu, a->dims.d);
+  return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+namespace lamp {
+
+Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
+  Workspace w{};
+  const int BH = p.B * p.H;
+  int nchunk = (2 * num_sms + BH - 1) / BH;
+  if (nchunk < 1) nchunk = 1;
+  if (nchunk > 64) nchunk = 64;
+  const int maxrows = p.n_q > p.n_k ? p.n_q : p.n_k;
+  if (nchunk > maxrows) nchunk = maxrows;
+  w.nchunk = nchunk;
+  w.counters = 0;
+  w.stats = 256;
+  size_t off = align256(w.stats + (size_t)BH * nchunk * 16);
+  w.nkp = ((p.n_k + 127) / 128) * 128 + 4;
+  w.spill = off;
+  w.spill_rows = 0;
+  w.grid = 0;
+  if (strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
+    const long long n_items = (long long)((p.n_q + kStrictBM - 1) / kStrictBM) * BH;
+    w.grid = (int)(n_items < num_sms ? n_items : num_sms);
+    w.spill_rows = 1;
+    off = align256(off + (size_t)w.grid * kStrictBM * w.nkp * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+}  // namespace lamp
+
+extern "C" {
+
+const char* lamp_last_error(void) { return g_err; }
+
+const char* lamp_version(void) { return "lamp-b200 0.1 (sm_100a)"; }
+
+size_t lamp_args_size(void) { return sizeof(lamp_args); }
+
+size_t lamp_workspace_size(const lamp_dims* dims, int variant) {
+  if (!dims || dims->B <= 0 || dims->H <= 0 || dims->n_q <= 0 || dims->n_k <= 0 ||
+      (dims->d != 64 && dims->d != 128) || variant < 0 || variant > 2)
+    return 0;
+  DeviceInfo info;
+  if (device_info(info) != cudaSuccess) return 0;
+  lamp::Problem p{};
+  p.B = dims->B; p.H = dims->H; p.n_q = dims->n_q; p.n_k = dims->n_k; p.d = dims->d;
+  p.variant = variant;
+  return lamp::plan_workspace(p, info.num_sms, info.smem_optin).total;
+}
+
+int lamp_attention_ex(const lamp_args* a) {
+  int rc = check_args(a);
+  if (rc != LAMP_OK) return rc;
+  DeviceInfo info;
+  cudaError_t e = device_info(info);
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
+  lamp::Problem p = make_problem(a);
+  lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
+  if (lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
+    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
+  if (a->workspace && a->workspace_bytes < ws.total)
+    return fail(LAMP_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu bytes needed",
+                a->workspace_bytes, ws.total);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  char* base = static_cast<char*>(a->workspace);
+  bool owned = false;
+  if (!base) {
+    e = cudaMallocAsync(reinterpret_cast<void**>(&base), ws.total, st);
+    if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "workspace allocation failed: %s", cudaGetErrorString(e));
+    owned = true;
+  }
+  e = lamp::launch_prep(p, ws, base, st);
+  if (e == cudaSuccess) e = lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
+  if (owned) {
+    cudaError_t fe = cudaFreeAsync(base, st);
+    if (e == cudaSuccess) e = fe;
+  }
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int lamp_attention(const lamp_dims* dims, const void* Q, const void* K, const void* V, void* out,
+                   uint32_t* mask_out, int mu, float tau, int variant, int causal, lamp_stream_t stream) {
+  if (!dims) return fail(LAMP_ERR_ARG, "dims is NULL");
+  if (variant == LAMP_GIVEN_MASK) return fail(LAMP_ERR_ARG, "LAMP_GIVEN_MASK needs lamp_attention_ex (mask_in)");
+  lamp_args a;
+  std::memset(&a, 0, sizeof(a));
+  a.dims = *dims;
+  a.Q = Q; a.K = K; a.V = V; a.out = out; a.mask_out = mask_out;
+  a.mu = mu; a.tau = tau; a.variant = variant; a.causal = causal; a.stream = stream;
+  return lamp_attention_ex(&a);
+}
+
+int lamp_ps_round(const float* x, float* y, size_t n, int mu, int path, lamp_stream_t stream) {
+  if ((!x || !y) && n) return fail(LAMP_ERR_ARG, "x and y must be non-NULL");
+  if (mu < 1 || mu > 23) return fail(LAMP_ERR_ARG, "mu must be in [1, 23] (got %d)", mu);
+  if (path != 0 && path != 1) return fail(LAMP_ERR_ARG, "path must be 0 or 1");
+  cudaError_t e = lamp::launch_ps_round(x, y, n, mu, path, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // extern "C"

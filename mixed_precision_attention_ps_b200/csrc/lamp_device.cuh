@@ -1,0 +1,200 @@
+// Device helpers shared by the LAMP attention kernels (sm_100a).
+//
+// Method: "LAMP: Look-Ahead Mixed-Precision Inference of Large Language Models"
+// (technical summary, gist.science paper 2601.21623). PS(mu) is the simulated
+// float of section "Experimental results"; the rounding contract is stated in
+// include/lamp.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lamp {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------
+// Packed binary32 pairs. sm_100 executes fma/mul/add on float pairs as one
+// instruction that occupies the FP32 pipe for two lanes' worth of work; one
+// issue slot per pair leaves issue bandwidth for loads and bookkeeping while the
+// FP32 pipe stays saturated. Each lane of the pair is an ordinary IEEE
+// round-to-nearest-even operation.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// ---------------------------------------------------------------------------
+// PS(mu) rounding. s = 23 - mu fraction bits are dropped, round to nearest,
+// ties to even, binary32 exponent range.
+//
+// Exact form (any input): on the bit pattern, add half of the dropped range
+// minus one plus the lowest kept bit, then clear the dropped bits; a carry
+// moves into the exponent (and to infinity past the largest finite value).
+// Infinities and NaNs pass through.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ps_round_exact(float x, int s) {
+  uint32_t u = __float_as_uint(x);
+  if (s == 0 || ((u >> 23) & 0xFFu) == 0xFFu) return x;
+  u += ((1u << (s - 1)) - 1u) + ((u >> s) & 1u);
+  u &= ~((1u << s) - 1u);
+  return __uint_as_float(u);
+}
+
+// Two-instruction form (Veltkamp/Dekker-style splitting, T. J. Dekker, "A
+// floating-point technique for extending the available precision", Numer.
+// Math. 18, 1971): with g = fl(-(2^s - 1) * x), the value fl(2^s * x + g)
+// (one fused multiply-add, exact because 2^s * x + g is representable) is x
+// rounded to 24 - s significant bits. Ties go to even because, for s >= 2, a
+// tie forces the dropped pattern 10..0, so the rounding of g resolves the tie on
+// the kept bits alone. Using 2^s - 1 (not 2^s + 1) keeps 2^s * x - x in or
+// below the binade of 2^s * x; the lower-binade case only arises for x within
+// 2^-s of a power of two, where rounding at twice the resolution agrees as long
+// as s >= mu + 2, i.e. mu <= 10. Valid for mu in [1, 10], x = +0, and normal x
+// with |x| < 2^(127 - s); checked against the exact form over every binary32
+// pattern in that domain. The kernels use it only when the inputs' exponent
+// range keeps every partial sum inside the domain.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ps_round_fast(float x, float neg_c, float pow2s) {
+  float g = __fmul_rn(x, neg_c);
+  return __fmaf_rn(x, pow2s, g);
+}
+
+__device__ __forceinline__ float2 ps_round_fast2(float2 x, float2 neg_c, float2 pow2s) {
+  return fma2(x, pow2s, mul2(x, neg_c));
+}
+
+// ---------------------------------------------------------------------------
+// bfloat16 helpers (inputs are raw 16-bit patterns).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x40u);  // quiet NaN
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// P = hi + lo with hi = bf16(P) and lo = bf16(P - hi): two bf16 values that
+// carry about 16 significant bits of P into the bf16 tensor-core product.
+__device__ __forceinline__ void split_bf16(float p, uint16_t& hi, uint16_t& lo) {
+  hi = f32_to_bf16_rne(p);
+  float r = __fsub_rn(p, __uint_as_float((uint32_t)hi << 16));
+  lo = f32_to_bf16_rne(r);
+}
+
+// ---------------------------------------------------------------------------
+// Warp reductions.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_min_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core helpers for P.V (bf16 inputs, fp32 accumulation).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                            uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                  uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+// ---------------------------------------------------------------------------
+// Per-(b,h) exponent statistics written by the preparation kernel. All four
+// are maxima of non-negative integers so that partial results combine by max:
+//   [0] largest exponent field of Q, [1] 255 - smallest "lsb field" of a nonzero
+//   Q element (lsb field = max(exponent field, 1); 0 when Q is all zero),
+//   [2], [3] the same for K.
+// ---------------------------------------------------------------------------
+struct HeadStats {
+  int v[4];
+};
+
+// True when every partial sum of every PS(mu) score of the head stays inside the
+// domain of ps_round_fast and every product q_k * k_k is exact in binary32, so
+// that fma(q, k, acc) equals fl(acc + fl(q * k)).
+//   emax_sum_limit: largest allowed e_q + e_k (unbiased exponents), computed on
+//   the host from mu and d (see lamp_api.cu).
+__device__ __forceinline__ bool head_fast_ok(const int* partials, int nchunk, int emax_sum_limit) {
+  int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+  for (int c = 0; c < nchunk; ++c) {
+    s0 = max(s0, partials[4 * c + 0]);
+    s1 = max(s1, partials[4 * c + 1]);
+    s2 = max(s2, partials[4 * c + 2]);
+    s3 = max(s3, partials[4 * c + 3]);
+  }
+  if (s1 == 0 || s3 == 0) return (s0 < 255 && s2 < 255);  // an all-zero side: every product is +-0
+  int eq = s0 - 127, ek = s2 - 127;
+  int lq = (255 - s1) - 134, lk = (255 - s3) - 134;  // exponent of the lowest set bit a nonzero value can have
+  return (eq + ek <= emax_sum_limit) && (lq + lk >= -126);
+}
+
+}  // namespace lamp

@@ -1,0 +1,65 @@
+// Host-side launch interface between the C ABI (lamp_api.cu) and the kernels.
+// Plain pointers and sizes only.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lamp {
+
+// Rounding class of mu, fixed per launch:
+//   kRndFast : mu in [1, 10]  (two-instruction rounding when the head allows it,
+//                              exact integer rounding otherwise)
+//   kRndExact: mu in [11, 22] (exact integer rounding only)
+//   kRndNone : mu = 23        (plain binary32; fused multiply-add when allowed)
+enum RoundClass { kRndFast = 0, kRndExact = 1, kRndNone = 2 };
+
+struct Problem {
+  int B, H, n_q, n_k, d;
+  int causal;
+  int mu;
+  float tau;
+  float scale;
+  int variant;
+  const uint16_t* Q;
+  const uint16_t* K;
+  const uint16_t* V;
+  uint16_t* out;
+  uint32_t* mask_out;
+  const uint32_t* mask_in;
+  float* out_f32;
+  float* ps_out;
+  float* mixed_out;
+  float* lse_out;
+  unsigned long long* nsel_out;
+  int emax_sum_limit;  // largest e_q + e_k for which the fast score path is exact
+};
+
+// Workspace layout (bytes from the base, all 256-byte aligned).
+struct Workspace {
+  size_t counters;     // uint32 work counters [4]
+  size_t stats;        // int32 [B*H][nchunk][4]
+  size_t spill;        // fp32 score rows [grid][BM][nkp] (strict path, when rows do not fit on chip)
+  size_t total;
+  int nchunk;
+  int spill_rows;      // 0 when the score rows stay in shared memory
+  int grid;            // persistent grid size used for the spill slabs
+  int nkp;             // padded row length (floats)
+};
+
+// Strict / given-mask configuration: rows per work item and threads.
+constexpr int kStrictBM = 32;
+constexpr int kStrictThreads = 256;
+// Bytes of the opt-in shared memory left for the kernels' static __shared__ data.
+constexpr size_t kStaticSmemReserve = 256;
+
+Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin);
+cudaError_t launch_prep(const Problem& p, const Workspace& ws, char* base, cudaStream_t st);
+cudaError_t launch_strict(const Problem& p, const Workspace& ws, char* base, int num_sms,
+                          size_t smem_optin, cudaStream_t st);
+cudaError_t launch_ps_round(const float* x, float* y, size_t n, int mu, int path, cudaStream_t st);
+
+size_t strict_smem_bytes(int d, int nkp, bool rows_on_chip);
+
+}  // namespace lamp

@@ -1,0 +1,120 @@
+"""Write tests/golden/tau.json: selection thresholds that give the recompute
+rates of the experiments, computed with the CPU oracle only.
+
+LAMP summary, "Experimental results": the accuracy figures are quoted at
+recompute rates of 0.3 %, 1.6 % and 7.6 % of the key-query products (mu = 4).
+For a workload, a variant and mu, tau is the (k+1)-th largest criterion value
+over the valid (query, key) entries, k = round(rate * entries); the entries
+strictly above it are selected, so the selected count is at most k (fewer when
+criterion values tie).
+
+Entries are taken from the whole workload, except for the 16K-token workload,
+where the oracle evaluates a uniform random sample of query rows (seeded; the
+row count is recorded). Sampling rows uniformly keeps the entry distribution,
+since every entry of a sampled row is counted.
+
+    python tests/golden/make_tau.py [--threads N] [--only NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+import synthetic as S  # noqa: E402
+
+OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tau.json")
+
+# (workload, variant, mu list, rates, sampled rows or None)
+PLAN = [
+    ("gpt2xl_1x25x1024x64", oracle.STRICT, [4, 7, 10], [0.003, 0.016, 0.076], None),
+    ("batch8_8x25x1024x64", oracle.RELAXED, [4], [0.016], None),
+    ("long_1x32x16384x128", oracle.RELAXED, [4], [0.01], 768),
+    ("outlier_4x25x4096x64", oracle.STRICT, [4, 6], [0.003, 0.076], None),
+]
+
+
+class TopK:
+    """The largest values of a stream, kept to at most `keep` entries."""
+
+    def __init__(self, keep: int):
+        self.keep = keep
+        self.vals = np.empty(0, np.float64)
+
+    def add(self, v: np.ndarray):
+        v = np.concatenate([self.vals, v])
+        if v.size > self.keep:
+            v = np.partition(v, v.size - self.keep)[v.size - self.keep:]
+        self.vals = v
+
+    def kth_largest(self, k: int) -> float:
+        """(k+1)-th largest value seen (k counted from 0)."""
+        s = np.sort(self.vals)[::-1]
+        return float(s[k])
+
+
+def calibrate(name, variant, mu, rates, sample_rows, threads):
+    w = S.WORKLOADS[name]
+    Q, K, V = S.make_qkv(w)
+    total_rows = w.B * w.H * w.n_q
+    if sample_rows:
+        rng = np.random.default_rng(12345)
+        rows = np.sort(rng.choice(total_rows, size=sample_rows, replace=False)).astype(np.int64)
+    else:
+        rows = np.arange(total_rows, dtype=np.int64)
+    nv = np.array([w.valid_keys(int(r) % w.n_q) for r in rows], dtype=np.int64)
+    entries = int(nv.sum())
+    ks = [int(round(r * entries)) for r in rates]
+    top = TopK(max(ks) + 1)
+    chunk = max(1, int(2 ** 25 // w.n_k))
+    for lo in range(0, rows.size, chunk):
+        sub = rows[lo:lo + chunk]
+        res = oracle.attention_rows(Q, K, V, causal=w.causal, mu=mu, tau=np.inf, variant=variant, rows=sub,
+                                    want_scores=False, want_crit=True, threads=threads)
+        vals = np.concatenate([res.crit[t, :nv[lo + t]] for t in range(sub.size)])
+        top.add(vals)
+    out = []
+    for rate, k in zip(rates, ks):
+        tau = top.kth_largest(k)
+        count = int(np.sum(top.vals > tau))
+        out.append({"workload": name, "variant": int(variant), "mu": mu, "rate": rate, "tau": tau,
+                    "k": k, "entries": entries, "selected_at_tau": count,
+                    "rows": "all" if not sample_rows else f"{sample_rows} random rows (seed 12345)"})
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--threads", type=int, default=os.cpu_count() or 1)
+    ap.add_argument("--only")
+    a = ap.parse_args()
+    table = []
+    if a.only and os.path.exists(OUT):
+        table = [e for e in json.load(open(OUT))["entries"] if e["workload"] != a.only]
+    for name, variant, mus, rates, sample in PLAN:
+        if a.only and name != a.only:
+            continue
+        for mu in mus:
+            t0 = time.time()
+            table += calibrate(name, variant, mu, rates, sample, a.threads)
+            print(f"{name} variant={variant} mu={mu}: {time.time() - t0:.1f} s", flush=True)
+    doc = {
+        "source": "LAMP summary (gist.science paper 2601.21623), 'Experimental results': recompute "
+                  "rates 0.3/1.6/7.6 % at mu = 4; tau = (k+1)-th largest oracle criterion value",
+        "written_by": "tests/golden/make_tau.py (CPU oracle only)",
+        "entries": table,
+    }
+    with open(OUT, "w") as f:
+        json.dump(doc, f, indent=1)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,109 @@
+"""The C ABI without a GPU: the library builds, loads, exports every entry point
+include/lamp.h declares, and rejects bad arguments on the host before any
+CUDA call (so these checks run on a machine with no device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixed_precision_attention_ps_b200 as lamp
+from mixed_precision_attention_ps_b200 import _native, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "lamp.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LAMP_API\s+[\w\s\*]*?\b(lamp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    assert {"lamp_attention", "lamp_attention_ex", "lamp_workspace_size", "lamp_last_error",
+            "lamp_ps_round", "lamp_version", "lamp_args_size"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) == set(_native.SIGNATURES)
+
+
+def test_struct_layout_matches(lib):
+    assert lamp.lamp_args_size() == ctypes.sizeof(_native.lamp_args) == 168
+    assert lamp.lamp_version().startswith("lamp-b200")
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced (checks fail first)
+
+
+def call_ex(**kw):
+    base = dict(dims=(1, 1, 128, 128, 64), Q=FAKE, K=FAKE, V=FAKE, out=FAKE, mu=4, tau=0.05,
+                variant=lamp.LAMP_STRICT, causal=1)
+    base.update(kw)
+    return lamp.lamp_attention_ex(check=False, **base)
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(Q=None), lamp.LAMP_ERR_ARG, "non-NULL"),
+    (dict(out=None), lamp.LAMP_ERR_ARG, "non-NULL"),
+    (dict(mu=0), lamp.LAMP_ERR_ARG, "mu"),
+    (dict(mu=24), lamp.LAMP_ERR_ARG, "mu"),
+    (dict(tau=float("nan")), lamp.LAMP_ERR_ARG, "tau"),
+    (dict(variant=3), lamp.LAMP_ERR_ARG, "variant"),
+    (dict(variant=lamp.LAMP_GIVEN_MASK), lamp.LAMP_ERR_ARG, "mask_in"),
+    (dict(causal=2), lamp.LAMP_ERR_ARG, "causal"),
+    (dict(scale=-1.0), lamp.LAMP_ERR_ARG, "scale"),
+    (dict(scale=float("inf")), lamp.LAMP_ERR_ARG, "scale"),
+    (dict(dims=(0, 1, 128, 128, 64)), lamp.LAMP_ERR_ARG, "positive"),
+    (dict(dims=(1, 1, 128, -1, 64)), lamp.LAMP_ERR_ARG, "positive"),
+    (dict(dims=(1, 1, 128, 128, 96)), lamp.LAMP_ERR_UNSUPPORTED, "d must be"),
+    (dict(dims=(1, 1, 128, 70000, 64)), lamp.LAMP_ERR_UNSUPPORTED, "n_k"),
+    (dict(Q=FAKE + 8), lamp.LAMP_ERR_UNSUPPORTED, "16-byte"),
+    (dict(out_f32=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
+    (dict(n_selected_out=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
+])
+def test_argument_checks(lib, kw, code, msg):
+    rc = call_ex(**kw)
+    assert rc == code
+    assert msg in lamp.lamp_last_error()
+
+
+def test_basic_entry_rejects_given_mask_and_null_dims(lib):
+    L = _native.load()
+    assert L.lamp_attention(None, FAKE, FAKE, FAKE, FAKE, None, 4, 0.1, 0, 1, None) == lamp.LAMP_ERR_ARG
+    rc = lamp.lamp_attention((1, 1, 8, 8, 64), FAKE, FAKE, FAKE, FAKE, None, 4, 0.1,
+                             lamp.LAMP_GIVEN_MASK, 1, check=False)
+    assert rc == lamp.LAMP_ERR_ARG and "lamp_attention_ex" in lamp.lamp_last_error()
+
+
+def test_checked_call_raises_with_message(lib):
+    with pytest.raises(lamp.LampError) as ei:
+        lamp.lamp_attention_ex(dims=(1, 1, 8, 8, 64), Q=FAKE, K=FAKE, V=FAKE, out=FAKE, mu=99)
+    assert ei.value.code == lamp.LAMP_ERR_ARG
+
+
+def test_workspace_size_of_invalid_dims_is_zero(lib):
+    assert lamp.lamp_workspace_size((1, 1, 0, 8, 64), 0) == 0
+    assert lamp.lamp_workspace_size((1, 1, 8, 8, 80), 0) == 0
+    assert lamp.lamp_workspace_size((1, 1, 8, 8, 64), 7) == 0
+
+
+def test_ps_round_argument_checks(lib):
+    assert lamp.lamp_ps_round(None, None, 0, 4, 0, check=False) == 0        # empty: nothing to do
+    assert lamp.lamp_ps_round(None, None, 5, 4, 0, check=False) == lamp.LAMP_ERR_ARG
+    assert lamp.lamp_ps_round(FAKE, FAKE, 5, 0, 0, check=False) == lamp.LAMP_ERR_ARG
+    assert lamp.lamp_ps_round(FAKE, FAKE, 5, 4, 2, check=False) == lamp.LAMP_ERR_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(_native, "_lib", None)
+    with pytest.raises(ImportError, match="no fallback"):
+        _native.load(str(tmp_path / "liblamp.so"))
