@@ -143,7 +143,9 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
   w.spill = off;
   w.spill_rows = 0;
   w.grid = 0;
-  if (strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
+  w.use_ws = ws_fits(p.d, p.n_k, smem_optin) ? 1 : 0;
+  w.rows_bm = w.use_ws ? 0 : rows_pick_bm(p.d, p.n_k, smem_optin);
+  if (!w.use_ws && !w.rows_bm && strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
     const long long n_items = (long long)((p.n_q + kStrictBM - 1) / kStrictBM) * BH;
     w.grid = (int)(n_items < num_sms ? n_items : num_sms);
     w.spill_rows = 1;
@@ -183,7 +185,8 @@ int lamp_attention_ex(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
+  if (!ws.use_ws && !ws.rows_bm &&
+      lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
     return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
   if (a->workspace && a->workspace_bytes < ws.total)
     return fail(LAMP_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu bytes needed",
@@ -197,7 +200,11 @@ int lamp_attention_ex(const lamp_args* a) {
     owned = true;
   }
   e = lamp::launch_prep(p, ws, base, st);
-  if (e == cudaSuccess) e = lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
+  if (e == cudaSuccess) {
+    if (ws.use_ws) e = lamp::launch_ws(p, ws, base, info.num_sms, st);
+    else if (ws.rows_bm) e = lamp::launch_rows(p, ws, base, info.num_sms, st);
+    else e = lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
+  }
   if (owned) {
     cudaError_t fe = cudaFreeAsync(base, st);
     if (e == cudaSuccess) e = fe;

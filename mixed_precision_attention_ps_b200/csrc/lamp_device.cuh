@@ -197,4 +197,130 @@ __device__ __forceinline__ bool head_fast_ok(const int* partials, int nchunk, in
   return (eq + ek <= emax_sum_limit) && (lq + lk >= -126);
 }
 
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// 64-bit packed pairs of binary32 (low word = first element).
+// ---------------------------------------------------------------------------
+typedef unsigned long long u64;
+
+__device__ __forceinline__ u64 fma2u(u64 a, u64 b, u64 c) {
+  u64 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ u64 mul2u(u64 a, u64 b) {
+  u64 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 pack2(float lo, float hi) {
+  return (u64)__float_as_uint(lo) | ((u64)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float lo_f(u64 v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f(u64 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+enum StepMode { kStepFast = 0, kStepF32 = 1, kStepExact = 2 };
+
+// One accumulation step of a pair of scores.
+template <int MODE>
+__device__ __forceinline__ u64 ps_step(u64 q, u64 k, u64 acc, u64 negc, u64 pow2s, int s) {
+  if (MODE == kStepFast) {
+    const u64 x = fma2u(q, k, acc);
+    return fma2u(x, pow2s, mul2u(x, negc));
+  } else if (MODE == kStepF32) {
+    return fma2u(q, k, acc);
+  } else {
+    const float x0 = __fadd_rn(lo_f(acc), __fmul_rn(lo_f(q), lo_f(k)));
+    const float x1 = __fadd_rn(hi_f(acc), __fmul_rn(hi_f(q), hi_f(k)));
+    return pack2(ps_round_exact(x0, s), ps_round_exact(x1, s));
+  }
+}
+
+// P_j stored in place of the score as one 32-bit word: bf16(P) in the low half
+// (the "hi" part) and bf16(P - hi) in the high half (the "lo" part), so that a
+// tensor-core step over k = 2j, 2j+1 against V row j twice yields (hi + lo) V_j.
+__device__ __forceinline__ uint32_t p_pair(float pj) {
+  const uint32_t hi = f32_to_bf16_rne(pj);
+  const float rest = __fsub_rn(pj, __uint_as_float(hi << 16));
+  return hi | ((uint32_t)f32_to_bf16_rne(rest) << 16);
+}
+
+__device__ __forceinline__ float exp_fast(float x) {  // 2^(x log2 e), approximate
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * kLog2e));
+  return y;
+}
+
+
+// ---------------------------------------------------------------------------
+// mbarriers in shared memory and bounded waits. A wait gives up after about two
+// seconds of wall time (%globaltimer), so that a protocol error ends the kernel
+// with an error status instead of a hang.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Wait until the phase with the given parity has completed; false after the limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Named-barrier helpers for warp groups.
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// OR of a predicate over the n threads of barrier id (all of them wait).
+__device__ __forceinline__ int named_or(int id, int n, int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %3, 0;\n\t"
+      "bar.red.or.pred q, %1, %2, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(n), "r"(pred)
+      : "memory");
+  return r;
+}
+
+// bf16 pair of P: low half bf16(P), high half bf16(P - bf16(P)).
+__device__ __forceinline__ uint32_t p_pair_cvt(float pj) {
+  unsigned short h;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(pj));
+  const float rest = __fsub_rn(pj, __uint_as_float((uint32_t)h << 16));
+  uint32_t packed;  // high half bf16(rest), low half bf16(pj)
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed) : "f"(rest), "f"(pj));
+  return packed;
+}
 }  // namespace lamp

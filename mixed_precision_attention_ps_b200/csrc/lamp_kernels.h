@@ -45,12 +45,16 @@ struct Workspace {
   int nchunk;
   int spill_rows;      // 0 when the score rows stay in shared memory
   int grid;            // persistent grid size used for the spill slabs
-  int nkp;             // padded row length (floats)
+  int nkp;             // padded row length (floats) of the global-slab kernel
+  int rows_bm;         // rows per item of the on-chip row kernel; 0 = global-slab kernel
+  int use_ws;          // 1: warp-specialised kernel (two 16-row buffers fit on chip)
 };
 
 // Strict / given-mask configuration: rows per work item and threads.
 constexpr int kStrictBM = 32;
 constexpr int kStrictThreads = 256;
+constexpr int kRowsThreads = 256;
+constexpr int kWsThreads = 512;
 // Bytes of the opt-in shared memory left for the kernels' static __shared__ data.
 constexpr size_t kStaticSmemReserve = 256;
 
@@ -58,6 +62,12 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin);
 cudaError_t launch_prep(const Problem& p, const Workspace& ws, char* base, cudaStream_t st);
 cudaError_t launch_strict(const Problem& p, const Workspace& ws, char* base, int num_sms,
                           size_t smem_optin, cudaStream_t st);
+cudaError_t launch_rows(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
+int rows_pick_bm(int d, int n_k, size_t smem_optin);
+cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
+bool ws_fits(int d, int n_k, size_t smem_optin);
+int rows_nkp(int bm, int n_k);
+size_t rows_smem_bytes(int d, int bm, int n_k);
 cudaError_t launch_ps_round(const float* x, float* y, size_t n, int mu, int path, cudaStream_t st);
 
 size_t strict_smem_bytes(int d, int nkp, bool rows_on_chip);
