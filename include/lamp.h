@@ -22,8 +22,9 @@
  *     contiguous row-major bfloat16 given as raw 16-bit patterns, 16-byte aligned.
  *   - Calls are asynchronous on `stream` (NULL = legacy default stream). Outputs
  *     are valid once the stream has reached the end of the call.
- *   - The library keeps no state between calls. It never traps on the device;
- *     errors are return codes (below), with a message from lamp_last_error().
+ *   - Between calls the library keeps only per-device attributes and a scratch
+ *     memory pool. It never traps on the device; errors are return codes
+ *     (below), with a message from lamp_last_error().
  *   - Arguments are checked on the host before anything is launched; a rejected
  *     call launches nothing and writes nothing.
  *   - Key j is valid for query row i when causal == 0, or when
@@ -82,7 +83,7 @@ enum lamp_status {
                                  B * H > 65535 */
   LAMP_ERR_WORKSPACE = -3,    /* workspace given but smaller than lamp_workspace_size() */
   LAMP_ERR_CUDA = -4,         /* a CUDA call failed (allocation, launch); see lamp_last_error() */
-  LAMP_ERR_TIMEOUT = -5,      /* reserved: a bounded device wait gave up (none in this version) */
+  LAMP_ERR_TIMEOUT = -5,      /* written to status_out by a kernel whose bounded wait gave up */
   LAMP_ERR_CHECK = -6         /* reserved: a device-side check failed (reported via status_out) */
 };
 
@@ -106,8 +107,10 @@ typedef struct {
  *             valid score; tau = +inf recomputes none. Ignored for variant 2.
  *   variant   LAMP_STRICT or LAMP_RELAXED (LAMP_GIVEN_MASK needs lamp_attention_ex).
  *   causal    0 or 1.
- * Scratch memory is taken from the stream-ordered allocator and returned before
- * the call completes on the stream. Returns LAMP_OK or a negative lamp_status.
+ * Scratch memory comes from a stream-ordered memory pool that the library creates
+ * for each device on first use and keeps (with the memory it has grown to) until
+ * the process exits; it is returned to that pool when the call completes on the
+ * stream. Returns LAMP_OK or a negative lamp_status.
  */
 LAMP_API int lamp_attention(const lamp_dims *dims, const void *Q, const void *K, const void *V,
                    void *out, uint32_t *mask_out, int mu, float tau, int variant,
@@ -133,9 +136,11 @@ typedef struct {
   float *lse_out;              /* fp32 [B, H, n_q]: log-sum-exp of the mixed row */
   unsigned long long *n_selected_out; /* device word: set to the number of recomputed
                                          scores of this call */
-  void *workspace;             /* device scratch; NULL = stream-ordered allocation */
+  void *workspace;             /* device scratch; NULL = the library's per-device pool */
   size_t workspace_bytes;
-  int *status_out;             /* reserved (device status word); may be NULL */
+  int *status_out;             /* device status word, may be NULL: set to LAMP_ERR_TIMEOUT when
+                                  a bounded wait inside a kernel gave up (the outputs of the
+                                  call are then undefined); never cleared by the library */
 } lamp_args;
 
 LAMP_API int lamp_attention_ex(const lamp_args *args);

@@ -29,6 +29,7 @@ int ok() {
 struct DeviceInfo {
   int num_sms = 0;
   size_t smem_optin = 0;
+  cudaMemPool_t pool = nullptr;  // scratch pool of this device; keeps its memory between calls
 };
 
 // Per-device attributes, queried once per device.
@@ -48,10 +49,24 @@ cudaError_t device_info(DeviceInfo& out) {
     if (qe == cudaSuccess) qe = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     g_dev[dev].num_sms = sms;
     g_dev[dev].smem_optin = (size_t)optin;
+    if (qe == cudaSuccess) {
+      cudaMemPoolProps props;
+      std::memset(&props, 0, sizeof(props));
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t pool = nullptr;
+      qe = cudaMemPoolCreate(&pool, &props);
+      if (qe == cudaSuccess) {
+        uint64_t keep = ~0ull;  // never hand freed scratch back to the driver
+        qe = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        g_dev[dev].pool = pool;
+      }
+    }
   });
   if (qe != cudaSuccess) return qe;
   out = g_dev[dev];
-  if (out.num_sms <= 0) return cudaErrorInvalidDevice;
+  if (out.num_sms <= 0 || !out.pool) return cudaErrorInvalidDevice;
   return cudaSuccess;
 }
 
@@ -93,7 +108,7 @@ int check_args(const lamp_args* a) {
   if ((a->mask_out && !aligned(a->mask_out, 4)) || (a->mask_in && !aligned(a->mask_in, 4)) ||
       (a->out_f32 && !aligned(a->out_f32, 8)) || (a->ps_scores_out && !aligned(a->ps_scores_out, 4)) ||
       (a->mixed_scores_out && !aligned(a->mixed_scores_out, 4)) || (a->lse_out && !aligned(a->lse_out, 4)) ||
-      (a->n_selected_out && !aligned(a->n_selected_out, 8)))
+      (a->n_selected_out && !aligned(a->n_selected_out, 8)) || (a->status_out && !aligned(a->status_out, 4)))
     return fail(LAMP_ERR_UNSUPPORTED, "optional outputs must be naturally aligned (out_f32: 8 bytes)");
   return LAMP_OK;
 }
@@ -117,6 +132,7 @@ lamp::Problem make_problem(const lamp_args* a) {
   p.mixed_out = a->mixed_scores_out;
   p.lse_out = a->lse_out;
   p.nsel_out = a->n_selected_out;
+  p.status_out = a->status_out;
   p.emax_sum_limit = emax_sum_limit(a->mu, a->dims.d);
   return p;
 }
@@ -195,7 +211,7 @@ int lamp_attention_ex(const lamp_args* a) {
   char* base = static_cast<char*>(a->workspace);
   bool owned = false;
   if (!base) {
-    e = cudaMallocAsync(reinterpret_cast<void**>(&base), ws.total, st);
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&base), ws.total, info.pool, st);
     if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "workspace allocation failed: %s", cudaGetErrorString(e));
     owned = true;
   }

@@ -33,6 +33,7 @@ struct Problem {
   float* mixed_out;
   float* lse_out;
   unsigned long long* nsel_out;
+  int* status_out;       // optional device status word (LAMP_ERR_TIMEOUT on a bounded wait that gave up)
   int emax_sum_limit;  // largest e_q + e_k for which the fast score path is exact
 };
 

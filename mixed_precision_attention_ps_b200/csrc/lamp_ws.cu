@@ -13,23 +13,27 @@
 // order over the CTAs. Two row buffers alternate between two warp groups:
 //
 //   producers (warps 0-7): PS(mu) scores of item k into buffer k & 1. The item's
-//     keys are cut into 32-key units dealt round-robin to the producer warps,
-//     continuing across items, so no warp idles at the end of an item. Each warp
-//     stages its own K slices (16 head dimensions x 32 keys, binary32, double
-//     buffered) and needs no block-wide barrier; a lane holds 4 rows x 4 keys as
-//     packed binary32 pairs; one accumulation step is fma.rn.f32x2 plus the
-//     two-instruction PS(mu) rounding (or the exact integer rounding).
-//   consumers (warps 8-15): for item k, two rows per warp processed together:
-//     row maximum and first argmax, S_rest in double (strict), the criterion with
-//     a double re-evaluation near tau, mask words, warp-compacted FP32 recompute,
-//     softmax numerators of the mixed row written in place as bf16 hi/lo pairs;
-//     then P.V on tensor cores (mma.sync, V staged by cp.async) and the output.
+//     keys are cut into 64-key units dealt round-robin to the producer warps,
+//     continuing across items. Each warp stages its own K slices (8 head
+//     dimensions x 64 keys, binary32, double buffered) and waits for nothing but
+//     a free buffer. A lane holds 8 rows x 4 keys as sixteen packed binary32
+//     pairs (two rows of one key per 64-bit register): one accumulation step is
+//     fma.rn.f32x2 plus the two-instruction PS(mu) rounding (or the exact
+//     integer rounding), and three shared-memory loads feed 16 packed steps.
+//   consumers (warps 8-15): for item k, two rows per warp, four keys per lane:
+//     row maximum and first argmax, S_rest in double (strict), the criterion
+//     with a double re-evaluation near tau, mask words, warp-compacted FP32
+//     recompute, softmax numerators of the mixed row written in place as bf16
+//     hi/lo pairs; then P.V on tensor cores (mma.sync, V staged by cp.async), the
+//     output, and the staging of Q for item k + 2.
 //
-// Hand-offs use named barriers: "full[b]" (producers arrive, consumers wait) and
-// "empty[b]" (consumers arrive, producers wait), so each side blocks only when
-// the other is a whole item behind.
+// Hand-offs use mbarriers: full[b] (256 producer arrivals per item) and empty[b]
+// (256 consumer arrivals: the buffer and its Q are ready for the next item).
+// Every wait is bounded; a wait that gives up records LAMP_ERR_TIMEOUT in the
+// caller's status word (when given) and ends the kernel.
 #include <cfloat>
 
+#include "lamp.h"
 #include "lamp_device.cuh"
 #include "lamp_kernels.h"
 
@@ -40,30 +44,19 @@ constexpr int WS_BM = 16;              // query rows per item
 constexpr int WS_NT = kWsThreads;      // 512
 constexpr int WS_NP = 8;               // producer warps
 constexpr int WS_NC = 8;               // consumer warps
-constexpr int WS_UNIT = 32;            // keys per producer unit
-constexpr int WS_DS = 16;              // head dimensions per K slice
+constexpr int WS_UNIT = 64;            // keys per producer unit
+constexpr int WS_DS = 8;               // head dimensions per K slice
 constexpr int WS_LIST = 64;            // per-warp recompute list capacity
 constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
-
-// named barriers (0 is __syncthreads, unused after the split)
-constexpr int BAR_EMPTY0 = 1;          // + buffer
-constexpr int BAR_FULL0 = 3;           // + buffer
-constexpr int BAR_PROD = 5;            // producers only
-constexpr int BAR_CONS = 6;            // consumers only
-
-__device__ __forceinline__ void bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ void bar_arrive(int id, int n) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
+constexpr int BAR_CONS = 1;            // named barrier of the consumer group
 
 template <int D>
 __host__ __device__ constexpr int ws_vkeys() { return D == 64 ? 128 : 64; }
 
 struct WsSmem {
-  int q;      // Q pairs [2][D][16] u64
-  int ks;     // producer K slices [8 warps][2][16][32] f32
+  int bars;   // mbarriers: full[2], empty[2]
+  int q;      // Q [2][D][16] f32
+  int ks;     // producer K slices [8 warps][2][8][64] f32
   int v;      // consumer V chunks [2][VK][D + 8] bf16, later the output sums [16][D] f32
   int list;   // consumer recompute lists [8][64] int
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
@@ -74,8 +67,9 @@ struct WsSmem {
 template <int D>
 __host__ __device__ inline WsSmem ws_plan(int nkp) {
   WsSmem s{};
-  s.q = 0;
-  s.ks = s.q + 2 * D * WS_BM * 8;
+  s.bars = 0;
+  s.q = 64;
+  s.ks = s.q + 2 * D * WS_BM * 4;
   s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
   const int vb = 2 * ws_vkeys<D>() * (D + 8) * 2;
   const int ob = WS_BM * D * 4;
@@ -94,10 +88,6 @@ struct WsArgs {
   int n_items;
   int n_rb;
 };
-
-// Row r (0..15) of the Q pair layout: lane group gr reads rows 4gr + 2h and
-// 4gr + 2h + 1 with one 16-byte load at h * 8 + 2gr.
-__device__ __forceinline__ int ws_qpos(int r) { return ((r >> 1) & 1) * 8 + (r >> 2) * 2 + (r & 1); }
 
 // The k-th item of CTA b (snake order over heaviest-first items), or -1.
 __device__ __forceinline__ int ws_item(int k, int b, int G, int n_items) {
@@ -126,22 +116,43 @@ __device__ __forceinline__ int ws_valid_keys(int i, const Problem& p) {
   return min(p.n_k, max(0, i + 1 + (p.n_k - p.n_q)));
 }
 
-// WS_DS accumulation steps of a lane's 4 x 4 score tile (16-row items).
-//   qs: Q pairs of this slice, [WS_DS][16] u64; ks: warp's K slice, [WS_DS][32] f32.
+__device__ __forceinline__ void ws_timeout(const Problem& p) {
+  if (p.status_out) atomicExch(p.status_out, LAMP_ERR_TIMEOUT);
+}
+
+// Q rows of an item as binary32 [D][16] (rows past the problem are zero).
+template <int D>
+__device__ __forceinline__ void ws_stage_q(float* sQ, const Problem& p, const ItemInfo& it, int t, int nthreads) {
+  for (int u = t; u < WS_BM * D / 8; u += nthreads) {
+    const int r = u / (D / 8), c8 = (u % (D / 8)) * 8;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (r < it.rows) w = __ldg(reinterpret_cast<const uint4*>(p.Q + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8));
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sQ[(c8 + 2 * e) * WS_BM + r] = bf16_lo(ws[e]);
+      sQ[(c8 + 2 * e + 1) * WS_BM + r] = bf16_hi(ws[e]);
+    }
+  }
+}
+
+// WS_DS accumulation steps of a lane's 8-row x 4-key tile.
+//   qs: Q of this slice, [WS_DS][16] f32 (lane rows 8gr..8gr+7 at qoff = 8gr);
+//   ks: warp's K slice, [WS_DS][64] f32 (lane keys at koff = 4gk).
 template <int MODE>
-__device__ __forceinline__ void score_slice_ws(const u64* __restrict__ qs, const float* __restrict__ ks, int qoff,
-                                               int koff, u64 (&acc)[4][2], u64 negc, u64 pow2s, int s) {
-#pragma unroll 4
+__device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, const float* __restrict__ ks, int qoff,
+                                               int koff, u64 (&acc)[4][4], u64 negc, u64 pow2s, int s) {
+#pragma unroll
   for (int dd = 0; dd < WS_DS; ++dd) {
     const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff);
-    const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + 8 + qoff);
-    const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(ks + dd * WS_UNIT + koff);
+    const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff + 4);
+    const float4 kk = *reinterpret_cast<const float4*>(ks + dd * WS_UNIT + koff);
     const u64 q[4] = {qa.x, qa.y, qb.x, qb.y};
+    const u64 k[4] = {pack2(kk.x, kk.x), pack2(kk.y, kk.y), pack2(kk.z, kk.z), pack2(kk.w, kk.w)};
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      acc[r][0] = ps_step<MODE>(q[r], kk.x, acc[r][0], negc, pow2s, s);
-      acc[r][1] = ps_step<MODE>(q[r], kk.y, acc[r][1], negc, pow2s, s);
-    }
+    for (int rp = 0; rp < 4; ++rp)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[rp][i] = ps_step<MODE>(q[rp], k[i], acc[rp][i], negc, pow2s, s);
   }
 }
 
@@ -153,38 +164,26 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
                                             int lane) {
   constexpr int NSL = D / WS_DS;  // K slices per unit
   const Problem& p = a.p;
-  const int tidp = warp * 32 + lane;
   const int G = gridDim.x, cta = blockIdx.x;
   const int s = 23 - p.mu;
   const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
   const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
   const u64 scale2 = pack2(p.scale, p.scale);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);  // full[0], full[1], empty[0], empty[1]
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
-  const int gr = lane & 3, gk = lane >> 2;  // rows 4gr..4gr+3, keys 4gk..4gk+3 of a unit
-  const int qoff = 2 * gr, koff = 4 * gk;
+  const int gr = lane & 1, gk = lane >> 1;  // rows 8gr..8gr+7, keys 4gk..4gk+3 of a unit
+  const int qoff = 8 * gr, koff = 4 * gk;
   int deal = 0;  // producer warp that takes the next unit
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
     if (q < 0) break;
     const int buf = k & 1;
     const ItemInfo it = ws_decode(q, a);
-    bar_sync(BAR_EMPTY0 + buf, WS_NT);  // the consumers are done with this buffer
-    u64* sQ = reinterpret_cast<u64*>(smem + L.q) + buf * D * WS_BM;
-    for (int u = tidp; u < WS_BM * D / 8; u += WS_NP * 32) {
-      const int r = u / (D / 8), c8 = (u % (D / 8)) * 8;
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (r < it.rows)
-        w = __ldg(reinterpret_cast<const uint4*>(p.Q + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8));
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-      const int pos = ws_qpos(r);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float v0 = bf16_lo(ws[e]), v1 = bf16_hi(ws[e]);
-        sQ[(c8 + 2 * e) * WS_BM + pos] = pack2(v0, v0);
-        sQ[(c8 + 2 * e + 1) * WS_BM + pos] = pack2(v1, v1);
-      }
+    if (!mbar_wait(bars + 2 + buf, (k >> 1) & 1)) {  // buffer free, Q staged
+      ws_timeout(p);
+      return;
     }
-    bar_sync(BAR_PROD, WS_NP * 32);
+    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + buf * D * WS_BM;
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
@@ -194,14 +193,13 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
     const int mine = first < U ? (U - first + WS_NP - 1) / WS_NP : 0;
     const int total = mine * NSL;
     uint4 kr[2];
-    auto load = [&](int pos) {  // slice of stream position pos into registers
+    auto load = [&](int pos) {  // keys lane and lane + 32 of the slice at stream position pos
       const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
-      const int key = j * WS_UNIT + lane;
-      kr[0] = kr[1] = make_uint4(0u, 0u, 0u, 0u);
-      if (key < it.kv_end) {
-        const uint4* src = reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS);
-        kr[0] = __ldg(src);
-        kr[1] = __ldg(src + 1);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int key = j * WS_UNIT + lane + 32 * h;
+        kr[h] = make_uint4(0u, 0u, 0u, 0u);
+        if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
       }
     };
     auto store = [&](int b2) {
@@ -211,8 +209,8 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
         const uint32_t ws[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          dst[(8 * h + 2 * e) * WS_UNIT] = bf16_lo(ws[e]);
-          dst[(8 * h + 2 * e + 1) * WS_UNIT] = bf16_hi(ws[e]);
+          dst[(2 * e) * WS_UNIT + 32 * h] = bf16_lo(ws[e]);
+          dst[(2 * e + 1) * WS_UNIT + 32 * h] = bf16_hi(ws[e]);
         }
       }
     };
@@ -221,47 +219,56 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
       store(0);
     }
     __syncwarp();
-    u64 acc[4][2];
+    u64 acc[4][4];
     for (int pos = 0; pos < total; ++pos) {
       const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
       if (pos + 1 < total) load(pos + 1);
       if (sl == 0) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = 0ull;
+        for (int rp = 0; rp < 4; ++rp)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[rp][i] = 0ull;
       }
-      const u64* qs = sQ + sl * WS_DS * WS_BM;
+      const float* qs = sQ + sl * WS_DS * WS_BM;
       const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
-      if (RND == kRndFast && fast) score_slice_ws<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      else if (RND == kRndNone && fast) score_slice_ws<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      else score_slice_ws<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+      if (RND == kRndFast && fast) ws_score_slice<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+      else if (RND == kRndNone && fast) ws_score_slice<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+      else ws_score_slice<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
       if (sl == NSL - 1) {
         const int j0 = j * WS_UNIT + koff;
 #pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-          const int r = 4 * gr + r4;
-          const int nv = r < it.rows ? ws_valid_keys(it.i0 + r, p) : 0;
-          const u64 y01 = mul2u(acc[r4][0], scale2), y23 = mul2u(acc[r4][1], scale2);
-          float4 y;
-          y.x = j0 < nv ? lo_f(y01) : -INFINITY;
-          y.y = j0 + 1 < nv ? hi_f(y01) : -INFINITY;
-          y.z = j0 + 2 < nv ? lo_f(y23) : -INFINITY;
-          y.w = j0 + 3 < nv ? hi_f(y23) : -INFINITY;
-          *reinterpret_cast<float4*>(rows + (size_t)r * a.nkp + j0) = y;
+        for (int rp = 0; rp < 4; ++rp) {
+          const int r0 = 8 * gr + 2 * rp;
+          const int nv0 = r0 < it.rows ? ws_valid_keys(it.i0 + r0, p) : 0;
+          const int nv1 = r0 + 1 < it.rows ? ws_valid_keys(it.i0 + r0 + 1, p) : 0;
+          float4 y0, y1;
+          const u64 a0 = mul2u(acc[rp][0], scale2), a1 = mul2u(acc[rp][1], scale2);
+          const u64 a2 = mul2u(acc[rp][2], scale2), a3 = mul2u(acc[rp][3], scale2);
+          y0.x = j0 < nv0 ? lo_f(a0) : -INFINITY;
+          y0.y = j0 + 1 < nv0 ? lo_f(a1) : -INFINITY;
+          y0.z = j0 + 2 < nv0 ? lo_f(a2) : -INFINITY;
+          y0.w = j0 + 3 < nv0 ? lo_f(a3) : -INFINITY;
+          y1.x = j0 < nv1 ? hi_f(a0) : -INFINITY;
+          y1.y = j0 + 1 < nv1 ? hi_f(a1) : -INFINITY;
+          y1.z = j0 + 2 < nv1 ? hi_f(a2) : -INFINITY;
+          y1.w = j0 + 3 < nv1 ? hi_f(a3) : -INFINITY;
+          *reinterpret_cast<float4*>(rows + (size_t)r0 * a.nkp + j0) = y0;
+          *reinterpret_cast<float4*>(rows + (size_t)(r0 + 1) * a.nkp + j0) = y1;
         }
       }
       if (pos + 1 < total) store((pos + 1) & 1);
       __syncwarp();
     }
     deal = (deal + U) % WS_NP;
-    bar_arrive(BAR_FULL0 + buf, WS_NT);  // scores of this item are in place
+    mbar_arrive(bars + buf);  // this thread's scores of item k are in place
   }
 }
 
-// FP32 recompute of score (row r, key j) from the Q pairs and K in global memory.
+// FP32 recompute of score (row r, key j): the sequential binary32 sum over
+// k = 0..D-1 (a fused multiply-add when the head's products are exact), then the scale.
 template <int D>
-__device__ __forceinline__ float ws_recompute(const u64* __restrict__ sQ, int r, const uint16_t* __restrict__ krow,
+__device__ __forceinline__ float ws_recompute(const float* __restrict__ sQ, int r, const uint16_t* __restrict__ krow,
                                               float scale, bool fused) {
-  const int pos = ws_qpos(r);
   float acc = 0.f;
 #pragma unroll
   for (int kk = 0; kk < D; kk += 8) {
@@ -270,8 +277,7 @@ __device__ __forceinline__ float ws_recompute(const u64* __restrict__ sQ, int r,
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float k0 = bf16_lo(ws[e]), k1 = bf16_hi(ws[e]);
-      const float q0 = lo_f(sQ[(kk + 2 * e) * WS_BM + pos]);
-      const float q1 = lo_f(sQ[(kk + 2 * e + 1) * WS_BM + pos]);
+      const float q0 = sQ[(kk + 2 * e) * WS_BM + r], q1 = sQ[(kk + 2 * e + 1) * WS_BM + r];
       if (fused) {
         acc = __fmaf_rn(q0, k0, acc);
         acc = __fmaf_rn(q1, k1, acc);
@@ -284,10 +290,14 @@ __device__ __forceinline__ float ws_recompute(const u64* __restrict__ sQ, int r,
   return __fmul_rn(scale, acc);
 }
 
+__device__ __forceinline__ float4 lds4_or_ninf(const float* ptr, bool ok) {
+  return ok ? *reinterpret_cast<const float4*>(ptr) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+}
+
 // ---------------------------------------------------------------------------
 // Consumers: selection, recompute, softmax, P.V and the output of every item.
 // ---------------------------------------------------------------------------
-template <int D, int RND>
+template <int D, int RND, int VAR>
 __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int cw,
                                             int lane) {
   constexpr int VK = ws_vkeys<D>();
@@ -296,38 +306,64 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   constexpr int KQ = WS_NC / NH;
   constexpr int SPW = (VK / 8) / KQ;
   constexpr int TPG = 8 / KQ;
+  constexpr int NCT = WS_NC * 32;  // consumer threads
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
   const int G = gridDim.x, cta = blockIdx.x;
   const int nwords = (p.n_k + 31) >> 5;
   const uint32_t lanemask_lt = (1u << lane) - 1u;
-  const bool strict = p.variant == 0, relaxed = p.variant == 1, given = p.variant == 2;
-  const bool refine_ok = isfinite(p.tau) && p.tau >= 0.f;
+  const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = WS_BAND * p.tau;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   int* list = reinterpret_cast<int*>(smem + L.list) + cw * WS_LIST;
   uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L.v);
   float* sO = reinterpret_cast<float*>(smem + L.v);
+  float* qbase = reinterpret_cast<float*>(smem + L.q);
   long long nsel = 0;
-  // the first two buffers start out free
-  if (ws_item(0, cta, G, a.n_items) >= 0) bar_arrive(BAR_EMPTY0 + 0, WS_NT);
-  if (ws_item(1, cta, G, a.n_items) >= 0) bar_arrive(BAR_EMPTY0 + 1, WS_NT);
+  // Q of the first two items, then both buffers are released to the producers
+  for (int k0 = 0; k0 < 2; ++k0) {
+    const int q0 = ws_item(k0, cta, G, a.n_items);
+    if (q0 < 0) break;
+    ws_stage_q<D>(qbase + k0 * D * WS_BM, p, ws_decode(q0, a), tidc, NCT);
+    mbar_arrive(bars + 2 + k0);
+  }
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
     if (q < 0) break;
     const int buf = k & 1;
     const ItemInfo it = ws_decode(q, a);
-    bar_sync(BAR_FULL0 + buf, WS_NT);  // the producers have written this item's scores
-    const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
-                                                          p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
-    const u64* sQ = reinterpret_cast<const u64*>(smem + L.q) + buf * D * WS_BM;
+    auto load_v = [&](int vc, int b2) {
+      uint16_t* dst = sV + b2 * VK * VS;
+      for (int u = tidc; u < VK * (D / 8); u += NCT) {
+        const int key = u / (D / 8), ch = u % (D / 8);
+        const int gkey = vc * VK + key;
+        uint16_t* dd = dst + key * VS + ch * 8;
+        if (gkey < p.n_k) cp_async16(dd, Vh + (size_t)gkey * D + ch * 8);
+        else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      cp_async_commit();
+    };
+    const int nvc = (it.kv_end + VK - 1) / VK;
+    if (nvc > 0) load_v(0, 0);  // V does not depend on the scores: fetch it while they are made
+    if (nvc > 1) load_v(1, 1);
+    const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
+    if (named_or(BAR_CONS, NCT, !ok)) {
+      ws_timeout(p);
+      cp_async_wait<0>();
+      return;
+    }
+    const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
+                                                          p.emax_sum_limit);
+    float* sQ = qbase + buf * D * WS_BM;
     float* rows = reinterpret_cast<float*>(smem + L.rows) + (size_t)buf * WS_BM * a.nkp;
     float* st = reinterpret_cast<float*>(smem + L.stats) + buf * WS_BM * 2;
     const int written = ((it.kv_end + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
-    const int nch_kv = written >> 5;
 
-    // ---- selection and recompute, rows 2cw and 2cw + 1 together ---------------------
+    // ---- selection and recompute, rows 2cw and 2cw + 1, four keys per lane -----------
+    // Keys past a row's valid range hold -inf: their criterion is NaN, which no
+    // comparison selects, so the hot loops need no validity test.
     int rr_[2], nv[2];
     size_t grow[2];
     float* row[2];
@@ -339,13 +375,13 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
       row[t] = rows + (size_t)rr_[t] * a.nkp;
     }
     const int nvmax = max(nv[0], nv[1]);
+    const int nit = (nvmax + 127) >> 7;
     int list_n = 0;
     auto flush = [&](int cnt) {
       if (lane < cnt) {
         const int e = list[lane];
         const int t = e >> 16, j = e & 0xFFFF;
-        const float y32 = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
-        rows[(size_t)(2 * cw + t) * a.nkp + j] = y32;
+        rows[(size_t)(2 * cw + t) * a.nkp + j] = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
       }
       __syncwarp();
       const int rest = list_n - cnt;
@@ -353,21 +389,24 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
       __syncwarp();
       list_n = rest;
     };
+    if (p.ps_out) {  // dump of the low-precision scores (before any recompute)
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (rr_[t] < it.rows)
+          for (int j = lane; j < p.n_k; j += 32) p.ps_out[grow[t] * p.n_k + j] = j < written ? row[t][j] : -INFINITY;
+    }
     // A: maximum and first argmax of each row
     float m[2] = {-INFINITY, -INFINITY};
     int am[2] = {0x7FFFFFFF, 0x7FFFFFFF};
-    const int nit = (nvmax + 127) >> 7;
     for (int i4 = 0; i4 < nit; ++i4) {
       const int j0 = 128 * i4 + 4 * lane;
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (j0 < written) {
-          const float4 v = *reinterpret_cast<const float4*>(row[t] + j0);
-          if (v.x > m[t]) { m[t] = v.x; am[t] = j0; }
-          if (v.y > m[t]) { m[t] = v.y; am[t] = j0 + 1; }
-          if (v.z > m[t]) { m[t] = v.z; am[t] = j0 + 2; }
-          if (v.w > m[t]) { m[t] = v.w; am[t] = j0 + 3; }
-        }
+        const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+        if (v.x > m[t]) { m[t] = v.x; am[t] = j0; }
+        if (v.y > m[t]) { m[t] = v.y; am[t] = j0 + 1; }
+        if (v.z > m[t]) { m[t] = v.z; am[t] = j0 + 2; }
+        if (v.w > m[t]) { m[t] = v.w; am[t] = j0 + 3; }
       }
     }
 #pragma unroll
@@ -376,142 +415,196 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
       am[t] = warp_min_i(m[t] == mw ? am[t] : 0x7FFFFFFF);
       m[t] = mw;
     }
-    // B: S_rest in double (strict)
+    // B: S_rest = sum_{j != argmax} exp(y_j - m) in double (strict)
     double srest[2] = {0.0, 0.0};
-    if (strict) {
+    if (VAR == LAMP_STRICT) {
       for (int i4 = 0; i4 < nit; ++i4) {
         const int j0 = 128 * i4 + 4 * lane;
-        if (j0 < written) {
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const float4 v = *reinterpret_cast<const float4*>(row[t] + j0);
-            const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float ex = expf(__fsub_rn(vv[e], m[t]));
-              srest[t] += (j0 + e != am[t]) ? (double)ex : 0.0;
-            }
+        for (int t = 0; t < 2; ++t) {
+          float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+          if (j0 == (am[t] & ~3)) {  // the argmax itself is not part of S_rest
+            const int e = am[t] & 3;
+            if (e == 0) v.x = -INFINITY;
+            else if (e == 1) v.y = -INFINITY;
+            else if (e == 2) v.z = -INFINITY;
+            else v.w = -INFINITY;
           }
+          srest[t] += (double)expf(__fsub_rn(v.x, m[t])) + (double)expf(__fsub_rn(v.y, m[t]));
+          srest[t] += (double)expf(__fsub_rn(v.z, m[t])) + (double)expf(__fsub_rn(v.w, m[t]));
         }
       }
 #pragma unroll
       for (int t = 0; t < 2; ++t) srest[t] = warp_sum_d(srest[t]);
     }
     double Sd[2];
-    float Sf[2], srest_f[2], invS2[2], mrun[2] = {-INFINITY, -INFINITY};
-    uint32_t myword[2] = {0u, 0u};
+    float Sf[2], srest_f[2], c2[2], mL[2], lo[2], hi[2], mrun[2] = {-INFINITY, -INFINITY};
+    const float tlo = refine_ok ? p.tau - band : INFINITY;
+    const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       Sd[t] = 1.0 + srest[t];
       Sf[t] = (float)Sd[t];
       srest_f[t] = (float)srest[t];
-      invS2[t] = (float)(1.0 / (Sd[t] * Sd[t]));
+      c2[t] = (float)(2.0 / (Sd[t] * Sd[t]));
+      mL[t] = m[t] * kLog2e;
+      lo[t] = tlo;
+      hi[t] = thi;
     }
     // C: criterion, mask words, compaction of the selected keys
-    const int nch = (nvmax + 31) >> 5;
-    for (int c = 0; c < nch; ++c) {
-      const int j = 32 * c + lane;
-      float y[2];
-      bool sel[2], near[2];
+    for (int i4 = 0; i4 < nit; ++i4) {
+      const int j0 = 128 * i4 + 4 * lane;
+      float y[2][4];
+      uint32_t nib[2] = {0u, 0u}, nearb[2] = {0u, 0u};
+      float mt[2] = {0.f, 0.f};
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        y[t] = row[t][j];
-        const bool valid = j < nv[t];
-        sel[t] = near[t] = false;
-        if (given) {
-          sel[t] = valid && ((__ldg(p.mask_in + grow[t] * nwords + c) >> lane) & 1u);
-        } else {
-          float cr;
-          if (relaxed) {
-            if ((c & 1) == 0) {
-              const float y2 = j + 32 < written ? row[t][j + 32] : -INFINITY;
-              mrun[t] = fmaxf(mrun[t], warp_max(fmaxf(y[t], y2)));
-            }
-            cr = 2.f * fabsf(y[t]) * exp_fast(__fsub_rn(y[t], mrun[t]));
-          } else {
-            const float e = (j == am[t]) ? 1.f : exp_fast(__fsub_rn(y[t], m[t]));
-            const float om = (j == am[t]) ? srest_f[t] : __fsub_rn(Sf[t], e);
-            cr = (2.f * fabsf(y[t]) * e) * (om * invS2[t]);
+        const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+        y[t][0] = v.x; y[t][1] = v.y; y[t][2] = v.z; y[t][3] = v.w;
+        if (VAR == LAMP_GIVEN_MASK) {
+          const int w = j0 >> 5;
+          const uint32_t word = w < nwords ? __ldg(p.mask_in + grow[t] * nwords + w) >> (j0 & 31) : 0u;
+          const int lim = nv[t] - j0;  // keys j0 .. j0 + lim - 1 are valid
+          nib[t] = lim >= 4 ? (word & 15u) : (lim <= 0 ? 0u : (word & ((1u << lim) - 1u)));
+        } else if (VAR == LAMP_RELAXED) {
+          // running maximum over 64-key tiles: lanes 0-15 hold tile 2 i4, lanes 16-31 tile 2 i4 + 1
+          float tm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xFFFFFFFFu, tm, o));
+          const float ma = fmaxf(mrun[t], __shfl_sync(0xFFFFFFFFu, tm, 0));
+          const float mb = fmaxf(ma, __shfl_sync(0xFFFFFFFFu, tm, 16));
+          mt[t] = lane < 16 ? ma : mb;
+          mrun[t] = mb;
+          const float mtL = mt[t] * kLog2e;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float ex;
+            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[t][e], kLog2e, -mtL)));
+            const float cr = 2.f * fabsf(y[t][e]) * ex;
+            nib[t] |= (uint32_t)(cr > p.tau) << e;
+            nearb[t] |= (uint32_t)(cr >= lo[t] && cr <= hi[t]) << e;
           }
-          sel[t] = valid && cr > p.tau;
-          near[t] = valid && refine_ok && (fabsf(cr - p.tau) <= band || (p.tau == 0.f && cr < 1e-30f));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float ex;
+            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[t][e], kLog2e, -mL[t])));
+            const float om = __fsub_rn(Sf[t], ex);
+            const float cr = (fabsf(y[t][e]) * ex) * (om * c2[t]);
+            nib[t] |= (uint32_t)(cr > p.tau) << e;
+            nearb[t] |= (uint32_t)(cr >= lo[t] && cr <= hi[t]) << e;
+          }
+          if (j0 == (am[t] & ~3)) {  // the argmax: z = 1 / S, 1 - z = S_rest / S
+            const int e = am[t] & 3;
+            const float ya = e == 0 ? y[t][0] : (e == 1 ? y[t][1] : (e == 2 ? y[t][2] : y[t][3]));
+            const float cr = fabsf(ya) * (srest_f[t] * c2[t]);
+            nib[t] = (nib[t] & ~(1u << e)) | ((uint32_t)(cr > p.tau) << e);
+            nearb[t] = (nearb[t] & ~(1u << e)) | ((uint32_t)(cr >= lo[t] && cr <= hi[t]) << e);
+          }
         }
       }
-      if (__any_sync(0xFFFFFFFFu, near[0] || near[1])) {
+      if (VAR != LAMP_GIVEN_MASK && __any_sync(0xFFFFFFFFu, (nearb[0] | nearb[1]) != 0u)) {
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (near[t]) {
-            double cd;
-            if (relaxed) {
-              cd = 2.0 * exp((double)y[t] - (double)mrun[t]) * fabs((double)y[t]);
-            } else {
-              const double ed = (j == am[t]) ? 1.0 : exp((double)y[t] - (double)m[t]);
-              const double z = ed / Sd[t];
-              const double omz = (j == am[t]) ? srest[t] / Sd[t] : (Sd[t] - ed) / Sd[t];
-              cd = 2.0 * z * omz * fabs((double)y[t]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if ((nearb[t] >> e) & 1u) {  // re-evaluate in double
+              const int j = j0 + e;
+              const double yd = (double)y[t][e];
+              double cd;
+              if (VAR == LAMP_RELAXED) {
+                cd = 2.0 * exp(yd - (double)mt[t]) * fabs(yd);
+              } else {
+                const double ed = (j == am[t]) ? 1.0 : exp(yd - (double)m[t]);
+                const double z = ed / Sd[t];
+                const double omz = (j == am[t]) ? srest[t] / Sd[t] : (Sd[t] - ed) / Sd[t];
+                cd = 2.0 * z * omz * fabs(yd);
+              }
+              nib[t] = (nib[t] & ~(1u << e)) | ((uint32_t)(cd > (double)p.tau) << e);
             }
-            sel[t] = cd > (double)p.tau;
           }
         }
       }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (p.ps_out && j < p.n_k && rr_[t] < it.rows) p.ps_out[grow[t] * p.n_k + j] = j < nv[t] ? y[t] : -INFINITY;
-        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sel[t]);
-        if ((c & 31) == lane) myword[t] = bal;
-        if (p.mask_out && rr_[t] < it.rows && ((c & 31) == 31 || c == nch - 1)) {
-          const int g0 = c & ~31;
-          if (g0 + lane <= c) p.mask_out[grow[t] * nwords + g0 + lane] = myword[t];
+        // mask word 4 i4 + lane / 8 gathers the nibbles of lanes 8w .. 8w + 7
+        uint32_t x = nib[t] << (4 * (lane & 7));
+        x |= __shfl_xor_sync(0xFFFFFFFFu, x, 1);
+        x |= __shfl_xor_sync(0xFFFFFFFFu, x, 2);
+        x |= __shfl_xor_sync(0xFFFFFFFFu, x, 4);
+        const int w = 4 * i4 + (lane >> 3);
+        if (p.mask_out && rr_[t] < it.rows && (lane & 7) == 0 && w < nwords) p.mask_out[grow[t] * nwords + w] = x;
+      }
+      if (__any_sync(0xFFFFFFFFu, (nib[0] | nib[1]) != 0u)) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool sb = (nib[t] >> e) & 1u;
+            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sb);
+            if (bal) {
+              if (sb) list[list_n + __popc(bal & lanemask_lt)] = (t << 16) | (j0 + e);
+              list_n += __popc(bal);
+              nsel += __popc(bal);
+              __syncwarp();
+              if (list_n >= 32) flush(32);
+            }
+          }
         }
-        nsel += __popc(bal);
-        if (sel[t]) list[list_n + __popc(bal & lanemask_lt)] = (t << 16) | j;
-        list_n += __popc(bal);
-        __syncwarp();
-        if (list_n >= 32) flush(32);
       }
     }
+    if (p.mask_out) {
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (rr_[t] >= it.rows) continue;
-      if (p.mask_out)
-        for (int w = nch + lane; w < nwords; w += 32) p.mask_out[grow[t] * nwords + w] = 0u;
-      if (p.ps_out)
-        for (int j = 32 * nch + lane; j < p.n_k; j += 32) p.ps_out[grow[t] * p.n_k + j] = -INFINITY;
+      for (int t = 0; t < 2; ++t)
+        if (rr_[t] < it.rows)
+          for (int w = 4 * nit + lane; w < nwords; w += 32) p.mask_out[grow[t] * nwords + w] = 0u;
     }
     if (list_n > 0) flush(list_n);
     __syncwarp();
+    if (p.mixed_out) {  // dump of the mixed scores
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (rr_[t] < it.rows)
+          for (int j = lane; j < p.n_k; j += 32)
+            p.mixed_out[grow[t] * p.n_k + j] = j < written ? row[t][j] : -INFINITY;
+    }
 
     // D: softmax numerators of the mixed rows, in place
-    float mm[2] = {-INFINITY, -INFINITY};
-    for (int i4 = 0; i4 < nit; ++i4) {
+    const int nitw = (written + 127) >> 7;
+    float mm[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    for (int i4 = 0; i4 < nitw; ++i4) {
       const int j0 = 128 * i4 + 4 * lane;
-      if (j0 < written) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const float4 v = *reinterpret_cast<const float4*>(row[t] + j0);
-          mm[t] = fmaxf(mm[t], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-        }
-      }
-    }
-    float l[2] = {0.f, 0.f};
-#pragma unroll
-    for (int t = 0; t < 2; ++t) mm[t] = warp_max(mm[t]);
-    for (int c = 0; c < nch_kv; ++c) {
-      const int j = 32 * c + lane;
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        const float yv = row[t][j];
-        const float pj = j < nv[t] ? exp_fast(__fsub_rn(yv, mm[t])) : 0.f;
-        l[t] += pj;
-        if (p.mixed_out && j < p.n_k && rr_[t] < it.rows)
-          p.mixed_out[grow[t] * p.n_k + j] = j < nv[t] ? yv : -INFINITY;
-        reinterpret_cast<uint32_t*>(row[t])[j] = p_pair(pj);
+        const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+        mm[t] = fmaxf(mm[t], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
       }
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      if (p.mixed_out && rr_[t] < it.rows)
-        for (int j = 32 * nch_kv + lane; j < p.n_k; j += 32) p.mixed_out[grow[t] * p.n_k + j] = -INFINITY;
+      mm[t] = warp_max(mm[t]);
+      mL[t] = mm[t] == -INFINITY ? 0.f : mm[t] * kLog2e;
+    }
+    for (int i4 = 0; i4 < nitw; ++i4) {
+      const int j0 = 128 * i4 + 4 * lane;
+      if (j0 >= written) continue;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float4 v = *reinterpret_cast<const float4*>(row[t] + j0);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t pw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float pj;  // exp(y - m'), 0 for -inf
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(pj) : "f"(fmaf(vv[e], kLog2e, -mL[t])));
+          l[t] += pj;
+          pw[e] = p_pair_cvt(pj);
+        }
+        *reinterpret_cast<uint4*>(row[t] + j0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
       l[t] = warp_sum(l[t]);
       if (lane == 0) {
         st[2 * rr_[t]] = mm[t];
@@ -519,7 +612,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         if (p.lse_out && rr_[t] < it.rows) p.lse_out[grow[t]] = nv[t] > 0 ? mm[t] + logf(l[t]) : -INFINITY;
       }
     }
-    bar_sync(BAR_CONS, WS_NC * 32);  // every P row of the item is in place
+    named_sync(BAR_CONS, NCT);  // every P row of the item is in place
 
     // ---- O = (P.V) / l on tensor cores ----------------------------------------------
     const int nh = NH == 2 ? (cw & 1) : 0;
@@ -530,27 +623,10 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     for (int tt = 0; tt < 8; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
-    const int nvc = (it.kv_end + VK - 1) / VK;
-    auto load_v = [&](int vc, int b2) {
-      uint16_t* dst = sV + b2 * VK * VS;
-      for (int u = tidc; u < VK * (D / 8); u += WS_NC * 32) {
-        const int key = u / (D / 8), ch = u % (D / 8);
-        const int gkey = vc * VK + key;
-        uint16_t* dd = dst + key * VS + ch * 8;
-        if (gkey < p.n_k) cp_async16(dd, Vh + (size_t)gkey * D + ch * 8);
-        else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
-      }
-      cp_async_commit();
-    };
-    if (nvc > 0) load_v(0, 0);
     for (int vc = 0; vc < nvc; ++vc) {
-      if (vc + 1 < nvc) {
-        load_v(vc + 1, (vc + 1) & 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      bar_sync(BAR_CONS, WS_NC * 32);
+      if (vc + 1 < nvc) cp_async_wait<1>();
+      else cp_async_wait<0>();
+      named_sync(BAR_CONS, NCT);
       const uint16_t* vb = sV + (vc & 1) * VK * VS;
 #pragma unroll
       for (int qq = 0; qq < SPW; ++qq) {
@@ -570,7 +646,8 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
           }
         }
       }
-      bar_sync(BAR_CONS, WS_NC * 32);
+      named_sync(BAR_CONS, NCT);
+      if (vc + 2 < nvc) load_v(vc + 2, vc & 1);
     }
 #pragma unroll
     for (int rho = 0; rho < KQ; ++rho) {
@@ -591,9 +668,9 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
           }
         }
       }
-      bar_sync(BAR_CONS, WS_NC * 32);
+      named_sync(BAR_CONS, NCT);
     }
-    for (int u = tidc; u < WS_BM * D / 2; u += WS_NC * 32) {
+    for (int u = tidc; u < WS_BM * D / 2; u += NCT) {
       const int rr = u / (D / 2), col = (u % (D / 2)) * 2;
       if (rr >= it.rows) continue;
       const float lv = st[2 * rr + 1];
@@ -605,28 +682,46 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
           (uint32_t)f32_to_bf16_rne(v0) | ((uint32_t)f32_to_bf16_rne(v1) << 16);
       if (p.out_f32) *reinterpret_cast<float2*>(p.out_f32 + off) = make_float2(v0, v1);
     }
-    bar_sync(BAR_CONS, WS_NC * 32);  // sO (the V area) is read before the next item's V loads
-    if (ws_item(k + 2, cta, G, a.n_items) >= 0) bar_arrive(BAR_EMPTY0 + buf, WS_NT);
+    named_sync(BAR_CONS, NCT);  // the output sums (V area) and this item's Q are no longer read
+    const int q2 = ws_item(k + 2, cta, G, a.n_items);
+    if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, a), tidc, NCT);
+    mbar_arrive(bars + 2 + buf);  // buffer free (and Q of item k + 2 staged)
   }
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
 }
 
-template <int D, int RND>
+template <int D, int RND, int VAR>
 __global__ void __launch_bounds__(WS_NT, 1) ws_kernel(const WsArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   const WsSmem L = ws_plan<D>(a.nkp);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+    mbar_init(bars + 0, WS_NP * 32);  // full[0]
+    mbar_init(bars + 1, WS_NP * 32);  // full[1]
+    mbar_init(bars + 2, WS_NC * 32);  // empty[0]
+    mbar_init(bars + 3, WS_NC * 32);  // empty[1]
+    mbar_fence_init();
+  }
+  __syncthreads();
   if (warp < WS_NP) ws_producer<D, RND>(a, smem, L, warp, lane);
-  else ws_consumer<D, RND>(a, smem, L, warp - WS_NP, lane);
+  else ws_consumer<D, RND, VAR>(a, smem, L, warp - WS_NP, lane);
 }
 
-template <int D, int RND>
+template <int D, int RND, int VAR>
 cudaError_t ws_launch_one(const WsArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto k = ws_kernel<D, RND>;
+  auto k = ws_kernel<D, RND, VAR>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, WS_NT, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int RND>
+cudaError_t ws_launch_var(const WsArgs& a, int grid, size_t smem, cudaStream_t st) {
+  if (a.p.variant == LAMP_RELAXED) return ws_launch_one<D, RND, LAMP_RELAXED>(a, grid, smem, st);
+  if (a.p.variant == LAMP_GIVEN_MASK) return ws_launch_one<D, RND, LAMP_GIVEN_MASK>(a, grid, smem, st);
+  return ws_launch_one<D, RND, LAMP_STRICT>(a, grid, smem, st);
 }
 
 }  // namespace
@@ -654,13 +749,13 @@ cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num
   const size_t smem = ws_smem_bytes(p.d, p.n_k);
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
   if (p.d == 64) {
-    if (rnd == kRndFast) return ws_launch_one<64, kRndFast>(a, grid, smem, st);
-    if (rnd == kRndNone) return ws_launch_one<64, kRndNone>(a, grid, smem, st);
-    return ws_launch_one<64, kRndExact>(a, grid, smem, st);
+    if (rnd == kRndFast) return ws_launch_var<64, kRndFast>(a, grid, smem, st);
+    if (rnd == kRndNone) return ws_launch_var<64, kRndNone>(a, grid, smem, st);
+    return ws_launch_var<64, kRndExact>(a, grid, smem, st);
   }
-  if (rnd == kRndFast) return ws_launch_one<128, kRndFast>(a, grid, smem, st);
-  if (rnd == kRndNone) return ws_launch_one<128, kRndNone>(a, grid, smem, st);
-  return ws_launch_one<128, kRndExact>(a, grid, smem, st);
+  if (rnd == kRndFast) return ws_launch_var<128, kRndFast>(a, grid, smem, st);
+  if (rnd == kRndNone) return ws_launch_var<128, kRndNone>(a, grid, smem, st);
+  return ws_launch_var<128, kRndExact>(a, grid, smem, st);
 }
 
 }  // namespace lamp
