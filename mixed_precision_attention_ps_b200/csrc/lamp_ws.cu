@@ -52,12 +52,14 @@ constexpr int BAR_CONS = 1;            // named barrier of the consumer group
 
 template <int D>
 __host__ __device__ constexpr int ws_vkeys() { return D == 64 ? 128 : 64; }
+template <int D>
+__host__ __device__ constexpr int ws_vstages() { return D == 64 ? 3 : 2; }  // V chunks in flight
 
 struct WsSmem {
   int bars;   // mbarriers: full[2], empty[2]
   int q;      // Q [2][D][16] f32
   int ks;     // producer K slices [8 warps][2][8][64] f32
-  int v;      // consumer V chunks [2][VK][D + 8] bf16, later the output sums [16][D] f32
+  int v;      // consumer V chunks [stages][VK][D + 8] bf16, later the partial outputs [KQ][16][D] f32
   int list;   // consumer recompute lists [8][64] int
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
   int rows;   // score rows [2][16][nkp] f32
@@ -71,8 +73,8 @@ __host__ __device__ inline WsSmem ws_plan(int nkp) {
   s.q = 64;
   s.ks = s.q + 2 * D * WS_BM * 4;
   s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
-  const int vb = 2 * ws_vkeys<D>() * (D + 8) * 2;
-  const int ob = WS_BM * D * 4;
+  const int vb = ws_vstages<D>() * ws_vkeys<D>() * (D + 8) * 2;
+  const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;  // per-warp partial outputs
   s.list = s.v + (vb > ob ? vb : ob);
   s.stats = s.list + WS_NC * WS_LIST * 4;
   s.rows = s.stats + 2 * WS_BM * 2 * 4;
@@ -192,8 +194,10 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
     const int first = (warp - deal + WS_NP) % WS_NP;
     const int mine = first < U ? (U - first + WS_NP - 1) / WS_NP : 0;
     const int total = mine * NSL;
-    uint4 kr[2];
-    auto load = [&](int pos) {  // keys lane and lane + 32 of the slice at stream position pos
+    // K slices travel global -> registers -> shared two stream positions ahead of
+    // their use, so an L2 round trip hides behind two slices of arithmetic.
+    uint4 kra[2], krb[2];
+    auto load = [&](int pos, uint4 (&kr)[2]) {  // keys lane and lane + 32 of the slice at pos
       const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -202,7 +206,7 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
         if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
       }
     };
-    auto store = [&](int b2) {
+    auto store = [&](int b2, const uint4 (&kr)[2]) {
       float* dst = ksw + b2 * WS_DS * WS_UNIT + lane;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -214,15 +218,12 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
         }
       }
     };
-    if (total > 0) {
-      load(0);
-      store(0);
-    }
-    __syncwarp();
     u64 acc[4][4];
-    for (int pos = 0; pos < total; ++pos) {
+    // one stream position: compute slice pos, move the slice held in `cur` (loaded
+    // two positions ago) into the free shared buffer, then reuse `cur` for the load
+    // of position pos + 3; two register sets alternate, so no load is waited on early
+    auto body = [&](int pos, uint4 (&cur)[2]) {
       const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
-      if (pos + 1 < total) load(pos + 1);
       if (sl == 0) {
 #pragma unroll
         for (int rp = 0; rp < 4; ++rp)
@@ -256,8 +257,21 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
           *reinterpret_cast<float4*>(rows + (size_t)(r0 + 1) * a.nkp + j0) = y1;
         }
       }
-      if (pos + 1 < total) store((pos + 1) & 1);
+      __syncwarp();  // every lane is done reading slice pos - 1's buffer
+      if (pos + 1 < total) store((pos + 1) & 1, cur);
+      if (pos + 3 < total) load(pos + 3, cur);
       __syncwarp();
+    };
+    if (total > 0) {
+      load(0, kra);
+      store(0, kra);
+    }
+    if (total > 1) load(1, kra);
+    if (total > 2) load(2, krb);
+    __syncwarp();
+    for (int pos = 0; pos < total; pos += 2) {
+      body(pos, kra);
+      if (pos + 1 < total) body(pos + 1, krb);
     }
     deal = (deal + U) % WS_NP;
     mbar_arrive(bars + buf);  // this thread's scores of item k are in place
@@ -305,7 +319,6 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   constexpr int NH = D / 64;
   constexpr int KQ = WS_NC / NH;
   constexpr int SPW = (VK / 8) / KQ;
-  constexpr int TPG = 8 / KQ;
   constexpr int NCT = WS_NC * 32;  // consumer threads
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
@@ -345,9 +358,10 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
       }
       cp_async_commit();
     };
+    constexpr int NST = ws_vstages<D>();
     const int nvc = (it.kv_end + VK - 1) / VK;
-    if (nvc > 0) load_v(0, 0);  // V does not depend on the scores: fetch it while they are made
-    if (nvc > 1) load_v(1, 1);
+    for (int c = 0; c < NST && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
+
     const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
     if (named_or(BAR_CONS, NCT, !ok)) {
       ws_timeout(p);
@@ -536,18 +550,40 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         if (p.mask_out && rr_[t] < it.rows && (lane & 7) == 0 && w < nwords) p.mask_out[grow[t] * nwords + w] = x;
       }
       if (__any_sync(0xFFFFFFFFu, (nib[0] | nib[1]) != 0u)) {
+        // compaction: an exclusive warp scan of the per-lane counts gives every
+        // lane the list slots of its selected keys (order: lane, row, key)
+        const int cnt = __popc(nib[0]) + __popc(nib[1]);
+        int incl = cnt;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        nsel += total;
+        if (list_n + total <= WS_LIST) {
+          int pos = list_n + incl - cnt;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const bool sb = (nib[t] >> e) & 1u;
-            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sb);
-            if (bal) {
-              if (sb) list[list_n + __popc(bal & lanemask_lt)] = (t << 16) | (j0 + e);
-              list_n += __popc(bal);
-              nsel += __popc(bal);
-              __syncwarp();
-              if (list_n >= 32) flush(32);
+          for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if ((nib[t] >> e) & 1u) list[pos++] = (t << 16) | (j0 + e);
+          list_n += total;
+          __syncwarp();
+          while (list_n >= 32) flush(32);
+        } else {  // more than the list holds: append 32-key groups one at a time
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const bool sb = (nib[t] >> e) & 1u;
+              const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sb);
+              if (bal) {
+                if (sb) list[list_n + __popc(bal & lanemask_lt)] = (t << 16) | (j0 + e);
+                list_n += __popc(bal);
+                __syncwarp();
+                if (list_n >= 32) flush(32);
+              }
             }
           }
         }
@@ -624,10 +660,12 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
     for (int vc = 0; vc < nvc; ++vc) {
-      if (vc + 1 < nvc) cp_async_wait<1>();
+      const int pending = min(nvc, vc + NST) - vc - 1;  // chunks issued after this one
+      if (pending >= 2) cp_async_wait<2>();
+      else if (pending == 1) cp_async_wait<1>();
       else cp_async_wait<0>();
       named_sync(BAR_CONS, NCT);
-      const uint16_t* vb = sV + (vc & 1) * VK * VS;
+      const uint16_t* vb = sV + (vc % NST) * VK * VS;
 #pragma unroll
       for (int qq = 0; qq < SPW; ++qq) {
         const int stp = kq + KQ * qq;
@@ -647,35 +685,31 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         }
       }
       named_sync(BAR_CONS, NCT);
-      if (vc + 2 < nvc) load_v(vc + 2, vc & 1);
+      if (vc + NST < nvc) load_v(vc + NST, vc % NST);
     }
+    // each warp's partial sums go to a slot of their own; then one pass adds the KQ
+    // slots of every output in a fixed order (deterministic) and scales by 1 / l
 #pragma unroll
-    for (int rho = 0; rho < KQ; ++rho) {
+    for (int tt = 0; tt < 8; ++tt)
 #pragma unroll
-      for (int tt = 0; tt < 8; ++tt) {
-        if ((tt / TPG - kq - rho + 2 * KQ) % KQ == 0) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int rr = (lane >> 2) + 8 * h;
-            float2* dst = reinterpret_cast<float2*>(sO + rr * D + nh * 64 + 8 * tt + 2 * (lane & 3));
-            const float2 v = make_float2(acc[tt][2 * h], acc[tt][2 * h + 1]);
-            if (rho == 0) {
-              *dst = v;
-            } else {
-              const float2 o = *dst;
-              *dst = make_float2(o.x + v.x, o.y + v.y);
-            }
-          }
-        }
+      for (int h = 0; h < 2; ++h) {
+        const int rr = (lane >> 2) + 8 * h;
+        *reinterpret_cast<float2*>(sO + ((size_t)kq * WS_BM + rr) * D + nh * 64 + 8 * tt + 2 * (lane & 3)) =
+            make_float2(acc[tt][2 * h], acc[tt][2 * h + 1]);
       }
-      named_sync(BAR_CONS, NCT);
-    }
+    named_sync(BAR_CONS, NCT);
     for (int u = tidc; u < WS_BM * D / 2; u += NCT) {
       const int rr = u / (D / 2), col = (u % (D / 2)) * 2;
       if (rr >= it.rows) continue;
+      float2 o = *reinterpret_cast<const float2*>(sO + rr * D + col);
+#pragma unroll
+      for (int g = 1; g < KQ; ++g) {
+        const float2 v = *reinterpret_cast<const float2*>(sO + ((size_t)g * WS_BM + rr) * D + col);
+        o.x += v.x;
+        o.y += v.y;
+      }
       const float lv = st[2 * rr + 1];
       const float inv = lv > 0.f ? 1.f / lv : 0.f;
-      const float2 o = *reinterpret_cast<const float2*>(sO + rr * D + col);
       const float v0 = o.x * inv, v1 = o.y * inv;
       const size_t off = ((size_t)it.bh * p.n_q + it.i0 + rr) * D + col;
       *reinterpret_cast<uint32_t*>(p.out + off) =
