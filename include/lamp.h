@@ -145,6 +145,29 @@ typedef struct {
 
 LAMP_API int lamp_attention_ex(const lamp_args *args);
 
+/*
+ * lamp_attention_noalloc -- lamp_attention_ex for callers that must not allocate
+ * device memory: a program that has handed the device's memory to an allocator
+ * of its own, or one that may allocate only at start-up and not on the path that
+ * computes attention. (The LAMP pages have no counterpart of this entry point; it
+ * is part of this library's interface only.)
+ *   args       as for lamp_attention_ex, except that workspace must be NULL and
+ *              workspace_bytes 0 (LAMP_ERR_ARG otherwise).
+ *   scratch    a fixed array of LAMP_NOALLOC_SCRATCH_BYTES in the memory of every
+ *              GPU that loads the library, held until the process exits. A problem
+ *              that needs more (strict rows too long for shared memory) is rejected
+ *              with LAMP_ERR_WORKSPACE before anything is launched.
+ *   first call on a device: looks up the device address of that array (no
+ *              allocation); make it before capturing a stream into a graph.
+ *   sharing    every call on a device uses the same array, and keeps nothing in it
+ *              from one call to the next (the call clears what must start at zero).
+ *              Calls whose kernels overlap on the GPU (work on two streams without
+ *              an ordering between them) race on the array: order them.
+ * The call makes no cudaMalloc, cudaFree or other allocating CUDA call.
+ */
+#define LAMP_NOALLOC_SCRATCH_BYTES (4u << 20)
+LAMP_API int lamp_attention_noalloc(const lamp_args *args);
+
 /* Bytes of device scratch lamp_attention_ex needs for these shapes and variant
  * (0 when dims is NULL or invalid). The content need not be initialised. */
 LAMP_API size_t lamp_workspace_size(const lamp_dims *dims, int variant);

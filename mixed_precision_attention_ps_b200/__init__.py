@@ -16,12 +16,14 @@ from dataclasses import dataclass
 
 from ._native import (LAMP_ERR_ARG, LAMP_ERR_CHECK, LAMP_ERR_CUDA, LAMP_ERR_TIMEOUT,  # noqa: F401
                       LAMP_ERR_UNSUPPORTED, LAMP_ERR_WORKSPACE, LAMP_GIVEN_MASK, LAMP_MAX_STRICT_NK,
-                      LAMP_OK, LAMP_RELAXED, LAMP_STRICT, LampError, lamp_args, lamp_args_size,
-                      lamp_attention, lamp_attention_ex, lamp_dims, lamp_last_error, lamp_ps_round,
+                      LAMP_NOALLOC_SCRATCH_BYTES, LAMP_OK, LAMP_RELAXED, LAMP_STRICT, LampError, lamp_args,
+                      lamp_args_size, lamp_attention, lamp_attention_ex, lamp_attention_noalloc, lamp_dims,
+                      lamp_last_error, lamp_ps_round,
                       lamp_version, lamp_workspace_size, load, make_args)
 
 __all__ = [
     "LAMP_STRICT", "LAMP_RELAXED", "LAMP_GIVEN_MASK", "LampError", "lamp_attention", "lamp_attention_ex",
+    "lamp_attention_noalloc",
     "lamp_workspace_size", "lamp_last_error", "lamp_ps_round", "lamp_version", "lamp_args_size",
     "attention", "LampOutputs", "load",
 ]

@@ -24,6 +24,7 @@ LAMP_ERR_CUDA = -4
 LAMP_ERR_TIMEOUT = -5
 LAMP_ERR_CHECK = -6
 LAMP_MAX_STRICT_NK = 65536
+LAMP_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 STATUS_NAMES = {
     LAMP_OK: "LAMP_OK", LAMP_ERR_ARG: "LAMP_ERR_ARG", LAMP_ERR_UNSUPPORTED: "LAMP_ERR_UNSUPPORTED",
@@ -80,6 +81,7 @@ SIGNATURES = {
     "lamp_attention": (ctypes.c_int, [ctypes.POINTER(lamp_dims), _P, _P, _P, _P, _P, ctypes.c_int,
                                       ctypes.c_float, ctypes.c_int, ctypes.c_int, _P]),
     "lamp_attention_ex": (ctypes.c_int, [ctypes.POINTER(lamp_args)]),
+    "lamp_attention_noalloc": (ctypes.c_int, [ctypes.POINTER(lamp_args)]),
     "lamp_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(lamp_dims), ctypes.c_int]),
     "lamp_last_error": (ctypes.c_char_p, []),
     "lamp_ps_round": (ctypes.c_int, [_P, _P, ctypes.c_size_t, ctypes.c_int, ctypes.c_int, _P]),
@@ -171,6 +173,15 @@ def lamp_attention_ex(args: lamp_args | None = None, check: bool = True, **kw) -
     if args is None:
         args = make_args(**kw)
     rc = load().lamp_attention_ex(ctypes.byref(args))
+    return _check(rc) if check else rc
+
+
+def lamp_attention_noalloc(args: lamp_args | None = None, check: bool = True, **kw) -> int:
+    """Entry point without device allocation: scratch comes from the library's fixed
+    per-device array (workspace must stay unset)."""
+    if args is None:
+        args = make_args(**kw)
+    rc = load().lamp_attention_noalloc(ctypes.byref(args))
     return _check(rc) if check else rc
 
 

@@ -27,47 +27,57 @@ int ok() {
 }
 
 struct DeviceInfo {
+  int dev = 0;
   int num_sms = 0;
   size_t smem_optin = 0;
-  cudaMemPool_t pool = nullptr;  // scratch pool of this device; keeps its memory between calls
 };
 
 // Per-device attributes, queried once per device.
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
+cudaMemPool_t g_pool[kMaxDevices];  // scratch pool of each device; keeps its memory between calls
+cudaError_t g_pool_err[kMaxDevices];
+std::once_flag g_pool_once[kMaxDevices];
 
 cudaError_t device_info(DeviceInfo& out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  cudaError_t qe = cudaSuccess;
   std::call_once(g_dev_once[dev], [&]() {
     int sms = 0, optin = 0;
-    qe = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (qe == cudaSuccess) qe = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      sms = optin = 0;
+    g_dev[dev].dev = dev;
     g_dev[dev].num_sms = sms;
     g_dev[dev].smem_optin = (size_t)optin;
-    if (qe == cudaSuccess) {
-      cudaMemPoolProps props;
-      std::memset(&props, 0, sizeof(props));
-      props.allocType = cudaMemAllocationTypePinned;
-      props.location.type = cudaMemLocationTypeDevice;
-      props.location.id = dev;
-      cudaMemPool_t pool = nullptr;
-      qe = cudaMemPoolCreate(&pool, &props);
-      if (qe == cudaSuccess) {
-        uint64_t keep = ~0ull;  // never hand freed scratch back to the driver
-        qe = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        g_dev[dev].pool = pool;
-      }
-    }
   });
-  if (qe != cudaSuccess) return qe;
   out = g_dev[dev];
-  if (out.num_sms <= 0 || !out.pool) return cudaErrorInvalidDevice;
+  if (out.num_sms <= 0) return cudaErrorInvalidDevice;
   return cudaSuccess;
+}
+
+// The library's scratch pool of the current device (created on first use).
+cudaError_t scratch_pool(int dev, cudaMemPool_t& pool) {
+  std::call_once(g_pool_once[dev], [&]() {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pl = nullptr;
+    cudaError_t pe = cudaMemPoolCreate(&pl, &props);
+    if (pe == cudaSuccess) {
+      uint64_t keep = ~0ull;  // never hand freed scratch back to the driver
+      pe = cudaMemPoolSetAttribute(pl, cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    g_pool[dev] = pe == cudaSuccess ? pl : nullptr;
+    g_pool_err[dev] = pe;
+  });
+  pool = g_pool[dev];
+  return g_pool_err[dev];
 }
 
 bool aligned(const void* ptr, size_t a) { return ((uintptr_t)ptr % a) == 0; }
@@ -138,6 +148,37 @@ lamp::Problem make_problem(const lamp_args* a) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// The launch sequence of one call: exponent statistics, then the row kernel.
+cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char* base, const DeviceInfo& info,
+                        cudaStream_t st) {
+  cudaError_t e = lamp::launch_prep(p, ws, base, st);
+  if (e != cudaSuccess) return e;
+  if (ws.use_ws) return lamp::launch_ws(p, ws, base, info.num_sms, st);
+  if (ws.rows_bm) return lamp::launch_rows(p, ws, base, info.num_sms, st);
+  return lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
+}
+
+// Scratch of lamp_attention_noalloc: one fixed array in the device memory of
+// every GPU that loads the library, held until the process exits. In host code
+// the name stands for a host-side shadow, not for a device address: kernels get
+// the address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LAMP_NOALLOC_SCRATCH_BYTES];
+char* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+
+// Device address of the scratch array on device dev (the current device),
+// looked up on the first call for that device.
+cudaError_t noalloc_scratch(int dev, char*& ptr) {
+  std::call_once(g_noalloc_once[dev], [&]() {
+    void* addr = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? static_cast<char*>(addr) : nullptr;
+  });
+  ptr = g_noalloc_ptr[dev];
+  return g_noalloc_err[dev];
+}
 
 }  // namespace
 
@@ -211,20 +252,44 @@ int lamp_attention_ex(const lamp_args* a) {
   char* base = static_cast<char*>(a->workspace);
   bool owned = false;
   if (!base) {
-    e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&base), ws.total, info.pool, st);
+    cudaMemPool_t pool = nullptr;
+    e = scratch_pool(info.dev, pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&base), ws.total, pool, st);
     if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "workspace allocation failed: %s", cudaGetErrorString(e));
     owned = true;
   }
-  e = lamp::launch_prep(p, ws, base, st);
-  if (e == cudaSuccess) {
-    if (ws.use_ws) e = lamp::launch_ws(p, ws, base, info.num_sms, st);
-    else if (ws.rows_bm) e = lamp::launch_rows(p, ws, base, info.num_sms, st);
-    else e = lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
-  }
+  e = run_kernels(p, ws, base, info, st);
   if (owned) {
     cudaError_t fe = cudaFreeAsync(base, st);
     if (e == cudaSuccess) e = fe;
   }
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int lamp_attention_noalloc(const lamp_args* a) {
+  int rc = check_args(a);
+  if (rc != LAMP_OK) return rc;
+  if (a->workspace || a->workspace_bytes)
+    return fail(LAMP_ERR_ARG, "lamp_attention_noalloc uses its own scratch: workspace must be NULL and 0");
+  DeviceInfo info;
+  cudaError_t e = device_info(info);
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
+  lamp::Problem p = make_problem(a);
+  lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
+  if (!ws.use_ws && !ws.rows_bm &&
+      lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
+    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
+  if (ws.total > (size_t)LAMP_NOALLOC_SCRATCH_BYTES)
+    return fail(LAMP_ERR_WORKSPACE,
+                "this problem needs %zu bytes of scratch, more than the %u bytes lamp_attention_noalloc "
+                "holds; use lamp_attention_ex",
+                ws.total, (unsigned)LAMP_NOALLOC_SCRATCH_BYTES);
+  char* base = nullptr;
+  e = noalloc_scratch(info.dev, base);
+  if (e != cudaSuccess || !base)
+    return fail(LAMP_ERR_CUDA, "scratch array address unavailable: %s", cudaGetErrorString(e));
+  e = run_kernels(p, ws, base, info, reinterpret_cast<cudaStream_t>(a->stream));
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
   return ok();
 }
