@@ -42,7 +42,8 @@ UNIT = "G-scores/s"
 TAU_FILE = os.path.join(ROOT, "tests", "golden", "tau.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["lamp_ws.cu", "lamp_rows.cu", "lamp_strict.cu", "lamp_prep.cu", "lamp_device.cuh",
+KERNEL_SOURCES = ["lamp_ws.cu", "lamp_ws_common.cuh", "lamp_stream.cu", "lamp_rows.cu", "lamp_strict.cu",
+                  "lamp_prep.cu", "lamp_device.cuh",
                   "lamp_kernels.h"]
 L2_FLUSH_BYTES = 256 << 20
 N_SM = 148

@@ -155,6 +155,7 @@ cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char*
   cudaError_t e = lamp::launch_prep(p, ws, base, st);
   if (e != cudaSuccess) return e;
   if (ws.use_ws) return lamp::launch_ws(p, ws, base, info.num_sms, st);
+  if (ws.use_stream) return lamp::launch_stream(p, ws, base, info.num_sms, st);
   if (ws.rows_bm) return lamp::launch_rows(p, ws, base, info.num_sms, st);
   return lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
 }
@@ -201,8 +202,11 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
   w.spill_rows = 0;
   w.grid = 0;
   w.use_ws = ws_fits(p.d, p.n_k, smem_optin) ? 1 : 0;
-  w.rows_bm = w.use_ws ? 0 : rows_pick_bm(p.d, p.n_k, smem_optin);
-  if (!w.use_ws && !w.rows_bm && strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
+  // the relaxed and given-mask tests need no whole row: rows too long for the
+  // whole-row kernel stream through 512-key tiles instead
+  w.use_stream = (!w.use_ws && p.variant != LAMP_STRICT && stream_smem_bytes(p.d) + kStaticSmemReserve <= smem_optin) ? 1 : 0;
+  w.rows_bm = (w.use_ws || w.use_stream) ? 0 : rows_pick_bm(p.d, p.n_k, smem_optin);
+  if (!w.use_ws && !w.use_stream && !w.rows_bm && strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
     const long long n_items = (long long)((p.n_q + kStrictBM - 1) / kStrictBM) * BH;
     w.grid = (int)(n_items < num_sms ? n_items : num_sms);
     w.spill_rows = 1;
@@ -242,7 +246,7 @@ int lamp_attention_ex(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (!ws.use_ws && !ws.rows_bm &&
+  if (!ws.use_ws && !ws.use_stream && !ws.rows_bm &&
       lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
     return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
   if (a->workspace && a->workspace_bytes < ws.total)
@@ -277,7 +281,7 @@ int lamp_attention_noalloc(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (!ws.use_ws && !ws.rows_bm &&
+  if (!ws.use_ws && !ws.use_stream && !ws.rows_bm &&
       lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
     return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
   if (ws.total > (size_t)LAMP_NOALLOC_SCRATCH_BYTES)

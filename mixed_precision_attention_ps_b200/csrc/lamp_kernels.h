@@ -49,6 +49,7 @@ struct Workspace {
   int nkp;             // padded row length (floats) of the global-slab kernel
   int rows_bm;         // rows per item of the on-chip row kernel; 0 = global-slab kernel
   int use_ws;          // 1: warp-specialised kernel (two 16-row buffers fit on chip)
+  int use_stream;      // 1: streamed one-pass kernel (relaxed / given mask, rows too long for use_ws)
 };
 
 // Strict / given-mask configuration: rows per work item and threads.
@@ -67,6 +68,8 @@ cudaError_t launch_rows(const Problem& p, const Workspace& ws, char* base, int n
 int rows_pick_bm(int d, int n_k, size_t smem_optin);
 cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
 bool ws_fits(int d, int n_k, size_t smem_optin);
+cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
+size_t stream_smem_bytes(int d);
 int rows_nkp(int bm, int n_k);
 size_t rows_smem_bytes(int d, int bm, int n_k);
 cudaError_t launch_ps_round(const float* x, float* y, size_t n, int mu, int path, cudaStream_t st);

@@ -1,0 +1,538 @@
+// LAMP attention, streamed one-pass kernel for the relaxed and given-mask
+// variants at any row length (the 16K-token shape): scores are produced and
+// consumed in tiles of 512 keys with an online softmax, so no complete row is
+// ever stored.
+//
+// Method ("LAMP: Look-Ahead Mixed-Precision Inference of Large Language Models",
+// technical summary, gist.science paper 2601.21623), section "Experimental
+// results": the relaxed relative-threshold test needs no normalising constant,
+// which keeps the softmax one-pass (FlashAttention style); the test here is
+// c_j = 2 exp(y_j - M_t) |y_j| > tau with M_t the running maximum of the
+// low-precision scores over 64-key tiles counted from key 0. Section
+// "Implementation strategy", steps 1-3: low-precision baseline, selection from
+// it, FP32 recompute of the selection before the softmax.
+//
+// Same organisation as the whole-row warp-specialised kernel: one persistent CTA
+// of 512 threads per SM, items (b, h, 16 query rows) in a snake order, producer
+// warps 0-7 fill tile buffers (64-key units dealt round-robin, PS(mu) steps as
+// packed binary32 pairs), consumer warps 8-15 take each tile: the relaxed
+// criterion (double re-evaluation near tau), mask words, warp-compacted FP32
+// recompute from K in global memory, then the online softmax (running maximum m
+// and normaliser l per row; the per-warp partial outputs are rescaled by
+// exp(m_old - m_new) before each tile's P.V on tensor cores). After an item's
+// last tile the partial outputs are added in a fixed order and divided by l.
+// Hand-offs per tile use mbarriers (full[b], empty[b]); every wait is bounded.
+#include <cfloat>
+
+#include "lamp_ws_common.cuh"
+
+namespace lamp {
+namespace {
+
+constexpr int ST_T = 512;   // keys per streamed tile
+constexpr int ST_TS = ST_T + 4;  // tile row stride (floats): 16-byte steps across banks
+
+template <int D>
+__host__ __device__ constexpr int st_vkeys() { return D == 64 ? 128 : 64; }
+constexpr int ST_NST = 3;   // V chunks in flight
+
+struct StSmem {
+  int bars;   // mbarriers: full[2], empty[2]
+  int q;      // Q [2][D][16] f32, by item parity
+  int ks;     // producer K slices [8 warps][2][8][64] f32
+  int v;      // V chunks [3][VK][D + 8] bf16, later the partial outputs [KQ][16][D] f32
+  int list;   // consumer recompute lists [8][64] int
+  int rstat;  // per row: m, l, alpha, spare [16][4] f32
+  int tiles;  // score tiles [2][16][ST_TS] f32
+  int total;
+};
+
+template <int D>
+__host__ __device__ inline StSmem st_plan() {
+  StSmem s{};
+  s.bars = 0;
+  s.q = 64;
+  s.ks = s.q + 2 * D * WS_BM * 4;
+  s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
+  const int vb = ST_NST * st_vkeys<D>() * (D + 8) * 2;
+  const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;
+  s.list = s.v + (vb > ob ? vb : ob);
+  s.rstat = s.list + WS_NC * WS_LIST * 4;
+  s.tiles = s.rstat + WS_BM * 4 * 4;
+  s.total = s.tiles + 2 * WS_BM * ST_TS * 4;
+  return s;
+}
+
+struct StArgs {
+  Problem p;
+  const int* stats;  // per-(b, h) exponent statistics
+  int nchunk;
+  int n_items;
+  int n_rb;
+};
+
+__device__ __forceinline__ int st_ntiles(int kv_end) { return kv_end > 0 ? (kv_end + ST_T - 1) / ST_T : 1; }
+
+// ---------------------------------------------------------------------------
+// Producers: every tile of every item, in the order the consumers take them.
+// ---------------------------------------------------------------------------
+template <int D, int RND>
+__device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem, const StSmem& L, int warp,
+                                            int lane) {
+  const Problem& p = a.p;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int s = 23 - p.mu;
+  const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
+  const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
+  const u64 scale2 = pack2(p.scale, p.scale);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);  // full[0], full[1], empty[0], empty[1]
+  float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
+  int deal = 0;  // producer warp that takes the next unit
+  int k = 0;     // tile counter: buffer k & 1, phase k >> 1
+  for (int ii = 0;; ++ii) {
+    const int q = ws_item(ii, cta, G, a.n_items);
+    if (q < 0) break;
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
+                                                          p.emax_sum_limit);
+    const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
+    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + (ii & 1) * D * WS_BM;
+    const int nt = st_ntiles(it.kv_end);
+    for (int t = 0; t < nt; ++t, ++k) {
+      const int buf = k & 1;
+      const int t0 = t * ST_T;
+      const int tlen = max(0, min(ST_T, it.kv_end - t0));
+      // one decision per warp: the tile routine synchronises the whole warp
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars + 2 + buf, (k >> 1) & 1))) {  // tile buffer free (and the item's Q staged)
+        ws_timeout(p);
+        return;
+      }
+      float* tile = reinterpret_cast<float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
+      ws_produce_tile<D, RND>(p, it, t0, tlen, sQ, tile, ST_TS, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
+                              Kh, negc, pow2s, scale2, s);
+      deal = (deal + (tlen + WS_UNIT - 1) / WS_UNIT) % WS_NP;
+      mbar_arrive(bars + buf);  // this thread's scores of the tile are in place
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Consumers: selection, recompute, online softmax and P.V, tile by tile.
+// ---------------------------------------------------------------------------
+template <int D, int RND, int VAR>
+__device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem, const StSmem& L, int cw,
+                                            int lane) {
+  constexpr int VK = st_vkeys<D>();
+  constexpr int VS = D + 8;
+  constexpr int NH = D / 64;
+  constexpr int KQ = WS_NC / NH;
+  constexpr int SPW = (VK / 8) / KQ;
+  constexpr int NCT = WS_NC * 32;
+  const Problem& p = a.p;
+  const int tidc = cw * 32 + lane;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int nwords = (p.n_k + 31) >> 5;
+  const uint32_t lanemask_lt = (1u << lane) - 1u;
+  const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
+  const float band = WS_BAND * p.tau;
+  const float tlo = refine_ok ? p.tau - band : INFINITY;
+  const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  int* list = reinterpret_cast<int*>(smem + L.list) + cw * WS_LIST;
+  uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L.v);
+  float* sO = reinterpret_cast<float*>(smem + L.v);
+  float* qbase = reinterpret_cast<float*>(smem + L.q);
+  float* rst = reinterpret_cast<float*>(smem + L.rstat);
+  const int nh = NH == 2 ? (cw & 1) : 0;
+  const int kq = NH == 2 ? (cw >> 1) : cw;
+  const int mi = lane >> 3;
+  long long nsel = 0;
+  // Q of the first two items; both tile buffers start out free
+  for (int k0 = 0; k0 < 2; ++k0) {
+    const int q0 = ws_item(k0, cta, G, a.n_items);
+    if (q0 < 0) break;
+    ws_stage_q<D>(qbase + k0 * D * WS_BM, p, ws_decode(q0, p, a.n_rb), tidc, NCT);
+  }
+  mbar_arrive(bars + 2);
+  mbar_arrive(bars + 3);
+  int k = 0;
+  for (int ii = 0;; ++ii) {
+    const int q = ws_item(ii, cta, G, a.n_items);
+    if (q < 0) break;
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
+                                                          p.emax_sum_limit);
+    const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
+    const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
+    float* sQ = qbase + (ii & 1) * D * WS_BM;
+    const int nt = st_ntiles(it.kv_end);
+    int rr_[2], nv[2];
+    size_t grow[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      rr_[t] = 2 * cw + t;
+      nv[t] = rr_[t] < it.rows ? ws_valid_keys(it.i0 + rr_[t], p) : 0;
+      grow[t] = (size_t)it.bh * p.n_q + it.i0 + rr_[t];
+    }
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, mrun[2] = {-INFINITY, -INFINITY};
+    float acc[8][4];
+#pragma unroll
+    for (int tt = 0; tt < 8; ++tt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
+
+    for (int t = 0; t < nt; ++t, ++k) {
+      const int buf = k & 1;
+      const int t0 = t * ST_T;
+      const int tlen = max(0, min(ST_T, it.kv_end - t0));
+      const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
+      float* tile = reinterpret_cast<float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
+      float* row[2] = {tile + (size_t)rr_[0] * ST_TS, tile + (size_t)rr_[1] * ST_TS};
+      auto load_v = [&](int vc, int b2) {
+        uint16_t* dst = sV + b2 * VK * VS;
+        for (int u = tidc; u < VK * (D / 8); u += NCT) {
+          const int key = u / (D / 8), ch = u % (D / 8);
+          const int gkey = t0 + vc * VK + key;
+          uint16_t* dd = dst + key * VS + ch * 8;
+          if (gkey < p.n_k) cp_async16(dd, Vh + (size_t)gkey * D + ch * 8);
+          else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        cp_async_commit();
+      };
+      const int nvc = (tlen + VK - 1) / VK;
+      for (int c = 0; c < ST_NST && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
+      const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
+      if (named_or(BAR_CONS, NCT, !ok)) {
+        ws_timeout(p);
+        cp_async_wait<0>();
+        return;
+      }
+      int nvr[2];
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) nvr[tt] = max(0, min(tlen, nv[tt] - t0));
+      const int nit = (max(nvr[0], nvr[1]) + 127) >> 7;
+      if (p.ps_out) {  // dump of the low-precision scores of this tile
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+          if (rr_[tt] < it.rows)
+            for (int j = lane; j < ST_T && t0 + j < p.n_k; j += 32)
+              p.ps_out[grow[tt] * p.n_k + t0 + j] = j < written ? row[tt][j] : -INFINITY;
+      }
+      int list_n = 0;
+      auto flush = [&](int cnt) {
+        if (lane < cnt) {
+          const int e = list[lane];
+          const int tt = e >> 16, j = e & 0xFFFF;
+          tile[(size_t)(2 * cw + tt) * ST_TS + j] =
+              ws_recompute<D>(sQ, 2 * cw + tt, Kh + (size_t)(t0 + j) * D, p.scale, fast);
+        }
+        __syncwarp();
+        const int rest = list_n - cnt;
+        if (lane < rest) list[lane] = list[cnt + lane];
+        __syncwarp();
+        list_n = rest;
+      };
+      // criterion, mask words, compaction of the selected keys
+      for (int i4 = 0; i4 < nit; ++i4) {
+        const int j0 = 128 * i4 + 4 * lane;  // relative to the tile
+        float y[2][4];
+        uint32_t nib[2] = {0u, 0u}, nearb[2] = {0u, 0u};
+        float mt[2] = {0.f, 0.f};
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const float4 v = lds4_or_ninf(row[tt] + j0, j0 < written);
+          y[tt][0] = v.x; y[tt][1] = v.y; y[tt][2] = v.z; y[tt][3] = v.w;
+          if (VAR == LAMP_GIVEN_MASK) {
+            const int w = (t0 + j0) >> 5;
+            const uint32_t word = w < nwords ? __ldg(p.mask_in + grow[tt] * nwords + w) >> (j0 & 31) : 0u;
+            const int lim = nvr[tt] - j0;
+            nib[tt] = lim >= 4 ? (word & 15u) : (lim <= 0 ? 0u : (word & ((1u << lim) - 1u)));
+          } else {
+            // running maximum over 64-key tiles: lanes 0-15 hold one, lanes 16-31 the next
+            float tm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xFFFFFFFFu, tm, o));
+            const float ma = fmaxf(mrun[tt], __shfl_sync(0xFFFFFFFFu, tm, 0));
+            const float mb = fmaxf(ma, __shfl_sync(0xFFFFFFFFu, tm, 16));
+            mt[tt] = lane < 16 ? ma : mb;
+            mrun[tt] = mb;
+            const float mtL = mt[tt] * kLog2e;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float ex;
+              asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[tt][e], kLog2e, -mtL)));
+              const float cr = 2.f * fabsf(y[tt][e]) * ex;
+              nib[tt] |= (uint32_t)(cr > p.tau) << e;
+              nearb[tt] |= (uint32_t)(cr >= tlo && cr <= thi) << e;
+            }
+          }
+        }
+        if (VAR != LAMP_GIVEN_MASK && __any_sync(0xFFFFFFFFu, (nearb[0] | nearb[1]) != 0u)) {
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if ((nearb[tt] >> e) & 1u) {  // re-evaluate in double
+                const double yd = (double)y[tt][e];
+                const double cd = 2.0 * exp(yd - (double)mt[tt]) * fabs(yd);
+                nib[tt] = (nib[tt] & ~(1u << e)) | ((uint32_t)(cd > (double)p.tau) << e);
+              }
+        }
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          uint32_t x = nib[tt] << (4 * (lane & 7));
+          x |= __shfl_xor_sync(0xFFFFFFFFu, x, 1);
+          x |= __shfl_xor_sync(0xFFFFFFFFu, x, 2);
+          x |= __shfl_xor_sync(0xFFFFFFFFu, x, 4);
+          const int w = (t0 >> 5) + 4 * i4 + (lane >> 3);
+          if (p.mask_out && rr_[tt] < it.rows && (lane & 7) == 0 && w < nwords) p.mask_out[grow[tt] * nwords + w] = x;
+        }
+        if (__any_sync(0xFFFFFFFFu, (nib[0] | nib[1]) != 0u)) {
+          const int cnt = __popc(nib[0]) + __popc(nib[1]);
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+          nsel += total;
+          if (list_n + total <= WS_LIST) {
+            int pos = list_n + incl - cnt;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if ((nib[tt] >> e) & 1u) list[pos++] = (tt << 16) | (j0 + e);
+            list_n += total;
+            __syncwarp();
+            while (list_n >= 32) flush(32);
+          } else {
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const bool sb = (nib[tt] >> e) & 1u;
+                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sb);
+                if (bal) {
+                  if (sb) list[list_n + __popc(bal & lanemask_lt)] = (tt << 16) | (j0 + e);
+                  list_n += __popc(bal);
+                  __syncwarp();
+                  if (list_n >= 32) flush(32);
+                }
+              }
+          }
+        }
+      }
+      if (p.mask_out) {  // the tile's words past the selection loop hold no selected key
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+          if (rr_[tt] < it.rows)
+            for (int w = 4 * nit + lane; w < ST_T / 32 && (t0 >> 5) + w < nwords; w += 32)
+              p.mask_out[grow[tt] * nwords + (t0 >> 5) + w] = 0u;
+      }
+      if (list_n > 0) flush(list_n);
+      __syncwarp();
+      if (p.mixed_out) {  // dump of the mixed scores of this tile
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+          if (rr_[tt] < it.rows)
+            for (int j = lane; j < ST_T && t0 + j < p.n_k; j += 32)
+              p.mixed_out[grow[tt] * p.n_k + t0 + j] = j < written ? row[tt][j] : -INFINITY;
+      }
+      // online softmax: new maximum, rescale factor, numerators of this tile in place
+      const int nitw = (written + 127) >> 7;
+      float tmax[2] = {-INFINITY, -INFINITY}, lt[2] = {0.f, 0.f}, mL[2], alpha[2];
+      for (int i4 = 0; i4 < nitw; ++i4) {
+        const int j0 = 128 * i4 + 4 * lane;
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const float4 v = lds4_or_ninf(row[tt] + j0, j0 < written);
+          tmax[tt] = fmaxf(tmax[tt], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        const float mn = fmaxf(m[tt], warp_max(tmax[tt]));
+        alpha[tt] = mn == -INFINITY ? 1.f : exp_fast(__fsub_rn(m[tt], mn));  // exp(-inf) = 0 on the first tile
+        mL[tt] = mn == -INFINITY ? 0.f : mn * kLog2e;
+        m[tt] = mn;
+      }
+      for (int i4 = 0; i4 < nitw; ++i4) {
+        const int j0 = 128 * i4 + 4 * lane;
+        if (j0 >= written) continue;
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const float4 v = *reinterpret_cast<const float4*>(row[tt] + j0);
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+          uint32_t pw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float pj;  // exp(y - m), 0 for -inf
+            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(pj) : "f"(fmaf(vv[e], kLog2e, -mL[tt])));
+            lt[tt] += pj;
+            pw[e] = p_pair_cvt(pj);
+          }
+          *reinterpret_cast<uint4*>(row[tt] + j0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        l[tt] = l[tt] * alpha[tt] + warp_sum(lt[tt]);
+        if (lane == 0) {
+          rst[4 * rr_[tt]] = m[tt];
+          rst[4 * rr_[tt] + 1] = l[tt];
+          rst[4 * rr_[tt] + 2] = alpha[tt];
+        }
+      }
+      named_sync(BAR_CONS, NCT);  // P of the tile and every row's rescale factor are in place
+
+      // rescale the partial outputs, then add P.V of this tile
+      {
+        const float a0 = rst[4 * (lane >> 2) + 2], a1 = rst[4 * ((lane >> 2) + 8) + 2];
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+          acc[tt][0] *= a0;
+          acc[tt][1] *= a0;
+          acc[tt][2] *= a1;
+          acc[tt][3] *= a1;
+        }
+      }
+      for (int vc = 0; vc < nvc; ++vc) {
+        const int pending = min(nvc, vc + ST_NST) - vc - 1;
+        if (pending >= 2) cp_async_wait<2>();
+        else if (pending == 1) cp_async_wait<1>();
+        else cp_async_wait<0>();
+        named_sync(BAR_CONS, NCT);
+        const uint16_t* vb = sV + (vc % ST_NST) * VK * VS;
+#pragma unroll
+        for (int qq = 0; qq < SPW; ++qq) {
+          const int stp = kq + KQ * qq;
+          const int kb = vc * VK + 8 * stp;  // relative to the tile
+          if (kb < tlen) {
+            uint32_t af[4];
+            const int ra = 8 * (mi & 1) + (lane & 7);
+            ldmatrix_x4(smem_u32(tile + (size_t)ra * ST_TS + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
+            const int kl = 8 * stp + 4 * (mi & 1) + ((lane & 7) >> 1);
+#pragma unroll
+            for (int nb = 0; nb < 4; ++nb) {
+              uint32_t b0, b1, b2, b3;
+              ldmatrix_x4_trans(smem_u32(vb + kl * VS + nh * 64 + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
+              mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
+              mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
+            }
+          }
+        }
+        named_sync(BAR_CONS, NCT);
+        if (vc + ST_NST < nvc) load_v(vc + ST_NST, vc % ST_NST);
+      }
+      if (nvc == 0) named_sync(BAR_CONS, NCT);  // every warp has read the rescale factors
+
+      if (t == nt - 1) {  // end of the item: add the partial outputs, divide by l
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int rr = (lane >> 2) + 8 * h;
+            *reinterpret_cast<float2*>(sO + ((size_t)kq * WS_BM + rr) * D + nh * 64 + 8 * tt + 2 * (lane & 3)) =
+                make_float2(acc[tt][2 * h], acc[tt][2 * h + 1]);
+          }
+        named_sync(BAR_CONS, NCT);
+        for (int u = tidc; u < WS_BM * D / 2; u += NCT) {
+          const int rr = u / (D / 2), col = (u % (D / 2)) * 2;
+          if (rr >= it.rows) continue;
+          float2 o = *reinterpret_cast<const float2*>(sO + rr * D + col);
+#pragma unroll
+          for (int g = 1; g < KQ; ++g) {
+            const float2 v = *reinterpret_cast<const float2*>(sO + ((size_t)g * WS_BM + rr) * D + col);
+            o.x += v.x;
+            o.y += v.y;
+          }
+          const float lv = rst[4 * rr + 1];
+          const float inv = lv > 0.f ? 1.f / lv : 0.f;
+          const float v0 = o.x * inv, v1 = o.y * inv;
+          const size_t off = ((size_t)it.bh * p.n_q + it.i0 + rr) * D + col;
+          *reinterpret_cast<uint32_t*>(p.out + off) =
+              (uint32_t)f32_to_bf16_rne(v0) | ((uint32_t)f32_to_bf16_rne(v1) << 16);
+          if (p.out_f32) *reinterpret_cast<float2*>(p.out_f32 + off) = make_float2(v0, v1);
+        }
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          if (rr_[tt] >= it.rows) continue;
+          if (lane == 0 && p.lse_out) p.lse_out[grow[tt]] = nv[tt] > 0 ? m[tt] + logf(l[tt]) : -INFINITY;
+          const int done = nt * ST_T;  // keys covered by the item's tiles
+          if (p.mask_out)
+            for (int w = (done >> 5) + lane; w < nwords; w += 32) p.mask_out[grow[tt] * nwords + w] = 0u;
+          if (p.ps_out)
+            for (int j = done + lane; j < p.n_k; j += 32) p.ps_out[grow[tt] * p.n_k + j] = -INFINITY;
+          if (p.mixed_out)
+            for (int j = done + lane; j < p.n_k; j += 32) p.mixed_out[grow[tt] * p.n_k + j] = -INFINITY;
+        }
+        named_sync(BAR_CONS, NCT);  // the output sums (V area) and this item's Q are no longer read
+        const int q2 = ws_item(ii + 2, cta, G, a.n_items);
+        if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
+      }
+      mbar_arrive(bars + 2 + buf);  // tile buffer free (and, after an item's last tile, Q of item + 2 staged)
+    }
+  }
+  if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
+}
+
+template <int D, int RND, int VAR>
+__global__ void __launch_bounds__(WS_NP * 32 + WS_NC * 32, 1) st_kernel(const StArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const StSmem L = st_plan<D>();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+    mbar_init(bars + 0, WS_NP * 32);  // full[0]
+    mbar_init(bars + 1, WS_NP * 32);  // full[1]
+    mbar_init(bars + 2, WS_NC * 32);  // empty[0]
+    mbar_init(bars + 3, WS_NC * 32);  // empty[1]
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp < WS_NP) st_producer<D, RND>(a, smem, L, warp, lane);
+  else st_consumer<D, RND, VAR>(a, smem, L, warp - WS_NP, lane);
+}
+
+template <int D, int RND, int VAR>
+cudaError_t st_launch_one(const StArgs& a, int grid, cudaStream_t st) {
+  auto k = st_kernel<D, RND, VAR>;
+  const size_t smem = (size_t)st_plan<D>().total;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, WS_NP * 32 + WS_NC * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int RND>
+cudaError_t st_launch_var(const StArgs& a, int grid, cudaStream_t st) {
+  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK>(a, grid, st);
+  return st_launch_one<D, RND, LAMP_RELAXED>(a, grid, st);
+}
+
+}  // namespace
+
+size_t stream_smem_bytes(int d) { return d == 64 ? (size_t)st_plan<64>().total : (size_t)st_plan<128>().total; }
+
+cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st) {
+  StArgs a;
+  a.p = p;
+  a.stats = reinterpret_cast<const int*>(base + ws.stats);
+  a.nchunk = ws.nchunk;
+  a.n_rb = (p.n_q + WS_BM - 1) / WS_BM;
+  a.n_items = a.n_rb * p.B * p.H;
+  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
+  if (p.d == 64) {
+    if (rnd == kRndFast) return st_launch_var<64, kRndFast>(a, grid, st);
+    if (rnd == kRndNone) return st_launch_var<64, kRndNone>(a, grid, st);
+    return st_launch_var<64, kRndExact>(a, grid, st);
+  }
+  if (rnd == kRndFast) return st_launch_var<128, kRndFast>(a, grid, st);
+  if (rnd == kRndNone) return st_launch_var<128, kRndNone>(a, grid, st);
+  return st_launch_var<128, kRndExact>(a, grid, st);
+}
+
+}  // namespace lamp

@@ -33,22 +33,10 @@
 // caller's status word (when given) and ends the kernel.
 #include <cfloat>
 
-#include "lamp.h"
-#include "lamp_device.cuh"
-#include "lamp_kernels.h"
+#include "lamp_ws_common.cuh"
 
 namespace lamp {
 namespace {
-
-constexpr int WS_BM = 16;              // query rows per item
-constexpr int WS_NT = kWsThreads;      // 512
-constexpr int WS_NP = 8;               // producer warps
-constexpr int WS_NC = 8;               // consumer warps
-constexpr int WS_UNIT = 64;            // keys per producer unit
-constexpr int WS_DS = 8;               // head dimensions per K slice
-constexpr int WS_LIST = 64;            // per-warp recompute list capacity
-constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
-constexpr int BAR_CONS = 1;            // named barrier of the consumer group
 
 template <int D>
 __host__ __device__ constexpr int ws_vkeys() { return D == 64 ? 128 : 64; }
@@ -91,80 +79,12 @@ struct WsArgs {
   int n_rb;
 };
 
-// The k-th item of CTA b (snake order over heaviest-first items), or -1.
-__device__ __forceinline__ int ws_item(int k, int b, int G, int n_items) {
-  const int q = (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
-  return q < n_items ? q : -1;
-}
-
-struct ItemInfo {
-  int bh, i0, rows, kv_end;
-};
-
-__device__ __forceinline__ ItemInfo ws_decode(int q, const WsArgs& a) {
-  const Problem& p = a.p;
-  const int BH = p.B * p.H;
-  ItemInfo it;
-  const int rb = p.causal ? a.n_rb - 1 - q / BH : q / BH;
-  it.bh = q % BH;
-  it.i0 = rb * WS_BM;
-  it.rows = min(WS_BM, p.n_q - it.i0);
-  it.kv_end = p.causal ? min(p.n_k, max(0, it.i0 + it.rows + (p.n_k - p.n_q))) : p.n_k;
-  return it;
-}
-
-__device__ __forceinline__ int ws_valid_keys(int i, const Problem& p) {
-  if (!p.causal) return p.n_k;
-  return min(p.n_k, max(0, i + 1 + (p.n_k - p.n_q)));
-}
-
-__device__ __forceinline__ void ws_timeout(const Problem& p) {
-  if (p.status_out) atomicExch(p.status_out, LAMP_ERR_TIMEOUT);
-}
-
-// Q rows of an item as binary32 [D][16] (rows past the problem are zero).
-template <int D>
-__device__ __forceinline__ void ws_stage_q(float* sQ, const Problem& p, const ItemInfo& it, int t, int nthreads) {
-  for (int u = t; u < WS_BM * D / 8; u += nthreads) {
-    const int r = u / (D / 8), c8 = (u % (D / 8)) * 8;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (r < it.rows) w = __ldg(reinterpret_cast<const uint4*>(p.Q + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8));
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      sQ[(c8 + 2 * e) * WS_BM + r] = bf16_lo(ws[e]);
-      sQ[(c8 + 2 * e + 1) * WS_BM + r] = bf16_hi(ws[e]);
-    }
-  }
-}
-
-// WS_DS accumulation steps of a lane's 8-row x 4-key tile.
-//   qs: Q of this slice, [WS_DS][16] f32 (lane rows 8gr..8gr+7 at qoff = 8gr);
-//   ks: warp's K slice, [WS_DS][64] f32 (lane keys at koff = 4gk).
-template <int MODE>
-__device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, const float* __restrict__ ks, int qoff,
-                                               int koff, u64 (&acc)[4][4], u64 negc, u64 pow2s, int s) {
-#pragma unroll
-  for (int dd = 0; dd < WS_DS; ++dd) {
-    const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff);
-    const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff + 4);
-    const float4 kk = *reinterpret_cast<const float4*>(ks + dd * WS_UNIT + koff);
-    const u64 q[4] = {qa.x, qa.y, qb.x, qb.y};
-    const u64 k[4] = {pack2(kk.x, kk.x), pack2(kk.y, kk.y), pack2(kk.z, kk.z), pack2(kk.w, kk.w)};
-#pragma unroll
-    for (int rp = 0; rp < 4; ++rp)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[rp][i] = ps_step<MODE>(q[rp], k[i], acc[rp][i], negc, pow2s, s);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Producers: PS(mu) scores of every item into the item's row buffer.
 // ---------------------------------------------------------------------------
 template <int D, int RND>
 __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int warp,
                                             int lane) {
-  constexpr int NSL = D / WS_DS;  // K slices per unit
   const Problem& p = a.p;
   const int G = gridDim.x, cta = blockIdx.x;
   const int s = 23 - p.mu;
@@ -173,15 +93,14 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
   const u64 scale2 = pack2(p.scale, p.scale);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);  // full[0], full[1], empty[0], empty[1]
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
-  const int gr = lane & 1, gk = lane >> 1;  // rows 8gr..8gr+7, keys 4gk..4gk+3 of a unit
-  const int qoff = 8 * gr, koff = 4 * gk;
   int deal = 0;  // producer warp that takes the next unit
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
     if (q < 0) break;
     const int buf = k & 1;
-    const ItemInfo it = ws_decode(q, a);
-    if (!mbar_wait(bars + 2 + buf, (k >> 1) & 1)) {  // buffer free, Q staged
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    // one decision per warp: the tile routine synchronises the whole warp
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars + 2 + buf, (k >> 1) & 1))) {  // buffer free, Q staged
       ws_timeout(p);
       return;
     }
@@ -191,121 +110,11 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     float* rows = reinterpret_cast<float*>(smem + L.rows) + (size_t)buf * WS_BM * a.nkp;
     const int U = (it.kv_end + WS_UNIT - 1) / WS_UNIT;
-    const int first = (warp - deal + WS_NP) % WS_NP;
-    const int mine = first < U ? (U - first + WS_NP - 1) / WS_NP : 0;
-    const int total = mine * NSL;
-    // K slices travel global -> registers -> shared two stream positions ahead of
-    // their use, so an L2 round trip hides behind two slices of arithmetic.
-    uint4 kra[2], krb[2];
-    auto load = [&](int pos, uint4 (&kr)[2]) {  // keys lane and lane + 32 of the slice at pos
-      const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int key = j * WS_UNIT + lane + 32 * h;
-        kr[h] = make_uint4(0u, 0u, 0u, 0u);
-        if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
-      }
-    };
-    auto store = [&](int b2, const uint4 (&kr)[2]) {
-      float* dst = ksw + b2 * WS_DS * WS_UNIT + lane;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t ws[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          dst[(2 * e) * WS_UNIT + 32 * h] = bf16_lo(ws[e]);
-          dst[(2 * e + 1) * WS_UNIT + 32 * h] = bf16_hi(ws[e]);
-        }
-      }
-    };
-    u64 acc[4][4];
-    // one stream position: compute slice pos, move the slice held in `cur` (loaded
-    // two positions ago) into the free shared buffer, then reuse `cur` for the load
-    // of position pos + 3; two register sets alternate, so no load is waited on early
-    auto body = [&](int pos, uint4 (&cur)[2]) {
-      const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
-      if (sl == 0) {
-#pragma unroll
-        for (int rp = 0; rp < 4; ++rp)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[rp][i] = 0ull;
-      }
-      const float* qs = sQ + sl * WS_DS * WS_BM;
-      const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
-      if (RND == kRndFast && fast) ws_score_slice<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      else if (RND == kRndNone && fast) ws_score_slice<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      else ws_score_slice<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      if (sl == NSL - 1) {
-        const int j0 = j * WS_UNIT + koff;
-#pragma unroll
-        for (int rp = 0; rp < 4; ++rp) {
-          const int r0 = 8 * gr + 2 * rp;
-          const int nv0 = r0 < it.rows ? ws_valid_keys(it.i0 + r0, p) : 0;
-          const int nv1 = r0 + 1 < it.rows ? ws_valid_keys(it.i0 + r0 + 1, p) : 0;
-          float4 y0, y1;
-          const u64 a0 = mul2u(acc[rp][0], scale2), a1 = mul2u(acc[rp][1], scale2);
-          const u64 a2 = mul2u(acc[rp][2], scale2), a3 = mul2u(acc[rp][3], scale2);
-          y0.x = j0 < nv0 ? lo_f(a0) : -INFINITY;
-          y0.y = j0 + 1 < nv0 ? lo_f(a1) : -INFINITY;
-          y0.z = j0 + 2 < nv0 ? lo_f(a2) : -INFINITY;
-          y0.w = j0 + 3 < nv0 ? lo_f(a3) : -INFINITY;
-          y1.x = j0 < nv1 ? hi_f(a0) : -INFINITY;
-          y1.y = j0 + 1 < nv1 ? hi_f(a1) : -INFINITY;
-          y1.z = j0 + 2 < nv1 ? hi_f(a2) : -INFINITY;
-          y1.w = j0 + 3 < nv1 ? hi_f(a3) : -INFINITY;
-          *reinterpret_cast<float4*>(rows + (size_t)r0 * a.nkp + j0) = y0;
-          *reinterpret_cast<float4*>(rows + (size_t)(r0 + 1) * a.nkp + j0) = y1;
-        }
-      }
-      __syncwarp();  // every lane is done reading slice pos - 1's buffer
-      if (pos + 1 < total) store((pos + 1) & 1, cur);
-      if (pos + 3 < total) load(pos + 3, cur);
-      __syncwarp();
-    };
-    if (total > 0) {
-      load(0, kra);
-      store(0, kra);
-    }
-    if (total > 1) load(1, kra);
-    if (total > 2) load(2, krb);
-    __syncwarp();
-    for (int pos = 0; pos < total; pos += 2) {
-      body(pos, kra);
-      if (pos + 1 < total) body(pos + 1, krb);
-    }
+    ws_produce_tile<D, RND>(p, it, 0, it.kv_end, sQ, rows, a.nkp, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
+                            negc, pow2s, scale2, s);
     deal = (deal + U) % WS_NP;
     mbar_arrive(bars + buf);  // this thread's scores of item k are in place
   }
-}
-
-// FP32 recompute of score (row r, key j): the sequential binary32 sum over
-// k = 0..D-1 (a fused multiply-add when the head's products are exact), then the scale.
-template <int D>
-__device__ __forceinline__ float ws_recompute(const float* __restrict__ sQ, int r, const uint16_t* __restrict__ krow,
-                                              float scale, bool fused) {
-  float acc = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < D; kk += 8) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(krow + kk));
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float k0 = bf16_lo(ws[e]), k1 = bf16_hi(ws[e]);
-      const float q0 = sQ[(kk + 2 * e) * WS_BM + r], q1 = sQ[(kk + 2 * e + 1) * WS_BM + r];
-      if (fused) {
-        acc = __fmaf_rn(q0, k0, acc);
-        acc = __fmaf_rn(q1, k1, acc);
-      } else {
-        acc = __fadd_rn(acc, __fmul_rn(q0, k0));
-        acc = __fadd_rn(acc, __fmul_rn(q1, k1));
-      }
-    }
-  }
-  return __fmul_rn(scale, acc);
-}
-
-__device__ __forceinline__ float4 lds4_or_ninf(const float* ptr, bool ok) {
-  return ok ? *reinterpret_cast<const float4*>(ptr) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
 }
 
 // ---------------------------------------------------------------------------
@@ -337,14 +146,14 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   for (int k0 = 0; k0 < 2; ++k0) {
     const int q0 = ws_item(k0, cta, G, a.n_items);
     if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * D * WS_BM, p, ws_decode(q0, a), tidc, NCT);
+    ws_stage_q<D>(qbase + k0 * D * WS_BM, p, ws_decode(q0, p, a.n_rb), tidc, NCT);
     mbar_arrive(bars + 2 + k0);
   }
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
     if (q < 0) break;
     const int buf = k & 1;
-    const ItemInfo it = ws_decode(q, a);
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
     auto load_v = [&](int vc, int b2) {
@@ -718,7 +527,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     named_sync(BAR_CONS, NCT);  // the output sums (V area) and this item's Q are no longer read
     const int q2 = ws_item(k + 2, cta, G, a.n_items);
-    if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, a), tidc, NCT);
+    if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
     mbar_arrive(bars + 2 + buf);  // buffer free (and Q of item k + 2 staged)
   }
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);

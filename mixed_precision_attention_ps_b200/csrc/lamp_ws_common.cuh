@@ -1,0 +1,219 @@
+// Device pieces shared by the warp-specialised LAMP kernels (whole-row and
+// streamed): work order, Q staging, the producer's score tile and the FP32
+// recompute. Method: "LAMP: Look-Ahead Mixed-Precision Inference of Large
+// Language Models" (technical summary, gist.science paper 2601.21623), sections
+// "Implementation strategy" (steps 1 and 3) and "Experimental results" (PS(mu)).
+#pragma once
+
+#include "lamp.h"
+#include "lamp_device.cuh"
+#include "lamp_kernels.h"
+
+namespace lamp {
+namespace {
+
+constexpr int WS_BM = 16;              // query rows per item
+constexpr int WS_NT = kWsThreads;      // 512
+constexpr int WS_NP = 8;               // producer warps
+constexpr int WS_NC = 8;               // consumer warps
+constexpr int WS_UNIT = 64;            // keys per producer unit
+constexpr int WS_DS = 8;               // head dimensions per K slice
+constexpr int WS_LIST = 64;            // per-warp recompute list capacity
+constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
+constexpr int BAR_CONS = 1;            // named barrier of the consumer group
+
+// The k-th item of CTA b (snake order over heaviest-first items), or -1.
+__device__ __forceinline__ int ws_item(int k, int b, int G, int n_items) {
+  const int q = (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
+  return q < n_items ? q : -1;
+}
+
+struct ItemInfo {
+  int bh, i0, rows, kv_end;
+};
+
+__device__ __forceinline__ ItemInfo ws_decode(int q, const Problem& p, int n_rb) {
+  const int BH = p.B * p.H;
+  ItemInfo it;
+  const int rb = p.causal ? n_rb - 1 - q / BH : q / BH;
+  it.bh = q % BH;
+  it.i0 = rb * WS_BM;
+  it.rows = min(WS_BM, p.n_q - it.i0);
+  it.kv_end = p.causal ? min(p.n_k, max(0, it.i0 + it.rows + (p.n_k - p.n_q))) : p.n_k;
+  return it;
+}
+
+__device__ __forceinline__ int ws_valid_keys(int i, const Problem& p) {
+  if (!p.causal) return p.n_k;
+  return min(p.n_k, max(0, i + 1 + (p.n_k - p.n_q)));
+}
+
+__device__ __forceinline__ void ws_timeout(const Problem& p) {
+  if (p.status_out) atomicExch(p.status_out, LAMP_ERR_TIMEOUT);
+}
+
+// Q rows of an item as binary32 [D][16] (rows past the problem are zero).
+template <int D>
+__device__ __forceinline__ void ws_stage_q(float* sQ, const Problem& p, const ItemInfo& it, int t, int nthreads) {
+  for (int u = t; u < WS_BM * D / 8; u += nthreads) {
+    const int r = u / (D / 8), c8 = (u % (D / 8)) * 8;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (r < it.rows) w = __ldg(reinterpret_cast<const uint4*>(p.Q + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8));
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sQ[(c8 + 2 * e) * WS_BM + r] = bf16_lo(ws[e]);
+      sQ[(c8 + 2 * e + 1) * WS_BM + r] = bf16_hi(ws[e]);
+    }
+  }
+}
+
+// WS_DS accumulation steps of a lane's 8-row x 4-key tile.
+//   qs: Q of this slice, [WS_DS][16] f32 (lane rows 8gr..8gr+7 at qoff = 8gr);
+//   ks: warp's K slice, [WS_DS][64] f32 (lane keys at koff = 4gk).
+template <int MODE>
+__device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, const float* __restrict__ ks, int qoff,
+                                               int koff, u64 (&acc)[4][4], u64 negc, u64 pow2s, int s) {
+#pragma unroll
+  for (int dd = 0; dd < WS_DS; ++dd) {
+    const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff);
+    const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff + 4);
+    const float4 kk = *reinterpret_cast<const float4*>(ks + dd * WS_UNIT + koff);
+    const u64 q[4] = {qa.x, qa.y, qb.x, qb.y};
+    const u64 k[4] = {pack2(kk.x, kk.x), pack2(kk.y, kk.y), pack2(kk.z, kk.z), pack2(kk.w, kk.w)};
+#pragma unroll
+    for (int rp = 0; rp < 4; ++rp)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[rp][i] = ps_step<MODE>(q[rp], k[i], acc[rp][i], negc, pow2s, s);
+  }
+}
+
+// Scores of one tile of an item, keys t0 .. t0 + tlen - 1, by one producer warp:
+// the tile's 64-key units j = first, first + 8, ... (the others belong to the other
+// producer warps). Unit j's scores go to rows[r * stride + 64 j + c] for the 16
+// rows r of the item; keys past a row's valid range hold -inf.
+template <int D, int RND>
+__device__ __forceinline__ void ws_produce_tile(const Problem& p, const ItemInfo& it, int t0, int tlen,
+                                                const float* sQ, float* rows, int stride, float* ksw, int lane,
+                                                int first, bool fast, const uint16_t* Kh, u64 negc, u64 pow2s,
+                                                u64 scale2, int s) {
+  constexpr int NSL = D / WS_DS;  // K slices per unit
+  const int gr = lane & 1, gk = lane >> 1;  // rows 8gr..8gr+7, keys 4gk..4gk+3 of a unit
+  const int qoff = 8 * gr, koff = 4 * gk;
+  const int U = (tlen + WS_UNIT - 1) / WS_UNIT;
+  const int mine = first < U ? (U - first + WS_NP - 1) / WS_NP : 0;
+  const int total = mine * NSL;
+    // K slices travel global -> registers -> shared two stream positions ahead of
+    // their use, so an L2 round trip hides behind two slices of arithmetic.
+    uint4 kra[2], krb[2];
+    auto load = [&](int pos, uint4 (&kr)[2]) {  // keys lane and lane + 32 of the slice at pos
+      const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int key = t0 + j * WS_UNIT + lane + 32 * h;
+        kr[h] = make_uint4(0u, 0u, 0u, 0u);
+        if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
+      }
+    };
+    auto store = [&](int b2, const uint4 (&kr)[2]) {
+      float* dst = ksw + b2 * WS_DS * WS_UNIT + lane;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t ws[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dst[(2 * e) * WS_UNIT + 32 * h] = bf16_lo(ws[e]);
+          dst[(2 * e + 1) * WS_UNIT + 32 * h] = bf16_hi(ws[e]);
+        }
+      }
+    };
+    u64 acc[4][4];
+    // one stream position: compute slice pos, move the slice held in `cur` (loaded
+    // two positions ago) into the free shared buffer, then reuse `cur` for the load
+    // of position pos + 3; two register sets alternate, so no load is waited on early
+    auto body = [&](int pos, uint4 (&cur)[2]) {
+      const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
+      if (sl == 0) {
+#pragma unroll
+        for (int rp = 0; rp < 4; ++rp)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[rp][i] = 0ull;
+      }
+      const float* qs = sQ + sl * WS_DS * WS_BM;
+      const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
+      if (RND == kRndFast && fast) ws_score_slice<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+      else if (RND == kRndNone && fast) ws_score_slice<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+      else ws_score_slice<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+      if (sl == NSL - 1) {
+        const int j0 = t0 + j * WS_UNIT + koff;  // absolute key of the lane's first column
+        float* dst = rows + j * WS_UNIT + koff;
+#pragma unroll
+        for (int rp = 0; rp < 4; ++rp) {
+          const int r0 = 8 * gr + 2 * rp;
+          const int nv0 = r0 < it.rows ? ws_valid_keys(it.i0 + r0, p) : 0;
+          const int nv1 = r0 + 1 < it.rows ? ws_valid_keys(it.i0 + r0 + 1, p) : 0;
+          float4 y0, y1;
+          const u64 a0 = mul2u(acc[rp][0], scale2), a1 = mul2u(acc[rp][1], scale2);
+          const u64 a2 = mul2u(acc[rp][2], scale2), a3 = mul2u(acc[rp][3], scale2);
+          y0.x = j0 < nv0 ? lo_f(a0) : -INFINITY;
+          y0.y = j0 + 1 < nv0 ? lo_f(a1) : -INFINITY;
+          y0.z = j0 + 2 < nv0 ? lo_f(a2) : -INFINITY;
+          y0.w = j0 + 3 < nv0 ? lo_f(a3) : -INFINITY;
+          y1.x = j0 < nv1 ? hi_f(a0) : -INFINITY;
+          y1.y = j0 + 1 < nv1 ? hi_f(a1) : -INFINITY;
+          y1.z = j0 + 2 < nv1 ? hi_f(a2) : -INFINITY;
+          y1.w = j0 + 3 < nv1 ? hi_f(a3) : -INFINITY;
+          *reinterpret_cast<float4*>(dst + (size_t)r0 * stride) = y0;
+          *reinterpret_cast<float4*>(dst + (size_t)(r0 + 1) * stride) = y1;
+        }
+      }
+      __syncwarp();  // every lane is done reading slice pos - 1's buffer
+      if (pos + 1 < total) store((pos + 1) & 1, cur);
+      if (pos + 3 < total) load(pos + 3, cur);
+      __syncwarp();
+    };
+    if (total > 0) {
+      load(0, kra);
+      store(0, kra);
+    }
+    if (total > 1) load(1, kra);
+    if (total > 2) load(2, krb);
+    __syncwarp();
+    for (int pos = 0; pos < total; pos += 2) {
+      body(pos, kra);
+      if (pos + 1 < total) body(pos + 1, krb);
+    }
+}
+
+// FP32 recompute of score (row r, key j): the sequential binary32 sum over
+// k = 0..D-1 (a fused multiply-add when the head's products are exact), then the scale.
+template <int D>
+__device__ __forceinline__ float ws_recompute(const float* __restrict__ sQ, int r, const uint16_t* __restrict__ krow,
+                                              float scale, bool fused) {
+  float acc = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D; kk += 8) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(krow + kk));
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float k0 = bf16_lo(ws[e]), k1 = bf16_hi(ws[e]);
+      const float q0 = sQ[(kk + 2 * e) * WS_BM + r], q1 = sQ[(kk + 2 * e + 1) * WS_BM + r];
+      if (fused) {
+        acc = __fmaf_rn(q0, k0, acc);
+        acc = __fmaf_rn(q1, k1, acc);
+      } else {
+        acc = __fadd_rn(acc, __fmul_rn(q0, k0));
+        acc = __fadd_rn(acc, __fmul_rn(q1, k1));
+      }
+    }
+  }
+  return __fmul_rn(scale, acc);
+}
+
+__device__ __forceinline__ float4 lds4_or_ninf(const float* ptr, bool ok) {
+  return ok ? *reinterpret_cast<const float4*>(ptr) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+}
+
+}  // namespace
+}  // namespace lamp
