@@ -52,7 +52,7 @@ __host__ __device__ inline StSmem st_plan() {
   StSmem s{};
   s.bars = 0;
   s.q = 64;
-  s.ks = s.q + 2 * D * WS_BM * 4;
+  s.ks = s.q + 2 * ws_qfloats<D>() * 4;
   s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
   const int vb = ST_NST * st_vkeys<D>() * (D + 8) * 2;
   const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;
@@ -96,7 +96,7 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
-    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + (ii & 1) * D * WS_BM;
+    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + (ii & 1) * ws_qfloats<D>();
     const int nt = st_ntiles(it.kv_end);
     for (int t = 0; t < nt; ++t, ++k) {
       const int buf = k & 1;
@@ -151,7 +151,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   for (int k0 = 0; k0 < 2; ++k0) {
     const int q0 = ws_item(k0, cta, G, a.n_items);
     if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * D * WS_BM, p, ws_decode(q0, p, a.n_rb), tidc, NCT);
+    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), tidc, NCT);
   }
   mbar_arrive(bars + 2);
   mbar_arrive(bars + 3);
@@ -164,7 +164,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
-    float* sQ = qbase + (ii & 1) * D * WS_BM;
+    float* sQ = qbase + (ii & 1) * ws_qfloats<D>();
     const int nt = st_ntiles(it.kv_end);
     int rr_[2], nv[2];
     size_t grow[2];
@@ -174,7 +174,13 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
       nv[t] = rr_[t] < it.rows ? ws_valid_keys(it.i0 + rr_[t], p) : 0;
       grow[t] = (size_t)it.bh * p.n_q + it.i0 + rr_[t];
     }
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, mrun[2] = {-INFINITY, -INFINITY};
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    SelRows S;
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      S.live[tt] = rr_[tt] < it.rows;
+      S.mrun[tt] = -INFINITY;
+    }
     float acc[8][4];
 #pragma unroll
     for (int tt = 0; tt < 8; ++tt)
@@ -223,8 +229,10 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         if (lane < cnt) {
           const int e = list[lane];
           const int tt = e >> 16, j = e & 0xFFFF;
-          tile[(size_t)(2 * cw + tt) * ST_TS + j] =
-              ws_recompute<D>(sQ, 2 * cw + tt, Kh + (size_t)(t0 + j) * D, p.scale, fast);
+          const float v = ws_recompute<D>(sQ, 2 * cw + tt, Kh + (size_t)(t0 + j) * D, p.scale, fast);
+          tile[(size_t)(2 * cw + tt) * ST_TS + j] = v;
+          if (tt == 0) S.mx[0] = fmaxf(S.mx[0], v);
+          else S.mx[1] = fmaxf(S.mx[1], v);
         }
         __syncwarp();
         const int rest = list_n - cnt;
@@ -232,98 +240,17 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         __syncwarp();
         list_n = rest;
       };
-      // criterion, mask words, compaction of the selected keys
-      for (int i4 = 0; i4 < nit; ++i4) {
-        const int j0 = 128 * i4 + 4 * lane;  // relative to the tile
-        float y[2][4];
-        uint32_t nib[2] = {0u, 0u}, nearb[2] = {0u, 0u};
-        float mt[2] = {0.f, 0.f};
+      // criterion, mask words, compaction and recompute of the selected keys
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const float4 v = lds4_or_ninf(row[tt] + j0, j0 < written);
-          y[tt][0] = v.x; y[tt][1] = v.y; y[tt][2] = v.z; y[tt][3] = v.w;
-          if (VAR == LAMP_GIVEN_MASK) {
-            const int w = (t0 + j0) >> 5;
-            const uint32_t word = w < nwords ? __ldg(p.mask_in + grow[tt] * nwords + w) >> (j0 & 31) : 0u;
-            const int lim = nvr[tt] - j0;
-            nib[tt] = lim >= 4 ? (word & 15u) : (lim <= 0 ? 0u : (word & ((1u << lim) - 1u)));
-          } else {
-            // running maximum over 64-key tiles: lanes 0-15 hold one, lanes 16-31 the next
-            float tm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xFFFFFFFFu, tm, o));
-            const float ma = fmaxf(mrun[tt], __shfl_sync(0xFFFFFFFFu, tm, 0));
-            const float mb = fmaxf(ma, __shfl_sync(0xFFFFFFFFu, tm, 16));
-            mt[tt] = lane < 16 ? ma : mb;
-            mrun[tt] = mb;
-            const float mtL = mt[tt] * kLog2e;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float ex;
-              asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[tt][e], kLog2e, -mtL)));
-              const float cr = 2.f * fabsf(y[tt][e]) * ex;
-              nib[tt] |= (uint32_t)(cr > p.tau) << e;
-              nearb[tt] |= (uint32_t)(cr >= tlo && cr <= thi) << e;
-            }
-          }
-        }
-        if (VAR != LAMP_GIVEN_MASK && __any_sync(0xFFFFFFFFu, (nearb[0] | nearb[1]) != 0u)) {
-#pragma unroll
-          for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if ((nearb[tt] >> e) & 1u) {  // re-evaluate in double
-                const double yd = (double)y[tt][e];
-                const double cd = 2.0 * exp(yd - (double)mt[tt]) * fabs(yd);
-                nib[tt] = (nib[tt] & ~(1u << e)) | ((uint32_t)(cd > (double)p.tau) << e);
-              }
-        }
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          uint32_t x = nib[tt] << (4 * (lane & 7));
-          x |= __shfl_xor_sync(0xFFFFFFFFu, x, 1);
-          x |= __shfl_xor_sync(0xFFFFFFFFu, x, 2);
-          x |= __shfl_xor_sync(0xFFFFFFFFu, x, 4);
-          const int w = (t0 >> 5) + 4 * i4 + (lane >> 3);
-          if (p.mask_out && rr_[tt] < it.rows && (lane & 7) == 0 && w < nwords) p.mask_out[grow[tt] * nwords + w] = x;
-        }
-        if (__any_sync(0xFFFFFFFFu, (nib[0] | nib[1]) != 0u)) {
-          const int cnt = __popc(nib[0]) + __popc(nib[1]);
-          int incl = cnt;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += v;
-          }
-          const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-          nsel += total;
-          if (list_n + total <= WS_LIST) {
-            int pos = list_n + incl - cnt;
-#pragma unroll
-            for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if ((nib[tt] >> e) & 1u) list[pos++] = (tt << 16) | (j0 + e);
-            list_n += total;
-            __syncwarp();
-            while (list_n >= 32) flush(32);
-          } else {
-#pragma unroll
-            for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const bool sb = (nib[tt] >> e) & 1u;
-                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sb);
-                if (bal) {
-                  if (sb) list[list_n + __popc(bal & lanemask_lt)] = (tt << 16) | (j0 + e);
-                  list_n += __popc(bal);
-                  __syncwarp();
-                  if (list_n >= 32) flush(32);
-                }
-              }
-          }
-        }
+      for (int tt = 0; tt < 2; ++tt) {
+        S.row[tt] = row[tt];
+        S.nv[tt] = nvr[tt];
+        S.word0[tt] = grow[tt] * nwords + (t0 >> 5);
+        S.mx[tt] = -INFINITY;
       }
+      for (int i4 = 0; i4 < nit; ++i4)
+        sel_step<VAR>(p, S, 128 * i4, written, nwords - (t0 >> 5), tlo, thi, lane, lanemask_lt, list, list_n, nsel,
+                      flush);
       if (p.mask_out) {  // the tile's words past the selection loop hold no selected key
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt)
@@ -331,6 +258,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
             for (int w = 4 * nit + lane; w < ST_T / 32 && (t0 >> 5) + w < nwords; w += 32)
               p.mask_out[grow[tt] * nwords + (t0 >> 5) + w] = 0u;
       }
+      __syncwarp();
       if (list_n > 0) flush(list_n);
       __syncwarp();
       if (p.mixed_out) {  // dump of the mixed scores of this tile
@@ -342,18 +270,10 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
       }
       // online softmax: new maximum, rescale factor, numerators of this tile in place
       const int nitw = (written + 127) >> 7;
-      float tmax[2] = {-INFINITY, -INFINITY}, lt[2] = {0.f, 0.f}, mL[2], alpha[2];
-      for (int i4 = 0; i4 < nitw; ++i4) {
-        const int j0 = 128 * i4 + 4 * lane;
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const float4 v = lds4_or_ninf(row[tt] + j0, j0 < written);
-          tmax[tt] = fmaxf(tmax[tt], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-        }
-      }
+      float lt[2] = {0.f, 0.f}, mL[2], alpha[2];
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
-        const float mn = fmaxf(m[tt], warp_max(tmax[tt]));
+        const float mn = fmaxf(m[tt], warp_max_redux(S.mx[tt]));
         alpha[tt] = mn == -INFINITY ? 1.f : exp_fast(__fsub_rn(m[tt], mn));  // exp(-inf) = 0 on the first tile
         mL[tt] = mn == -INFINITY ? 0.f : mn * kLog2e;
         m[tt] = mn;

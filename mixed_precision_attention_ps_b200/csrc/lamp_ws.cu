@@ -59,7 +59,7 @@ __host__ __device__ inline WsSmem ws_plan(int nkp) {
   WsSmem s{};
   s.bars = 0;
   s.q = 64;
-  s.ks = s.q + 2 * D * WS_BM * 4;
+  s.ks = s.q + 2 * ws_qfloats<D>() * 4;
   s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
   const int vb = ws_vstages<D>() * ws_vkeys<D>() * (D + 8) * 2;
   const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;  // per-warp partial outputs
@@ -104,7 +104,7 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
       ws_timeout(p);
       return;
     }
-    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + buf * D * WS_BM;
+    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + buf * ws_qfloats<D>();
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
@@ -146,7 +146,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   for (int k0 = 0; k0 < 2; ++k0) {
     const int q0 = ws_item(k0, cta, G, a.n_items);
     if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * D * WS_BM, p, ws_decode(q0, p, a.n_rb), tidc, NCT);
+    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), tidc, NCT);
     mbar_arrive(bars + 2 + k0);
   }
   for (int k = 0;; ++k) {
@@ -179,23 +179,30 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
-    float* sQ = qbase + buf * D * WS_BM;
+    float* sQ = qbase + buf * ws_qfloats<D>();
     float* rows = reinterpret_cast<float*>(smem + L.rows) + (size_t)buf * WS_BM * a.nkp;
     float* st = reinterpret_cast<float*>(smem + L.stats) + buf * WS_BM * 2;
     const int written = ((it.kv_end + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
 
-    // ---- selection and recompute, rows 2cw and 2cw + 1, four keys per lane -----------
+    // ---- selection and recompute, rows 2cw and 2cw + 1 ------------------------------
     // Keys past a row's valid range hold -inf: their criterion is NaN, which no
     // comparison selects, so the hot loops need no validity test.
     int rr_[2], nv[2];
     size_t grow[2];
     float* row[2];
+    SelRows S;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       rr_[t] = 2 * cw + t;
       nv[t] = rr_[t] < it.rows ? ws_valid_keys(it.i0 + rr_[t], p) : 0;
       grow[t] = (size_t)it.bh * p.n_q + it.i0 + rr_[t];
       row[t] = rows + (size_t)rr_[t] * a.nkp;
+      S.row[t] = row[t];
+      S.nv[t] = nv[t];
+      S.word0[t] = grow[t] * nwords;
+      S.live[t] = rr_[t] < it.rows;
+      S.mx[t] = -INFINITY;
+      S.mrun[t] = -INFINITY;
     }
     const int nvmax = max(nv[0], nv[1]);
     const int nit = (nvmax + 127) >> 7;
@@ -204,7 +211,10 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
       if (lane < cnt) {
         const int e = list[lane];
         const int t = e >> 16, j = e & 0xFFFF;
-        rows[(size_t)(2 * cw + t) * a.nkp + j] = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
+        const float v = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
+        rows[(size_t)(2 * cw + t) * a.nkp + j] = v;
+        if (t == 0) S.mx[0] = fmaxf(S.mx[0], v);
+        else S.mx[1] = fmaxf(S.mx[1], v);
       }
       __syncwarp();
       const int rest = list_n - cnt;
@@ -218,29 +228,29 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         if (rr_[t] < it.rows)
           for (int j = lane; j < p.n_k; j += 32) p.ps_out[grow[t] * p.n_k + j] = j < written ? row[t][j] : -INFINITY;
     }
-    // A: maximum and first argmax of each row
-    float m[2] = {-INFINITY, -INFINITY};
-    int am[2] = {0x7FFFFFFF, 0x7FFFFFFF};
-    for (int i4 = 0; i4 < nit; ++i4) {
-      const int j0 = 128 * i4 + 4 * lane;
+    if (VAR == LAMP_STRICT) {
+      // A: maximum and first argmax of each row
+      float m[2] = {-INFINITY, -INFINITY};
+      int am[2] = {0x7FFFFFFF, 0x7FFFFFFF};
+      for (int i4 = 0; i4 < nit; ++i4) {
+        const int j0 = 128 * i4 + 4 * lane;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+          if (v.x > m[t]) { m[t] = v.x; am[t] = j0; }
+          if (v.y > m[t]) { m[t] = v.y; am[t] = j0 + 1; }
+          if (v.z > m[t]) { m[t] = v.z; am[t] = j0 + 2; }
+          if (v.w > m[t]) { m[t] = v.w; am[t] = j0 + 3; }
+        }
+      }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
-        if (v.x > m[t]) { m[t] = v.x; am[t] = j0; }
-        if (v.y > m[t]) { m[t] = v.y; am[t] = j0 + 1; }
-        if (v.z > m[t]) { m[t] = v.z; am[t] = j0 + 2; }
-        if (v.w > m[t]) { m[t] = v.w; am[t] = j0 + 3; }
+        const float mw = warp_max_redux(m[t]);
+        am[t] = __reduce_min_sync(0xFFFFFFFFu, m[t] == mw ? am[t] : 0x7FFFFFFF);
+        m[t] = mw;
       }
-    }
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const float mw = warp_max(m[t]);
-      am[t] = warp_min_i(m[t] == mw ? am[t] : 0x7FFFFFFF);
-      m[t] = mw;
-    }
-    // B: S_rest = sum_{j != argmax} exp(y_j - m) in double (strict)
-    double srest[2] = {0.0, 0.0};
-    if (VAR == LAMP_STRICT) {
+      // B: S_rest = sum_{j != argmax} exp(y_j - m) in double, two chains per row
+      double sa[2] = {0.0, 0.0}, sb[2] = {0.0, 0.0};
       for (int i4 = 0; i4 < nit; ++i4) {
         const int j0 = 128 * i4 + 4 * lane;
 #pragma unroll
@@ -253,157 +263,35 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
             else if (e == 2) v.z = -INFINITY;
             else v.w = -INFINITY;
           }
-          srest[t] += (double)expf(__fsub_rn(v.x, m[t])) + (double)expf(__fsub_rn(v.y, m[t]));
-          srest[t] += (double)expf(__fsub_rn(v.z, m[t])) + (double)expf(__fsub_rn(v.w, m[t]));
+          sa[t] += (double)expf(__fsub_rn(v.x, m[t])) + (double)expf(__fsub_rn(v.y, m[t]));
+          sb[t] += (double)expf(__fsub_rn(v.z, m[t])) + (double)expf(__fsub_rn(v.w, m[t]));
         }
       }
 #pragma unroll
-      for (int t = 0; t < 2; ++t) srest[t] = warp_sum_d(srest[t]);
+      for (int t = 0; t < 2; ++t) {
+        const double srest = warp_sum_d(sa[t] + sb[t]);
+        S.m[t] = m[t];
+        S.am[t] = am[t];
+        S.srest[t] = srest;
+        S.Sd[t] = 1.0 + srest;
+        S.Sf[t] = (float)S.Sd[t];
+        S.srest_f[t] = (float)srest;
+        S.c2[t] = (float)(2.0 / (S.Sd[t] * S.Sd[t]));
+        S.mL[t] = m[t] * kLog2e;
+      }
     }
-    double Sd[2];
-    float Sf[2], srest_f[2], c2[2], mL[2], lo[2], hi[2], mrun[2] = {-INFINITY, -INFINITY};
+    // C: criterion, mask words, compaction and recompute of the selected keys
     const float tlo = refine_ok ? p.tau - band : INFINITY;
     const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      Sd[t] = 1.0 + srest[t];
-      Sf[t] = (float)Sd[t];
-      srest_f[t] = (float)srest[t];
-      c2[t] = (float)(2.0 / (Sd[t] * Sd[t]));
-      mL[t] = m[t] * kLog2e;
-      lo[t] = tlo;
-      hi[t] = thi;
-    }
-    // C: criterion, mask words, compaction of the selected keys
-    for (int i4 = 0; i4 < nit; ++i4) {
-      const int j0 = 128 * i4 + 4 * lane;
-      float y[2][4];
-      uint32_t nib[2] = {0u, 0u}, nearb[2] = {0u, 0u};
-      float mt[2] = {0.f, 0.f};
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
-        y[t][0] = v.x; y[t][1] = v.y; y[t][2] = v.z; y[t][3] = v.w;
-        if (VAR == LAMP_GIVEN_MASK) {
-          const int w = j0 >> 5;
-          const uint32_t word = w < nwords ? __ldg(p.mask_in + grow[t] * nwords + w) >> (j0 & 31) : 0u;
-          const int lim = nv[t] - j0;  // keys j0 .. j0 + lim - 1 are valid
-          nib[t] = lim >= 4 ? (word & 15u) : (lim <= 0 ? 0u : (word & ((1u << lim) - 1u)));
-        } else if (VAR == LAMP_RELAXED) {
-          // running maximum over 64-key tiles: lanes 0-15 hold tile 2 i4, lanes 16-31 tile 2 i4 + 1
-          float tm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xFFFFFFFFu, tm, o));
-          const float ma = fmaxf(mrun[t], __shfl_sync(0xFFFFFFFFu, tm, 0));
-          const float mb = fmaxf(ma, __shfl_sync(0xFFFFFFFFu, tm, 16));
-          mt[t] = lane < 16 ? ma : mb;
-          mrun[t] = mb;
-          const float mtL = mt[t] * kLog2e;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float ex;
-            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[t][e], kLog2e, -mtL)));
-            const float cr = 2.f * fabsf(y[t][e]) * ex;
-            nib[t] |= (uint32_t)(cr > p.tau) << e;
-            nearb[t] |= (uint32_t)(cr >= lo[t] && cr <= hi[t]) << e;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float ex;
-            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[t][e], kLog2e, -mL[t])));
-            const float om = __fsub_rn(Sf[t], ex);
-            const float cr = (fabsf(y[t][e]) * ex) * (om * c2[t]);
-            nib[t] |= (uint32_t)(cr > p.tau) << e;
-            nearb[t] |= (uint32_t)(cr >= lo[t] && cr <= hi[t]) << e;
-          }
-          if (j0 == (am[t] & ~3)) {  // the argmax: z = 1 / S, 1 - z = S_rest / S
-            const int e = am[t] & 3;
-            const float ya = e == 0 ? y[t][0] : (e == 1 ? y[t][1] : (e == 2 ? y[t][2] : y[t][3]));
-            const float cr = fabsf(ya) * (srest_f[t] * c2[t]);
-            nib[t] = (nib[t] & ~(1u << e)) | ((uint32_t)(cr > p.tau) << e);
-            nearb[t] = (nearb[t] & ~(1u << e)) | ((uint32_t)(cr >= lo[t] && cr <= hi[t]) << e);
-          }
-        }
-      }
-      if (VAR != LAMP_GIVEN_MASK && __any_sync(0xFFFFFFFFu, (nearb[0] | nearb[1]) != 0u)) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((nearb[t] >> e) & 1u) {  // re-evaluate in double
-              const int j = j0 + e;
-              const double yd = (double)y[t][e];
-              double cd;
-              if (VAR == LAMP_RELAXED) {
-                cd = 2.0 * exp(yd - (double)mt[t]) * fabs(yd);
-              } else {
-                const double ed = (j == am[t]) ? 1.0 : exp(yd - (double)m[t]);
-                const double z = ed / Sd[t];
-                const double omz = (j == am[t]) ? srest[t] / Sd[t] : (Sd[t] - ed) / Sd[t];
-                cd = 2.0 * z * omz * fabs(yd);
-              }
-              nib[t] = (nib[t] & ~(1u << e)) | ((uint32_t)(cd > (double)p.tau) << e);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        // mask word 4 i4 + lane / 8 gathers the nibbles of lanes 8w .. 8w + 7
-        uint32_t x = nib[t] << (4 * (lane & 7));
-        x |= __shfl_xor_sync(0xFFFFFFFFu, x, 1);
-        x |= __shfl_xor_sync(0xFFFFFFFFu, x, 2);
-        x |= __shfl_xor_sync(0xFFFFFFFFu, x, 4);
-        const int w = 4 * i4 + (lane >> 3);
-        if (p.mask_out && rr_[t] < it.rows && (lane & 7) == 0 && w < nwords) p.mask_out[grow[t] * nwords + w] = x;
-      }
-      if (__any_sync(0xFFFFFFFFu, (nib[0] | nib[1]) != 0u)) {
-        // compaction: an exclusive warp scan of the per-lane counts gives every
-        // lane the list slots of its selected keys (order: lane, row, key)
-        const int cnt = __popc(nib[0]) + __popc(nib[1]);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        nsel += total;
-        if (list_n + total <= WS_LIST) {
-          int pos = list_n + incl - cnt;
-#pragma unroll
-          for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if ((nib[t] >> e) & 1u) list[pos++] = (t << 16) | (j0 + e);
-          list_n += total;
-          __syncwarp();
-          while (list_n >= 32) flush(32);
-        } else {  // more than the list holds: append 32-key groups one at a time
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const bool sb = (nib[t] >> e) & 1u;
-              const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sb);
-              if (bal) {
-                if (sb) list[list_n + __popc(bal & lanemask_lt)] = (t << 16) | (j0 + e);
-                list_n += __popc(bal);
-                __syncwarp();
-                if (list_n >= 32) flush(32);
-              }
-            }
-          }
-        }
-      }
-    }
+    for (int i4 = 0; i4 < nit; ++i4)
+      sel_step<VAR>(p, S, 128 * i4, written, nwords, tlo, thi, lane, lanemask_lt, list, list_n, nsel, flush);
     if (p.mask_out) {
 #pragma unroll
       for (int t = 0; t < 2; ++t)
         if (rr_[t] < it.rows)
           for (int w = 4 * nit + lane; w < nwords; w += 32) p.mask_out[grow[t] * nwords + w] = 0u;
     }
+    __syncwarp();
     if (list_n > 0) flush(list_n);
     __syncwarp();
     if (p.mixed_out) {  // dump of the mixed scores
@@ -414,20 +302,13 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
             p.mixed_out[grow[t] * p.n_k + j] = j < written ? row[t][j] : -INFINITY;
     }
 
-    // D: softmax numerators of the mixed rows, in place
+    // D: softmax numerators of the mixed rows, in place; the maximum m' of each
+    // mixed row was tracked through the selection and the recompute
     const int nitw = (written + 127) >> 7;
-    float mm[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-    for (int i4 = 0; i4 < nitw; ++i4) {
-      const int j0 = 128 * i4 + 4 * lane;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
-        mm[t] = fmaxf(mm[t], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-      }
-    }
+    float mm[2], mL[2], l[2] = {0.f, 0.f};
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      mm[t] = warp_max(mm[t]);
+      mm[t] = warp_max_redux(S.mx[t]);
       mL[t] = mm[t] == -INFINITY ? 0.f : mm[t] * kLog2e;
     }
     for (int i4 = 0; i4 < nitw; ++i4) {

@@ -21,6 +21,10 @@ constexpr int WS_DS = 8;               // head dimensions per K slice
 constexpr int WS_LIST = 64;            // per-warp recompute list capacity
 constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
 constexpr int BAR_CONS = 1;            // named barrier of the consumer group
+// Q of an item in shared memory: [D][16 rows] f32 (dimension-major, so a 16-byte
+// load gives four rows of one dimension: the packed pairs of two row pairs)
+template <int D>
+__host__ __device__ constexpr int ws_qfloats() { return D * WS_BM; }
 
 // The k-th item of CTA b (snake order over heaviest-first items), or -1.
 __device__ __forceinline__ int ws_item(int k, int b, int G, int n_items) {
@@ -68,7 +72,8 @@ __device__ __forceinline__ void ws_stage_q(float* sQ, const Problem& p, const It
   }
 }
 
-// WS_DS accumulation steps of a lane's 8-row x 4-key tile.
+// WS_DS accumulation steps of a lane's 8-row x 4-key tile; the packed pairs run
+// over rows: acc[rp][i] holds rows 8gr + 2rp, 8gr + 2rp + 1 at key 4gk + i.
 //   qs: Q of this slice, [WS_DS][16] f32 (lane rows 8gr..8gr+7 at qoff = 8gr);
 //   ks: warp's K slice, [WS_DS][64] f32 (lane keys at koff = 4gk).
 template <int MODE>
@@ -213,6 +218,145 @@ __device__ __forceinline__ float ws_recompute(const float* __restrict__ sQ, int 
 
 __device__ __forceinline__ float4 lds4_or_ninf(const float* ptr, bool ok) {
   return ok ? *reinterpret_cast<const float4*>(ptr) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+}
+
+// ---------------------------------------------------------------------------
+// Selection pass of a consumer warp: the look-ahead test on its two rows, 128 keys
+// per step. Lane l takes keys kb + 32 m + l (m = 0..3) of step kb, so the ballot
+// of key column m over the lanes is mask word kb / 32 + m itself, and its prefix
+// popcount gives each selected key its slot in the recompute list (no scan).
+// ---------------------------------------------------------------------------
+struct SelRows {
+  float* row[2];     // the two score rows (key j of the pass at row[t][j])
+  int nv[2];         // valid keys of each row, counted from the pass's key 0
+  size_t word0[2];   // mask word of the pass's key 0 in mask_out / mask_in
+  bool live[2];      // the row exists (only live rows write mask words)
+  float mx[2];       // running maximum of the mixed row (kept and recomputed scores)
+  float mrun[2];     // relaxed: running maximum of the low-precision scores over 64-key tiles
+  // strict: statistics of the low-precision row (maximum m, first argmax am,
+  // S = 1 + S_rest in double and binary32, 2 / S^2 in binary32)
+  float mL[2], Sf[2], c2[2], srest_f[2], m[2];
+  double Sd[2], srest[2];
+  int am[2];
+};
+
+// One step (keys kb .. kb + 127 of the pass). `written` bounds the keys holding
+// scores (a multiple of 64); keys at or past it read as -inf. flush(n) recomputes
+// the first n list entries; the caller flushes what is left after the last step.
+template <int VAR, typename Flush>
+__device__ __forceinline__ void sel_step(const Problem& p, SelRows& S, int kb, int written, int nwords_left,
+                                         float tlo, float thi, int lane, uint32_t lanemask_lt, int* list,
+                                         int& list_n, long long& nsel, Flush&& flush) {
+  float y[2][4];
+  uint32_t sel[2] = {0u, 0u}, nearb[2] = {0u, 0u};
+  float mh[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // relaxed: running maximum for columns 0-1 and 2-3
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) y[t][m] = kb + 32 * m < written ? S.row[t][kb + 32 * m + lane] : -INFINITY;
+    if (VAR == LAMP_GIVEN_MASK) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int w = (kb >> 5) + m;
+        const uint32_t word = w < nwords_left ? __ldg(p.mask_in + S.word0[t] + w) : 0u;
+        sel[t] |= (uint32_t)(((word >> lane) & 1u) && kb + 32 * m + lane < S.nv[t]) << m;
+      }
+    } else if (VAR == LAMP_RELAXED) {
+      // 64-key tiles: columns 0-1 form one, columns 2-3 the next
+      const float ta = warp_max_redux(fmaxf(y[t][0], y[t][1]));
+      const float tb = warp_max_redux(fmaxf(y[t][2], y[t][3]));
+      mh[t][0] = fmaxf(S.mrun[t], ta);
+      mh[t][1] = fmaxf(mh[t][0], tb);
+      S.mrun[t] = mh[t][1];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float ex;
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[t][m], kLog2e, -(mh[t][m >> 1] * kLog2e))));
+        const float cr = 2.f * fabsf(y[t][m]) * ex;
+        sel[t] |= (uint32_t)(cr > p.tau) << m;
+        nearb[t] |= (uint32_t)(cr >= tlo && cr <= thi) << m;
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float ex;
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(y[t][m], kLog2e, -S.mL[t])));
+        const float om = __fsub_rn(S.Sf[t], ex);
+        const float cr = (fabsf(y[t][m]) * ex) * (om * S.c2[t]);
+        sel[t] |= (uint32_t)(cr > p.tau) << m;
+        nearb[t] |= (uint32_t)(cr >= tlo && cr <= thi) << m;
+      }
+      const int da = S.am[t] - kb;
+      if (da >= 0 && da < 128 && (da & 31) == lane) {  // the argmax: z = 1 / S, 1 - z = S_rest / S
+        const int ma = da >> 5;
+        const float ya = ma == 0 ? y[t][0] : (ma == 1 ? y[t][1] : (ma == 2 ? y[t][2] : y[t][3]));
+        const float cr = fabsf(ya) * (S.srest_f[t] * S.c2[t]);
+        sel[t] = (sel[t] & ~(1u << ma)) | ((uint32_t)(cr > p.tau) << ma);
+        nearb[t] = (nearb[t] & ~(1u << ma)) | ((uint32_t)(cr >= tlo && cr <= thi) << ma);
+      }
+    }
+  }
+  if (VAR != LAMP_GIVEN_MASK && __any_sync(0xFFFFFFFFu, (nearb[0] | nearb[1]) != 0u)) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if ((nearb[t] >> m) & 1u) {  // close to tau: the test again in double
+          const double yd = (double)y[t][m];
+          double cd;
+          if (VAR == LAMP_RELAXED) {
+            cd = 2.0 * exp(yd - (double)mh[t][m >> 1]) * fabs(yd);
+          } else {
+            const bool isa = kb + 32 * m + lane == S.am[t];
+            const double ed = isa ? 1.0 : exp(yd - (double)S.m[t]);
+            const double z = ed / S.Sd[t];
+            const double omz = isa ? S.srest[t] / S.Sd[t] : (S.Sd[t] - ed) / S.Sd[t];
+            cd = 2.0 * z * omz * fabs(yd);
+          }
+          sel[t] = (sel[t] & ~(1u << m)) | ((uint32_t)(cd > (double)p.tau) << m);
+        }
+  }
+  // mask words and list slots from the ballots: column (t, m) takes the slots after
+  // those of the columns before it, lane order within the column
+  uint32_t bal[2][4];
+  int off[2][4];
+  int tot = 0;
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      bal[t][m] = __ballot_sync(0xFFFFFFFFu, (sel[t] >> m) & 1u);
+      off[t][m] = tot;
+      tot += __popc(bal[t][m]);
+      const int w = (kb >> 5) + m;
+      if (p.mask_out && lane == 4 * t + m && S.live[t] && w < nwords_left) p.mask_out[S.word0[t] + w] = bal[t][m];
+      if (!((sel[t] >> m) & 1u)) S.mx[t] = fmaxf(S.mx[t], y[t][m]);
+    }
+  if (tot) {
+    nsel += tot;
+    if (list_n + tot <= WS_LIST) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if ((sel[t] >> m) & 1u)
+            list[list_n + off[t][m] + __popc(bal[t][m] & lanemask_lt)] = (t << 16) | (kb + 32 * m + lane);
+      list_n += tot;
+      __syncwarp();
+      while (list_n >= 32) flush(32);
+    } else {  // more than the list holds: one column at a time
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if (bal[t][m]) {
+            if ((sel[t] >> m) & 1u) list[list_n + __popc(bal[t][m] & lanemask_lt)] = (t << 16) | (kb + 32 * m + lane);
+            list_n += __popc(bal[t][m]);
+            __syncwarp();
+            if (list_n >= 32) flush(32);
+          }
+    }
+  }
 }
 
 }  // namespace
