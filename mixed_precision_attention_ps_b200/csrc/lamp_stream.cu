@@ -41,7 +41,7 @@ struct StSmem {
   int q;      // Q [2][D][16] f32, by item parity
   int ks;     // producer K slices [8 warps][2][8][64] f32
   int v;      // V chunks [3][VK][D + 8] bf16, later the partial outputs [KQ][16][D] f32
-  int list;   // consumer recompute lists [8][64] int
+  int list;   // consumer mask-word buffers [8][2][32] uint32
   int rstat;  // per row: m, l, alpha, spare [16][4] f32
   int tiles;  // score tiles [2][16][ST_TS] f32
   int total;
@@ -57,7 +57,7 @@ __host__ __device__ inline StSmem st_plan() {
   const int vb = ST_NST * st_vkeys<D>() * (D + 8) * 2;
   const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;
   s.list = s.v + (vb > ob ? vb : ob);
-  s.rstat = s.list + WS_NC * WS_LIST * 4;
+  s.rstat = s.list + WS_NC * 2 * SEL_WMAX * 4;
   s.tiles = s.rstat + WS_BM * 4 * 4;
   s.total = s.tiles + 2 * WS_BM * ST_TS * 4;
   return s;
@@ -132,13 +132,12 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   const int tidc = cw * 32 + lane;
   const int G = gridDim.x, cta = blockIdx.x;
   const int nwords = (p.n_k + 31) >> 5;
-  const uint32_t lanemask_lt = (1u << lane) - 1u;
   const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = WS_BAND * p.tau;
   const float tlo = refine_ok ? p.tau - band : INFINITY;
   const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  int* list = reinterpret_cast<int*>(smem + L.list) + cw * WS_LIST;
+  uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
   uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L.v);
   float* sO = reinterpret_cast<float*>(smem + L.v);
   float* qbase = reinterpret_cast<float*>(smem + L.q);
@@ -206,7 +205,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         cp_async_commit();
       };
       const int nvc = (tlen + VK - 1) / VK;
-      for (int c = 0; c < ST_NST && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
+      for (int c = 0; c < ST_NST - 1 && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
       const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
       if (named_or(BAR_CONS, NCT, !ok)) {
         ws_timeout(p);
@@ -224,22 +223,6 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
             for (int j = lane; j < ST_T && t0 + j < p.n_k; j += 32)
               p.ps_out[grow[tt] * p.n_k + t0 + j] = j < written ? row[tt][j] : -INFINITY;
       }
-      int list_n = 0;
-      auto flush = [&](int cnt) {
-        if (lane < cnt) {
-          const int e = list[lane];
-          const int tt = e >> 16, j = e & 0xFFFF;
-          const float v = ws_recompute<D>(sQ, 2 * cw + tt, Kh + (size_t)(t0 + j) * D, p.scale, fast);
-          tile[(size_t)(2 * cw + tt) * ST_TS + j] = v;
-          if (tt == 0) S.mx[0] = fmaxf(S.mx[0], v);
-          else S.mx[1] = fmaxf(S.mx[1], v);
-        }
-        __syncwarp();
-        const int rest = list_n - cnt;
-        if (lane < rest) list[lane] = list[cnt + lane];
-        __syncwarp();
-        list_n = rest;
-      };
       // criterion, mask words, compaction and recompute of the selected keys
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
@@ -249,17 +232,13 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         S.mx[tt] = -INFINITY;
       }
       for (int i4 = 0; i4 < nit; ++i4)
-        sel_step<VAR>(p, S, 128 * i4, written, nwords - (t0 >> 5), tlo, thi, lane, lanemask_lt, list, list_n, nsel,
-                      flush);
-      if (p.mask_out) {  // the tile's words past the selection loop hold no selected key
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-          if (rr_[tt] < it.rows)
-            for (int w = 4 * nit + lane; w < ST_T / 32 && (t0 >> 5) + w < nwords; w += 32)
-              p.mask_out[grow[tt] * nwords + (t0 >> 5) + w] = 0u;
-      }
-      __syncwarp();
-      if (list_n > 0) flush(list_n);
+        sel_step<VAR>(p, S, 128 * i4, written, nwords - (t0 >> 5), tlo, thi, lane, wbuf, nsel);
+      sel_finish(p, S, wbuf, 4 * nit, min(ST_T / 32, nwords - (t0 >> 5)), lane, [&](int tt, int j) {
+        const float v = ws_recompute<D>(sQ, 2 * cw + tt, Kh + (size_t)(t0 + j) * D, p.scale, fast);
+        tile[(size_t)(2 * cw + tt) * ST_TS + j] = v;
+        if (tt == 0) S.mx[0] = fmaxf(S.mx[0], v);
+        else S.mx[1] = fmaxf(S.mx[1], v);
+      });
       __syncwarp();
       if (p.mixed_out) {  // dump of the mixed scores of this tile
 #pragma unroll
@@ -319,11 +298,10 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         }
       }
       for (int vc = 0; vc < nvc; ++vc) {
-        const int pending = min(nvc, vc + ST_NST) - vc - 1;
-        if (pending >= 2) cp_async_wait<2>();
-        else if (pending == 1) cp_async_wait<1>();
+        if (vc + 1 < nvc) cp_async_wait<1>();  // chunk vc + 1 may still be in flight
         else cp_async_wait<0>();
-        named_sync(BAR_CONS, NCT);
+        named_sync(BAR_CONS, NCT);  // chunk vc landed everywhere; chunk vc - 1 is done with
+        if (vc + ST_NST - 1 < nvc) load_v(vc + ST_NST - 1, (vc + ST_NST - 1) % ST_NST);
         const uint16_t* vb = sV + (vc % ST_NST) * VK * VS;
 #pragma unroll
         for (int qq = 0; qq < SPW; ++qq) {
@@ -343,10 +321,8 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
             }
           }
         }
-        named_sync(BAR_CONS, NCT);
-        if (vc + ST_NST < nvc) load_v(vc + ST_NST, vc % ST_NST);
       }
-      if (nvc == 0) named_sync(BAR_CONS, NCT);  // every warp has read the rescale factors
+      named_sync(BAR_CONS, NCT);  // V stages and rescale factors are no longer read
 
       if (t == nt - 1) {  // end of the item: add the partial outputs, divide by l
 #pragma unroll

@@ -48,7 +48,7 @@ struct WsSmem {
   int q;      // Q [2][D][16] f32
   int ks;     // producer K slices [8 warps][2][8][64] f32
   int v;      // consumer V chunks [stages][VK][D + 8] bf16, later the partial outputs [KQ][16][D] f32
-  int list;   // consumer recompute lists [8][64] int
+  int list;   // consumer mask-word buffers [8][2][32] uint32
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
   int rows;   // score rows [2][16][nkp] f32
   int total;
@@ -64,7 +64,7 @@ __host__ __device__ inline WsSmem ws_plan(int nkp) {
   const int vb = ws_vstages<D>() * ws_vkeys<D>() * (D + 8) * 2;
   const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;  // per-warp partial outputs
   s.list = s.v + (vb > ob ? vb : ob);
-  s.stats = s.list + WS_NC * WS_LIST * 4;
+  s.stats = s.list + WS_NC * 2 * SEL_WMAX * 4;
   s.rows = s.stats + 2 * WS_BM * 2 * 4;
   s.total = s.rows + 2 * WS_BM * nkp * 4;
   return s;
@@ -133,11 +133,10 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   const int tidc = cw * 32 + lane;
   const int G = gridDim.x, cta = blockIdx.x;
   const int nwords = (p.n_k + 31) >> 5;
-  const uint32_t lanemask_lt = (1u << lane) - 1u;
   const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = WS_BAND * p.tau;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  int* list = reinterpret_cast<int*>(smem + L.list) + cw * WS_LIST;
+  uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
   uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L.v);
   float* sO = reinterpret_cast<float*>(smem + L.v);
   float* qbase = reinterpret_cast<float*>(smem + L.q);
@@ -169,7 +168,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     };
     constexpr int NST = ws_vstages<D>();
     const int nvc = (it.kv_end + VK - 1) / VK;
-    for (int c = 0; c < NST && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
+    for (int c = 0; c < NST - 1 && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
 
     const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
     if (named_or(BAR_CONS, NCT, !ok)) {
@@ -206,22 +205,6 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     const int nvmax = max(nv[0], nv[1]);
     const int nit = (nvmax + 127) >> 7;
-    int list_n = 0;
-    auto flush = [&](int cnt) {
-      if (lane < cnt) {
-        const int e = list[lane];
-        const int t = e >> 16, j = e & 0xFFFF;
-        const float v = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
-        rows[(size_t)(2 * cw + t) * a.nkp + j] = v;
-        if (t == 0) S.mx[0] = fmaxf(S.mx[0], v);
-        else S.mx[1] = fmaxf(S.mx[1], v);
-      }
-      __syncwarp();
-      const int rest = list_n - cnt;
-      if (lane < rest) list[lane] = list[cnt + lane];
-      __syncwarp();
-      list_n = rest;
-    };
     if (p.ps_out) {  // dump of the low-precision scores (before any recompute)
 #pragma unroll
       for (int t = 0; t < 2; ++t)
@@ -283,16 +266,13 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     // C: criterion, mask words, compaction and recompute of the selected keys
     const float tlo = refine_ok ? p.tau - band : INFINITY;
     const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
-    for (int i4 = 0; i4 < nit; ++i4)
-      sel_step<VAR>(p, S, 128 * i4, written, nwords, tlo, thi, lane, lanemask_lt, list, list_n, nsel, flush);
-    if (p.mask_out) {
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-        if (rr_[t] < it.rows)
-          for (int w = 4 * nit + lane; w < nwords; w += 32) p.mask_out[grow[t] * nwords + w] = 0u;
-    }
-    __syncwarp();
-    if (list_n > 0) flush(list_n);
+    for (int i4 = 0; i4 < nit; ++i4) sel_step<VAR>(p, S, 128 * i4, written, nwords, tlo, thi, lane, wbuf, nsel);
+    sel_finish(p, S, wbuf, 4 * nit, nwords, lane, [&](int t, int j) {
+      const float v = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
+      rows[(size_t)(2 * cw + t) * a.nkp + j] = v;
+      if (t == 0) S.mx[0] = fmaxf(S.mx[0], v);
+      else S.mx[1] = fmaxf(S.mx[1], v);
+    });
     __syncwarp();
     if (p.mixed_out) {  // dump of the mixed scores
 #pragma unroll
@@ -349,12 +329,13 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     for (int tt = 0; tt < 8; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
+    // one barrier per chunk: after it every copy of chunk vc has landed and every
+    // warp is done with chunk vc - 1, whose stage then takes chunk vc + NST - 1
     for (int vc = 0; vc < nvc; ++vc) {
-      const int pending = min(nvc, vc + NST) - vc - 1;  // chunks issued after this one
-      if (pending >= 2) cp_async_wait<2>();
-      else if (pending == 1) cp_async_wait<1>();
+      if (vc + 1 < nvc) cp_async_wait<1>();  // chunk vc + 1 may still be in flight
       else cp_async_wait<0>();
       named_sync(BAR_CONS, NCT);
+      if (vc + NST - 1 < nvc) load_v(vc + NST - 1, (vc + NST - 1) % NST);
       const uint16_t* vb = sV + (vc % NST) * VK * VS;
 #pragma unroll
       for (int qq = 0; qq < SPW; ++qq) {
@@ -374,9 +355,8 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
           }
         }
       }
-      named_sync(BAR_CONS, NCT);
-      if (vc + NST < nvc) load_v(vc + NST, vc % NST);
     }
+    named_sync(BAR_CONS, NCT);  // every warp is done with the V stages (the partial sums reuse them)
     // each warp's partial sums go to a slot of their own; then one pass adds the KQ
     // slots of every output in a fixed order (deterministic) and scales by 1 / l
 #pragma unroll
@@ -458,7 +438,7 @@ size_t ws_smem_bytes(int d, int n_k) {
 }
 
 bool ws_fits(int d, int n_k, size_t smem_optin) {
-  return n_k <= 0xFFFF && ws_smem_bytes(d, n_k) + kStaticSmemReserve <= smem_optin;
+  return n_k <= 32 * SEL_WMAX && ws_smem_bytes(d, n_k) + kStaticSmemReserve <= smem_optin;
 }
 
 cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st) {

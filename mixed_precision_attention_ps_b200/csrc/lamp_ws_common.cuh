@@ -18,7 +18,6 @@ constexpr int WS_NP = 8;               // producer warps
 constexpr int WS_NC = 8;               // consumer warps
 constexpr int WS_UNIT = 64;            // keys per producer unit
 constexpr int WS_DS = 8;               // head dimensions per K slice
-constexpr int WS_LIST = 64;            // per-warp recompute list capacity
 constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
 constexpr int BAR_CONS = 1;            // named barrier of the consumer group
 // Q of an item in shared memory: [D][16 rows] f32 (dimension-major, so a 16-byte
@@ -223,9 +222,13 @@ __device__ __forceinline__ float4 lds4_or_ninf(const float* ptr, bool ok) {
 // ---------------------------------------------------------------------------
 // Selection pass of a consumer warp: the look-ahead test on its two rows, 128 keys
 // per step. Lane l takes keys kb + 32 m + l (m = 0..3) of step kb, so the ballot
-// of key column m over the lanes is mask word kb / 32 + m itself, and its prefix
-// popcount gives each selected key its slot in the recompute list (no scan).
+// of key column m over the lanes is mask word kb / 32 + m itself. The words go to
+// a per-warp buffer in shared memory; after the pass one scan over the buffer
+// gives every selected key its recompute slot and the words leave for mask_out
+// in one coalesced store per row.
 // ---------------------------------------------------------------------------
+constexpr int SEL_WMAX = 32;  // mask words per row a pass holds (1024 keys)
+
 struct SelRows {
   float* row[2];     // the two score rows (key j of the pass at row[t][j])
   int nv[2];         // valid keys of each row, counted from the pass's key 0
@@ -241,12 +244,11 @@ struct SelRows {
 };
 
 // One step (keys kb .. kb + 127 of the pass). `written` bounds the keys holding
-// scores (a multiple of 64); keys at or past it read as -inf. flush(n) recomputes
-// the first n list entries; the caller flushes what is left after the last step.
-template <int VAR, typename Flush>
+// scores (a multiple of 64); keys at or past it read as -inf. wbuf is the warp's
+// [2][SEL_WMAX] word buffer.
+template <int VAR>
 __device__ __forceinline__ void sel_step(const Problem& p, SelRows& S, int kb, int written, int nwords_left,
-                                         float tlo, float thi, int lane, uint32_t lanemask_lt, int* list,
-                                         int& list_n, long long& nsel, Flush&& flush) {
+                                         float tlo, float thi, int lane, uint32_t* wbuf, long long& nsel) {
   float y[2][4];
   uint32_t sel[2] = {0u, 0u}, nearb[2] = {0u, 0u};
   float mh[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // relaxed: running maximum for columns 0-1 and 2-3
@@ -316,45 +318,54 @@ __device__ __forceinline__ void sel_step(const Problem& p, SelRows& S, int kb, i
           sel[t] = (sel[t] & ~(1u << m)) | ((uint32_t)(cd > (double)p.tau) << m);
         }
   }
-  // mask words and list slots from the ballots: column (t, m) takes the slots after
-  // those of the columns before it, lane order within the column
-  uint32_t bal[2][4];
-  int off[2][4];
-  int tot = 0;
 #pragma unroll
   for (int t = 0; t < 2; ++t)
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      bal[t][m] = __ballot_sync(0xFFFFFFFFu, (sel[t] >> m) & 1u);
-      off[t][m] = tot;
-      tot += __popc(bal[t][m]);
-      const int w = (kb >> 5) + m;
-      if (p.mask_out && lane == 4 * t + m && S.live[t] && w < nwords_left) p.mask_out[S.word0[t] + w] = bal[t][m];
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, (sel[t] >> m) & 1u);
+      if (lane == 4 * t + m) wbuf[t * SEL_WMAX + (kb >> 5) + m] = bal;
+      nsel += __popc(bal);
       if (!((sel[t] >> m) & 1u)) S.mx[t] = fmaxf(S.mx[t], y[t][m]);
     }
-  if (tot) {
-    nsel += tot;
-    if (list_n + tot <= WS_LIST) {
+}
+
+// After the pass: the first nw mask words of each row are in wbuf. Writes them
+// (and zeros up to nwrite words) to mask_out, then hands every selected key to
+// rec(t, j) (row t of the warp, key j of the pass), 32 keys per warp round.
+template <typename Rec>
+__device__ __forceinline__ void sel_finish(const Problem& p, const SelRows& S, const uint32_t* wbuf, int nw,
+                                           int nwrite, int lane, Rec&& rec) {
+  __syncwarp();
+  const uint32_t w0 = lane < nw ? wbuf[lane] : 0u;
+  const uint32_t w1 = lane < nw ? wbuf[SEL_WMAX + lane] : 0u;
+  if (p.mask_out) {
+    if (S.live[0])
+      for (int w = lane; w < nwrite; w += 32) p.mask_out[S.word0[0] + w] = w == lane ? w0 : 0u;
+    if (S.live[1])
+      for (int w = lane; w < nwrite; w += 32) p.mask_out[S.word0[1] + w] = w == lane ? w1 : 0u;
+  }
+  const int c0 = __popc(w0), cnt = c0 + __popc(w1);
+  int incl = cnt;
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  for (int base = 0; base < total; base += 32) {
+    const int e = base + lane;  // this lane's entry: owner lane L has incl[L - 1] <= e < incl[L]
+    int L = 0;
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          if ((sel[t] >> m) & 1u)
-            list[list_n + off[t][m] + __popc(bal[t][m] & lanemask_lt)] = (t << 16) | (kb + 32 * m + lane);
-      list_n += tot;
-      __syncwarp();
-      while (list_n >= 32) flush(32);
-    } else {  // more than the list holds: one column at a time
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-          if (bal[t][m]) {
-            if ((sel[t] >> m) & 1u) list[list_n + __popc(bal[t][m] & lanemask_lt)] = (t << 16) | (kb + 32 * m + lane);
-            list_n += __popc(bal[t][m]);
-            __syncwarp();
-            if (list_n >= 32) flush(32);
-          }
+    for (int step = 16; step > 0; step >>= 1)
+      if (__shfl_sync(0xFFFFFFFFu, incl, L + step - 1) <= e) L += step;
+    const uint32_t a0 = __shfl_sync(0xFFFFFFFFu, w0, L), a1 = __shfl_sync(0xFFFFFFFFu, w1, L);
+    const int r = e - (__shfl_sync(0xFFFFFFFFu, incl, L) - __popc(a0) - __popc(a1));
+    if (e < total) {
+      const int ca = __popc(a0);
+      const int t = r < ca ? 0 : 1;
+      const uint32_t word = t == 0 ? a0 : a1;
+      const int bit = __fns(word, 0, (t == 0 ? r : r - ca) + 1);
+      rec(t, 32 * L + bit);
     }
   }
 }
