@@ -39,15 +39,13 @@ namespace lamp {
 namespace {
 
 template <int D>
-__host__ __device__ constexpr int ws_vkeys() { return D == 64 ? 128 : 64; }
-template <int D>
-__host__ __device__ constexpr int ws_vstages() { return D == 64 ? 3 : 2; }  // V chunks in flight
+__host__ __device__ constexpr int ws_vring() { return D == 64 ? 6 : 4; }  // V steps in each consumer warp's ring
 
 struct WsSmem {
   int bars;   // mbarriers: full[2], empty[2]
   int q;      // Q [2][D][16] f32
   int ks;     // producer K slices [8 warps][2][8][64] f32
-  int v;      // consumer V chunks [stages][VK][D + 8] bf16, later the partial outputs [KQ][16][D] f32
+  int v;      // consumer V rings [8 warps][WR][8][72] bf16, later the partial outputs [KQ][16][D] f32
   int list;   // consumer mask-word buffers [8][2][32] uint32
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
   int rows;   // score rows [2][16][nkp] f32
@@ -61,7 +59,7 @@ __host__ __device__ inline WsSmem ws_plan(int nkp) {
   s.q = 64;
   s.ks = s.q + 2 * ws_qfloats<D>() * 4;
   s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
-  const int vb = ws_vstages<D>() * ws_vkeys<D>() * (D + 8) * 2;
+  const int vb = WS_NC * ws_vring<D>() * 8 * WS_VSW * 2;  // per-warp V rings
   const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;  // per-warp partial outputs
   s.list = s.v + (vb > ob ? vb : ob);
   s.stats = s.list + WS_NC * 2 * SEL_WMAX * 4;
@@ -123,11 +121,9 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
 template <int D, int RND, int VAR>
 __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int cw,
                                             int lane) {
-  constexpr int VK = ws_vkeys<D>();
-  constexpr int VS = D + 8;
   constexpr int NH = D / 64;
   constexpr int KQ = WS_NC / NH;
-  constexpr int SPW = (VK / 8) / KQ;
+  constexpr int WR = ws_vring<D>();
   constexpr int NCT = WS_NC * 32;  // consumer threads
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
@@ -155,20 +151,30 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
-    auto load_v = [&](int vc, int b2) {
-      uint16_t* dst = sV + b2 * VK * VS;
-      for (int u = tidc; u < VK * (D / 8); u += NCT) {
-        const int key = u / (D / 8), ch = u % (D / 8);
-        const int gkey = vc * VK + key;
-        uint16_t* dd = dst + key * VS + ch * 8;
-        if (gkey < p.n_k) cp_async16(dd, Vh + (size_t)gkey * D + ch * 8);
-        else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
+    // P.V split: warp (kq, nh) takes the 8-key steps kq, kq + KQ, ... of the row and
+    // the value columns nh*64 .. nh*64 + 63. It stages exactly those V rows in a
+    // ring of WR steps of its own (cp.async, one group per step, empty groups past
+    // the end), so the P.V loop needs no group barrier.
+    const int nh = NH == 2 ? (cw & 1) : 0;
+    const int kq = NH == 2 ? (cw >> 1) : cw;
+    const int ns_all = (it.kv_end + 7) >> 3;
+    const int nsw = ns_all > kq ? (ns_all - kq + KQ - 1) / KQ : 0;  // this warp's steps
+    uint16_t* vring = sV + cw * WR * 8 * WS_VSW;
+    auto load_step = [&](int i) {  // step i of this warp into ring slot i % WR
+      if (i < nsw) {
+        const int key0 = 8 * (kq + KQ * i);
+        uint16_t* dst = vring + (i % WR) * 8 * WS_VSW;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = lane + 32 * h, key = c >> 3, ch = c & 7;
+          uint16_t* dd = dst + key * WS_VSW + ch * 8;
+          if (key0 + key < p.n_k) cp_async16(dd, Vh + (size_t)(key0 + key) * D + nh * 64 + ch * 8);
+          else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       cp_async_commit();
     };
-    constexpr int NST = ws_vstages<D>();
-    const int nvc = (it.kv_end + VK - 1) / VK;
-    for (int c = 0; c < NST - 1 && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
+    for (int i = 0; i < WR - 1; ++i) load_step(i);  // V does not depend on the scores
 
     const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
     if (named_or(BAR_CONS, NCT, !ok)) {
@@ -321,41 +327,31 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     named_sync(BAR_CONS, NCT);  // every P row of the item is in place
 
     // ---- O = (P.V) / l on tensor cores ----------------------------------------------
-    const int nh = NH == 2 ? (cw & 1) : 0;
-    const int kq = NH == 2 ? (cw >> 1) : cw;
     const int mi = lane >> 3;
     float acc[8][4];
 #pragma unroll
     for (int tt = 0; tt < 8; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
-    // one barrier per chunk: after it every copy of chunk vc has landed and every
-    // warp is done with chunk vc - 1, whose stage then takes chunk vc + NST - 1
-    for (int vc = 0; vc < nvc; ++vc) {
-      if (vc + 1 < nvc) cp_async_wait<1>();  // chunk vc + 1 may still be in flight
-      else cp_async_wait<0>();
-      named_sync(BAR_CONS, NCT);
-      if (vc + NST - 1 < nvc) load_v(vc + NST - 1, (vc + NST - 1) % NST);
-      const uint16_t* vb = sV + (vc % NST) * VK * VS;
+    const int ra = 8 * (mi & 1) + (lane & 7);
+    const int kl = 4 * (mi & 1) + ((lane & 7) >> 1);  // each V row serves the hi and the lo half of P
+    for (int i = 0; i < nsw; ++i) {
+      cp_async_wait<WR - 2>();  // step i has landed (this lane's copies)
+      __syncwarp();             // ... and every lane's; step i - 1's slot is free
+      load_step(i + WR - 1);
+      const int kb = 8 * (kq + KQ * i);
+      const uint16_t* vb = vring + (i % WR) * 8 * WS_VSW;
+      uint32_t af[4];
+      ldmatrix_x4(smem_u32(rows + (size_t)ra * a.nkp + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
 #pragma unroll
-      for (int qq = 0; qq < SPW; ++qq) {
-        const int stp = kq + KQ * qq;
-        const int kb = vc * VK + 8 * stp;
-        if (kb < it.kv_end) {
-          uint32_t af[4];
-          const int ra = 8 * (mi & 1) + (lane & 7);
-          ldmatrix_x4(smem_u32(rows + (size_t)ra * a.nkp + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
-          const int kl = 8 * stp + 4 * (mi & 1) + ((lane & 7) >> 1);
-#pragma unroll
-          for (int nb = 0; nb < 4; ++nb) {
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4_trans(smem_u32(vb + kl * VS + nh * 64 + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
-            mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
-            mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
-          }
-        }
+      for (int nb = 0; nb < 4; ++nb) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(smem_u32(vb + kl * WS_VSW + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
+        mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
       }
     }
+    cp_async_wait<0>();
     named_sync(BAR_CONS, NCT);  // every warp is done with the V stages (the partial sums reuse them)
     // each warp's partial sums go to a slot of their own; then one pass adds the KQ
     // slots of every output in a fixed order (deterministic) and scales by 1 / l
