@@ -32,15 +32,12 @@ namespace {
 constexpr int ST_T = 512;   // keys per streamed tile
 constexpr int ST_TS = ST_T + 4;  // tile row stride (floats): 16-byte steps across banks
 
-template <int D>
-__host__ __device__ constexpr int st_vkeys() { return D == 64 ? 128 : 64; }
-constexpr int ST_NST = 3;   // V chunks in flight
 
 struct StSmem {
   int bars;   // mbarriers: full[2], empty[2]
   int q;      // Q [2][D][16] f32, by item parity
   int ks;     // producer K slices [8 warps][2][8][64] f32
-  int v;      // V chunks [3][VK][D + 8] bf16, later the partial outputs [KQ][16][D] f32
+  int v;      // consumer V rings [8 warps][WR][8][72] bf16, later the partial outputs [KQ][16][D] f32
   int list;   // consumer mask-word buffers [8][2][32] uint32
   int rstat;  // per row: m, l, alpha, spare [16][4] f32
   int tiles;  // score tiles [2][16][ST_TS] f32
@@ -54,7 +51,7 @@ __host__ __device__ inline StSmem st_plan() {
   s.q = 64;
   s.ks = s.q + 2 * ws_qfloats<D>() * 4;
   s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
-  const int vb = ST_NST * st_vkeys<D>() * (D + 8) * 2;
+  const int vb = WS_NC * ws_vring<D>() * 8 * WS_VSW * 2;  // per-warp V rings
   const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;
   s.list = s.v + (vb > ob ? vb : ob);
   s.rstat = s.list + WS_NC * 2 * SEL_WMAX * 4;
@@ -122,11 +119,9 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
 template <int D, int RND, int VAR>
 __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem, const StSmem& L, int cw,
                                             int lane) {
-  constexpr int VK = st_vkeys<D>();
-  constexpr int VS = D + 8;
   constexpr int NH = D / 64;
   constexpr int KQ = WS_NC / NH;
-  constexpr int SPW = (VK / 8) / KQ;
+  constexpr int WR = ws_vring<D>();
   constexpr int NCT = WS_NC * 32;
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
@@ -145,6 +140,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   const int nh = NH == 2 ? (cw & 1) : 0;
   const int kq = NH == 2 ? (cw >> 1) : cw;
   const int mi = lane >> 3;
+  uint16_t* vring = sV + cw * WR * 8 * WS_VSW;
   long long nsel = 0;
   // Q of the first two items; both tile buffers start out free
   for (int k0 = 0; k0 < 2; ++k0) {
@@ -193,19 +189,25 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
       const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
       float* tile = reinterpret_cast<float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
       float* row[2] = {tile + (size_t)rr_[0] * ST_TS, tile + (size_t)rr_[1] * ST_TS};
-      auto load_v = [&](int vc, int b2) {
-        uint16_t* dst = sV + b2 * VK * VS;
-        for (int u = tidc; u < VK * (D / 8); u += NCT) {
-          const int key = u / (D / 8), ch = u % (D / 8);
-          const int gkey = t0 + vc * VK + key;
-          uint16_t* dd = dst + key * VS + ch * 8;
-          if (gkey < p.n_k) cp_async16(dd, Vh + (size_t)gkey * D + ch * 8);
-          else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
+      // P.V split as in the whole-row kernel: warp (kq, nh) takes the tile's 8-key
+      // steps kq, kq + KQ, ... and columns nh*64 .. nh*64 + 63, staged in its own ring
+      const int ns_all = (tlen + 7) >> 3;
+      const int nsw = ns_all > kq ? (ns_all - kq + KQ - 1) / KQ : 0;
+      auto load_step = [&](int i) {  // step i of this warp into ring slot i % WR
+        if (i < nsw) {
+          const int key0 = t0 + 8 * (kq + KQ * i);
+          uint16_t* dst = vring + (i % WR) * 8 * WS_VSW;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = lane + 32 * h, key = c >> 3, ch = c & 7;
+            uint16_t* dd = dst + key * WS_VSW + ch * 8;
+            if (key0 + key < p.n_k) cp_async16(dd, Vh + (size_t)(key0 + key) * D + nh * 64 + ch * 8);
+            else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
         cp_async_commit();
       };
-      const int nvc = (tlen + VK - 1) / VK;
-      for (int c = 0; c < ST_NST - 1 && c < nvc; ++c) load_v(c, c);  // V does not depend on the scores
+      for (int i = 0; i < WR - 1; ++i) load_step(i);  // V does not depend on the scores
       const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
       if (named_or(BAR_CONS, NCT, !ok)) {
         ws_timeout(p);
@@ -297,31 +299,25 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
           acc[tt][3] *= a1;
         }
       }
-      for (int vc = 0; vc < nvc; ++vc) {
-        if (vc + 1 < nvc) cp_async_wait<1>();  // chunk vc + 1 may still be in flight
-        else cp_async_wait<0>();
-        named_sync(BAR_CONS, NCT);  // chunk vc landed everywhere; chunk vc - 1 is done with
-        if (vc + ST_NST - 1 < nvc) load_v(vc + ST_NST - 1, (vc + ST_NST - 1) % ST_NST);
-        const uint16_t* vb = sV + (vc % ST_NST) * VK * VS;
+      const int ra = 8 * (mi & 1) + (lane & 7);
+      const int kl = 4 * (mi & 1) + ((lane & 7) >> 1);  // each V row serves the hi and the lo half of P
+      for (int i = 0; i < nsw; ++i) {
+        cp_async_wait<WR - 2>();  // step i has landed (this lane's copies)
+        __syncwarp();             // ... and every lane's; step i - 1's slot is free
+        load_step(i + WR - 1);
+        const int kb = 8 * (kq + KQ * i);  // relative to the tile
+        const uint16_t* vb = vring + (i % WR) * 8 * WS_VSW;
+        uint32_t af[4];
+        ldmatrix_x4(smem_u32(tile + (size_t)ra * ST_TS + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
 #pragma unroll
-        for (int qq = 0; qq < SPW; ++qq) {
-          const int stp = kq + KQ * qq;
-          const int kb = vc * VK + 8 * stp;  // relative to the tile
-          if (kb < tlen) {
-            uint32_t af[4];
-            const int ra = 8 * (mi & 1) + (lane & 7);
-            ldmatrix_x4(smem_u32(tile + (size_t)ra * ST_TS + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
-            const int kl = 8 * stp + 4 * (mi & 1) + ((lane & 7) >> 1);
-#pragma unroll
-            for (int nb = 0; nb < 4; ++nb) {
-              uint32_t b0, b1, b2, b3;
-              ldmatrix_x4_trans(smem_u32(vb + kl * VS + nh * 64 + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
-              mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
-              mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
-            }
-          }
+        for (int nb = 0; nb < 4; ++nb) {
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(smem_u32(vb + kl * WS_VSW + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
+          mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
         }
       }
+      cp_async_wait<0>();
       named_sync(BAR_CONS, NCT);  // V stages and rescale factors are no longer read
 
       if (t == nt - 1) {  // end of the item: add the partial outputs, divide by l

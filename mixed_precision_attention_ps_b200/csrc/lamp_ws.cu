@@ -38,9 +38,6 @@
 namespace lamp {
 namespace {
 
-template <int D>
-__host__ __device__ constexpr int ws_vring() { return D == 64 ? 6 : 4; }  // V steps in each consumer warp's ring
-
 struct WsSmem {
   int bars;   // mbarriers: full[2], empty[2]
   int q;      // Q [2][D][16] f32

@@ -21,6 +21,8 @@ constexpr int WS_DS = 8;               // head dimensions per K slice
 constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
 constexpr int BAR_CONS = 1;            // named barrier of the consumer group
 constexpr int WS_VSW = 72;             // row stride (bf16) of a consumer warp's V ring: 64 columns + pad
+template <int D>
+__host__ __device__ constexpr int ws_vring() { return D == 64 ? 6 : 4; }  // V steps in a consumer warp's ring
 // Q of an item in shared memory: [D][16 rows] f32 (dimension-major, so a 16-byte
 // load gives four rows of one dimension: the packed pairs of two row pairs)
 template <int D>
