@@ -71,6 +71,7 @@ DEFAULTS = {  # workload -> (variant, rate)
     "gpt2xl_1x25x1024x64": (0, 0.016),
     "batch8_8x25x1024x64": (1, 0.016),
     "long_1x32x16384x128": (1, 0.01),
+    "long_1x8x4096x128": (1, 0.01),
     "outlier_4x25x4096x64": (0, 0.003),
     "single_head_128": (0, None),
 }

@@ -202,5 +202,7 @@ WORKLOADS = {
     "gpt2xl_1x25x1024x64": Workload(1, 25, 1024, 1024, 64),
     "batch8_8x25x1024x64": Workload(8, 25, 1024, 1024, 64),
     "long_1x32x16384x128": Workload(1, 32, 16384, 16384, 128),
+    # a smaller case of the streamed relaxed kernel, sized for profiling captures
+    "long_1x8x4096x128": Workload(1, 8, 4096, 4096, 128),
     "outlier_4x25x4096x64": Workload(4, 25, 4096, 4096, 64, outlier_frac=0.01),
 }
