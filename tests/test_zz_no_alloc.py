@@ -48,6 +48,9 @@ def call(entry, w, Qd, Kd, Vd, o, mu, tau, variant, **extra):
     (S.Workload(1, 3, 300, 300, 64, seed=21), 4, 0.03, lamp.LAMP_STRICT),
     (S.Workload(2, 2, 100, 517, 128, causal=False, seed=22), 6, 0.5, lamp.LAMP_RELAXED),
     (S.Workload(1, 2, 40, 3000, 64, causal=False, seed=23), 4, 0.02, lamp.LAMP_STRICT),
+    # relaxed rows longer than 1024 keys: the streamed one-pass kernel
+    (S.Workload(1, 2, 40, 2500, 64, causal=False, seed=26), 4, 0.3, lamp.LAMP_RELAXED),
+    (S.Workload(1, 1, 24, 1500, 128, seed=27), 6, 0.2, lamp.LAMP_RELAXED),
 ])
 def test_matches_the_allocating_entry_on_two_calls_in_a_row(w, mu, tau, variant):
     Q, K, V = S.make_qkv(w)
