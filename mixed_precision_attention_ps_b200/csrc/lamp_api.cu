@@ -154,6 +154,7 @@ cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char*
                         cudaStream_t st) {
   cudaError_t e = lamp::launch_prep(p, ws, base, st);
   if (e != cudaSuccess) return e;
+  if (ws.use_decode) return lamp::launch_decode(p, ws, base, st);
   if (ws.use_ws) return lamp::launch_ws(p, ws, base, info.num_sms, st);
   if (ws.use_stream) return lamp::launch_stream(p, ws, base, info.num_sms, st);
   if (ws.rows_bm) return lamp::launch_rows(p, ws, base, info.num_sms, st);
@@ -201,6 +202,20 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
   w.spill = off;
   w.spill_rows = 0;
   w.grid = 0;
+  // decode shapes (a few query rows per head, long rows): split over the keys
+  if (p.n_q <= kDecodeMaxQ && p.n_k >= kDecodeMinKeys) {
+    w.use_decode = 1;
+    w.dec_chunks = (p.n_k + kDecodeChunk - 1) / kDecodeChunk;
+    const size_t rows = (size_t)BH * p.n_q;
+    w.dec_scores = off;
+    off = align256(off + rows * w.dec_chunks * kDecodeChunk * 4);
+    w.dec_stat = off;
+    off = align256(off + rows * w.dec_chunks * 16);
+    w.dec_part = off;
+    off = align256(off + rows * w.dec_chunks * (2 + (size_t)p.d) * 4);
+    w.total = off;
+    return w;
+  }
   w.use_ws = ws_fits(p.d, p.n_k, smem_optin) ? 1 : 0;
   // the relaxed and given-mask tests need no whole row: rows too long for the
   // whole-row kernel stream through 512-key tiles instead
@@ -246,7 +261,7 @@ int lamp_attention_ex(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (!ws.use_ws && !ws.use_stream && !ws.rows_bm &&
+  if (!ws.use_decode && !ws.use_ws && !ws.use_stream && !ws.rows_bm &&
       lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
     return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
   if (a->workspace && a->workspace_bytes < ws.total)
@@ -281,7 +296,7 @@ int lamp_attention_noalloc(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (!ws.use_ws && !ws.use_stream && !ws.rows_bm &&
+  if (!ws.use_decode && !ws.use_ws && !ws.use_stream && !ws.rows_bm &&
       lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
     return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
   if (ws.total > (size_t)LAMP_NOALLOC_SCRATCH_BYTES)

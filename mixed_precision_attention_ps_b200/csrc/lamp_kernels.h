@@ -50,6 +50,11 @@ struct Workspace {
   int rows_bm;         // rows per item of the on-chip row kernel; 0 = global-slab kernel
   int use_ws;          // 1: warp-specialised kernel (two 16-row buffers fit on chip)
   int use_stream;      // 1: streamed one-pass kernel (relaxed / given mask, rows too long for use_ws)
+  int use_decode;      // 1: split-key decode kernels (few query rows, long rows)
+  int dec_chunks;      // decode: 512-key chunks per row
+  size_t dec_scores;   // decode: fp32 low-precision scores [B*H][n_q][dec_chunks * 512]
+  size_t dec_stat;     // decode: per (row, chunk) maximum, first argmax, S_rest (16 bytes)
+  size_t dec_part;     // decode: per (row, chunk) softmax maximum, normaliser, partial output [2 + d] f32
 };
 
 // Strict / given-mask configuration: rows per work item and threads.
@@ -69,6 +74,10 @@ int rows_pick_bm(int d, int n_k, size_t smem_optin);
 cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
 bool ws_fits(int d, int n_k, size_t smem_optin);
 cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
+cudaError_t launch_decode(const Problem& p, const Workspace& ws, char* base, cudaStream_t st);
+constexpr int kDecodeMaxQ = 4;       // query rows per (b, h) the decode kernels take
+constexpr int kDecodeMinKeys = 512;  // shortest rows routed to them
+constexpr int kDecodeChunk = 512;    // keys per chunk (one CTA)
 size_t stream_smem_bytes(int d);
 int rows_nkp(int bm, int n_k);
 size_t rows_smem_bytes(int d, int bm, int n_k);
