@@ -72,6 +72,7 @@ DEFAULTS = {  # workload -> (variant, rate)
     "batch8_8x25x1024x64": (1, 0.016),
     "long_1x32x16384x128": (1, 0.01),
     "long_1x8x4096x128": (1, 0.01),
+    "decode_1x32x1x16384x128": (0, 0.016),
     "outlier_4x25x4096x64": (0, 0.003),
     "single_head_128": (0, None),
 }
@@ -85,6 +86,11 @@ def lookup_tau(workload: str, variant: int, mu: int, rate: float | None) -> tupl
         if e["workload"] == workload and e["variant"] == variant and e["mu"] == mu and abs(e["rate"] - rate) < 1e-12:
             return float(e["tau"]), float(e["rate"])
     raise SystemExit(f"no tau for {workload} variant={variant} mu={mu} rate={rate} in {TAU_FILE}")
+
+
+def is_decode(w) -> bool:
+    """The library's decode routing: few query rows per head against long rows."""
+    return w.n_q <= 4 and w.n_k >= 512
 
 
 def dist_env():
@@ -328,7 +334,7 @@ def run_ours(a, w, variant, mu, tau, cfg):
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    launches_per_step = 2  # exponent-statistics kernel + row kernel
+    launches_per_step = 4 if is_decode(w) else 2  # exponent statistics + row kernel (decode: + 3)
 
     # ---- end to end through the C ABI with host buffers ---------------------------------
     # Every step copies its inputs from pinned host memory and reads its output and
@@ -418,7 +424,7 @@ def run_ours(a, w, variant, mu, tau, cfg):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e, ms_serial = float(t[0].item()), float(t[1].item())
         dist.barrier()
-    h2d = 3 * Q.nbytes
+    h2d = Q.nbytes + K.nbytes + V.nbytes
     d2h = out.numel() * 2 + mask.numel() * 4
 
     result = None
@@ -437,6 +443,21 @@ def run_ours(a, w, variant, mu, tau, cfg):
                 "kernel": "one call: exponent-statistics kernel + the row kernel for the shape "
                           "(ws_kernel for n_k <= 1024 at d = 64); the row kernel is ~97% of the call",
                 "peak_basis": f"148 SMs x 128 lanes/clk x {f_max / 1e6:.0f} MHz (max SM clock)"}
+        if is_decode(w):
+            # decode shapes stream K and V once per call: HBM bounds them. Algorithmic
+            # bytes: K and V read, Q read, out and mask written (the score scratch is
+            # L2 resident).
+            nbytes = (2 * w.B * w.H * w.n_k * w.d * 2 + 2 * w.B * w.H * w.n_q * w.d * 2
+                      + w.B * w.H * w.n_q * ((w.n_k + 31) // 32) * 4)
+            hbm = float(peaks.get("hbm_gbs", 6650.0))
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                    "traffic": traffic_bytes(a.workload, variant, mu), "bytes_per_call": nbytes,
+                    "kernel": "one call: exponent statistics + the three decode kernels (scores and chunk "
+                              "statistics, selection and partial P.V, combine)",
+                    "peak_basis": "MEASURED_PEAKS.json hbm_gbs (copy)" if "hbm_gbs" in peaks
+                                  else "fallback 6650 GB/s",
+                    "alu_frac": achieved / peak}
         result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
                   "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                   "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,

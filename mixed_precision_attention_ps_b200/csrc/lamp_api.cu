@@ -152,9 +152,10 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // The launch sequence of one call: exponent statistics, then the row kernel.
 cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char* base, const DeviceInfo& info,
                         cudaStream_t st) {
+  // the decode kernels fold their own exponent statistics and reset the count
+  if (ws.use_decode) return lamp::launch_decode(p, ws, base, st);
   cudaError_t e = lamp::launch_prep(p, ws, base, st);
   if (e != cudaSuccess) return e;
-  if (ws.use_decode) return lamp::launch_decode(p, ws, base, st);
   if (ws.use_ws) return lamp::launch_ws(p, ws, base, info.num_sms, st);
   if (ws.use_stream) return lamp::launch_stream(p, ws, base, info.num_sms, st);
   if (ws.rows_bm) return lamp::launch_rows(p, ws, base, info.num_sms, st);
@@ -213,6 +214,10 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
     off = align256(off + rows * w.dec_chunks * 16);
     w.dec_part = off;
     off = align256(off + rows * w.dec_chunks * (2 + (size_t)p.d) * 4);
+    w.dec_flag = off;
+    off = align256(off + (size_t)BH * w.dec_chunks * 4);
+    w.dec_done = off;
+    off = align256(off + rows * 4);
     w.total = off;
     return w;
   }

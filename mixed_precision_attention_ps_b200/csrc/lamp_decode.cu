@@ -22,10 +22,12 @@
 //      compacted from the ballot words), then the chunk's softmax numerators
 //      against its own maximum, their sum, and the partial output sum_j p_j V_j
 //      in binary32 (CUDA cores: one row needs no tensor cores).
-//   3. combine: per row, the chunk partials rescaled to the row maximum, summed in
-//      chunk order and divided by the normaliser.
+//   3. combine: the last chunk of a row to finish (a per-row counter) rescales
+//      the row's chunk partials to the row maximum, adds them in chunk order and
+//      divides by the normaliser.
 // Memory traffic is K once, V once and the small scratch: the split keeps HBM
-// busy, which bounds this shape.
+// busy, which bounds this shape. Each CTA asks for its chunk of K (scores) or V
+// (selection) towards L2 with one bulk prefetch when it starts.
 #include <cfloat>
 
 #include "lamp.h"
@@ -47,12 +49,12 @@ struct DecStat {
 
 struct DecArgs {
   Problem p;
-  const int* stats;  // per-(b, h) exponent statistics
-  int nchunk;        // their records per head
   int n_ch;          // key chunks per row
   float* scores;     // [BH][n_q][n_ch * DC_CK]
   DecStat* cstat;    // [BH][n_q][n_ch]
   float* part;       // [BH][n_q][n_ch][2 + d]
+  int* cfast;        // [BH][n_ch]: the chunk's products are exact (the recompute may fuse)
+  unsigned* rowdone; // [BH][n_q]: chunks of the row whose partials are written
 };
 
 __device__ __forceinline__ int dec_valid(int i, const Problem& p) {
@@ -109,20 +111,96 @@ __device__ __forceinline__ float block_sum_f(float v, float* red) {
 
 // ---------------------------------------------------------------------------
 // 1. Scores and chunk statistics. grid (n_ch, B*H).
-// Shared memory: K chunk [DC_CK keys][D/8 pieces] uint4 (piece c of key j at
-// c ^ ((j >> 1) & 7)), then Q as packed pairs {q, q} [n_q][D] u64.
+// K comes in slices of 16 dimensions of all 512 keys through a ring of DC_NR
+// slots (cp.async, [2 pieces][512 keys] uint4 per slot, so the 16-byte loads of
+// consecutive threads are consecutive). Thread t computes keys t and t + 256 for
+// the NQ query rows at once; a slice's 16 values of each Q row sit in registers.
+// The two-instruction rounding is taken optimistically: the largest and smallest
+// magnitudes of the chunk's K values are folded on the way (binary32 max / min of
+// the widened values; padding keys hold 1.0), and a chunk outside the rounding's
+// domain (or holding an exact zero, conservatively) is computed again with the
+// exact rounding.
 // ---------------------------------------------------------------------------
+constexpr int DC_NR = 4;  // K slices in the ring
+
 template <int D>
 __host__ __device__ constexpr size_t dec_scores_smem() {
-  return (size_t)DC_CK * D * 2 + (size_t)DC_MAXQ * D * 8;
+  return (size_t)DC_MAXQ * D * 4 + (size_t)DC_NR * 2 * DC_CK * 16;
 }
 
-template <int D, int RND>
+__device__ __forceinline__ int f32_exp(float v) { return (int)((__float_as_uint(v) >> 23) & 0xFFu); }
+
+// The rounding-domain test of the exponent-statistics kernel, from the largest
+// and smallest nonzero magnitudes of Q and of K (exponent fields).
+__device__ __forceinline__ bool dec_fast_ok(float qmax, float qmin, float kmax, float kmin, int emax_sum_limit) {
+  if (!(kmin > 0.f) || !(qmin > 0.f)) return false;  // a zero (or NaN): take the exact rounding
+  const int s0 = f32_exp(qmax), s2 = f32_exp(kmax);
+  if (s0 >= 255 || s2 >= 255) return false;
+  const int eq = s0 - 127, ek = s2 - 127;
+  const int lq = max(f32_exp(qmin), 1) - 134, lk = max(f32_exp(kmin), 1) - 134;
+  return (eq + ek <= emax_sum_limit) && (lq + lk >= -126);
+}
+
+template <int D, int NQ, int MODE, bool FOLD>
+__device__ __forceinline__ void dec_slices(const uint16_t* Kh, int k0, int n_k, const float* sQf, uint4* ring,
+                                           u64 (&acc)[NQ], float& kmax, float& kmin, u64 negc, u64 pow2s, int s) {
+  constexpr int NSL = D / 16;
+  const int t = threadIdx.x;
+  auto issue = [&](int sl) {
+    if (sl < NSL) {
+      uint4* slot = ring + (sl % DC_NR) * 2 * DC_CK;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int u = t + DC_T * r, j = u >> 1, pc = u & 1;
+        uint4* dst = slot + pc * DC_CK + j;
+        if (k0 + j < n_k) cp_async16(dst, Kh + (size_t)(k0 + j) * D + sl * 16 + pc * 8);
+        else *dst = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // 1.0: no effect on the test
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) acc[i] = 0ull;
+  for (int sl = 0; sl < DC_NR - 1; ++sl) issue(sl);
+  for (int sl = 0; sl < NSL; ++sl) {
+    cp_async_wait<DC_NR - 2>();
+    __syncthreads();  // slice sl has landed everywhere; every thread is done with slice sl - 1
+    issue(sl + DC_NR - 1);
+    const uint4* slot = ring + (sl % DC_NR) * 2 * DC_CK;
+    const uint4 a0 = slot[t], a1 = slot[DC_CK + t], b0 = slot[t + DC_T], b1 = slot[DC_CK + t + DC_T];
+    const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    float q[NQ][16];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float4 f = *reinterpret_cast<const float4*>(sQf + i * D + sl * 16 + 4 * v);
+        q[i][4 * v] = f.x; q[i][4 * v + 1] = f.y; q[i][4 * v + 2] = f.z; q[i][4 * v + 3] = f.w;
+      }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t xa = (e & 1) ? (wa[e >> 1] & 0xFFFF0000u) : (wa[e >> 1] << 16);
+      const uint32_t xb = (e & 1) ? (wb[e >> 1] & 0xFFFF0000u) : (wb[e >> 1] << 16);
+      if (FOLD) {
+        const float fa = fabsf(__uint_as_float(xa)), fb = fabsf(__uint_as_float(xb));
+        kmax = fmaxf(kmax, fmaxf(fa, fb));
+        kmin = fminf(kmin, fminf(fa, fb));
+      }
+      const u64 kp = (u64)xa | ((u64)xb << 32);
+#pragma unroll
+      for (int i = 0; i < NQ; ++i) acc[i] = ps_step<MODE>(pack2(q[i][e], q[i][e]), kp, acc[i], negc, pow2s, s);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();  // the ring may be refilled
+}
+
+template <int D, int RND, int NQ>
 __global__ void __launch_bounds__(DC_T) dec_scores_kernel(const DecArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int NP = D / 8;  // 16-byte pieces per K row
-  uint4* sK = reinterpret_cast<uint4*>(smem);
-  u64* sQ = reinterpret_cast<u64*>(smem + (size_t)DC_CK * D * 2);
+  float* sQf = reinterpret_cast<float*>(smem);
+  uint4* ring = reinterpret_cast<uint4*>(smem + (size_t)DC_MAXQ * D * 4);
   __shared__ float redf[DC_T / 32];
   __shared__ int redi[DC_T / 32];
   __shared__ double redd[DC_T / 32];
@@ -130,63 +208,60 @@ __global__ void __launch_bounds__(DC_T) dec_scores_kernel(const DecArgs a) {
   const int c = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int k0 = c * DC_CK;
   const uint16_t* Kh = p.K + (size_t)bh * p.n_k * D;
-  for (int u = t; u < DC_CK * NP; u += DC_T) {
-    const int j = u / NP, pc = u % NP;
-    uint4* dst = sK + j * NP + (pc ^ ((j >> 1) & 7));
-    if (k0 + j < p.n_k) cp_async16(dst, Kh + (size_t)(k0 + j) * D + pc * 8);
-    else *dst = make_uint4(0u, 0u, 0u, 0u);
+  if (t == 0) {  // the whole chunk of K towards L2 at once; the ring then reads it from there
+    const int nk = min(DC_CK, p.n_k - k0);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(Kh + (size_t)k0 * D), "r"(nk * D * 2) : "memory");
   }
-  cp_async_commit();
-  for (int u = t; u < p.n_q * D; u += DC_T) {
-    const int i = u / D, dd = u % D;
-    const float q = __uint_as_float((uint32_t)p.Q[((size_t)bh * p.n_q + i) * D + dd] << 16);
-    sQ[u] = pack2(q, q);
+  if (c == 0 && t < NQ) a.rowdone[(size_t)bh * NQ + t] = 0;  // the selection kernel counts finished chunks
+  if (c == 0 && bh == 0 && t == 0 && p.nsel_out) *p.nsel_out = 0ull;
+  // Q rows, binary32, and their largest and smallest magnitudes
+  float qmax = 0.f, qmin = INFINITY;
+  for (int u = t; u < NQ * D; u += DC_T) {
+    const float q = __uint_as_float((uint32_t)p.Q[(size_t)bh * NQ * D + u] << 16);
+    sQf[u] = q;
+    qmax = fmaxf(qmax, fabsf(q));
+    qmin = fminf(qmin, fabsf(q));
   }
-  const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)bh * a.nchunk * 4, a.nchunk,
-                                                        p.emax_sum_limit);
   const int s = 23 - p.mu;
   const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
   const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
   const u64 scale2 = pack2(p.scale, p.scale);
-  cp_async_wait<0>();
-  __syncthreads();
-  const int j0 = 2 * t, sw = t & 7;  // keys j0, j0 + 1 of the chunk (same swizzle)
-  const uint4* ka = sK + j0 * NP;
-  const uint4* kb = sK + (j0 + 1) * NP;
-  for (int i = 0; i < p.n_q; ++i) {
-    u64 acc = 0ull;
-    const u64* qrow = sQ + i * D;
-#pragma unroll 2
-    for (int pc = 0; pc < NP; ++pc) {
-      const uint4 va = ka[pc ^ sw], vb = kb[pc ^ sw];
-      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+  u64 acc[NQ];
+  float kmax = 0.f, kmin = INFINITY;
+  int fast = 0;
+  if (RND == kRndExact) {
+    dec_slices<D, NQ, kStepExact, false>(Kh, k0, p.n_k, sQf, ring, acc, kmax, kmin, negc, pow2s, s);
+  } else {
+    dec_slices<D, NQ, RND == kRndFast ? kStepFast : kStepF32, true>(Kh, k0, p.n_k, sQf, ring, acc, kmax, kmin, negc,
+                                                                    pow2s, s);
+    qmax = block_max(qmax, redf);
+    qmin = -block_max(-qmin, redf);
+    kmax = block_max(kmax, redf);
+    kmin = -block_max(-kmin, redf);
+    fast = dec_fast_ok(qmax, qmin, kmax, kmin, p.emax_sum_limit) ? 1 : 0;
+    if (!fast)  // outside the two-instruction rounding's domain: the exact rounding
+      dec_slices<D, NQ, kStepExact, false>(Kh, k0, p.n_k, sQf, ring, acc, kmax, kmin, negc, pow2s, s);
+  }
+  if (t == 0) a.cfast[(size_t)bh * a.n_ch + c] = fast;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t xa = (e & 1) ? (wa[e >> 1] & 0xFFFF0000u) : (wa[e >> 1] << 16);
-        const uint32_t xb = (e & 1) ? (wb[e >> 1] & 0xFFFF0000u) : (wb[e >> 1] << 16);
-        const u64 kp = (u64)xa | ((u64)xb << 32);
-        const u64 q = qrow[pc * 8 + e];
-        if (RND == kRndFast && fast) acc = ps_step<kStepFast>(q, kp, acc, negc, pow2s, s);
-        else if (RND == kRndNone && fast) acc = ps_step<kStepF32>(q, kp, acc, negc, pow2s, s);
-        else acc = ps_step<kStepExact>(q, kp, acc, negc, pow2s, s);
-      }
-    }
-    const u64 y2 = mul2u(acc, scale2);
+  for (int i = 0; i < NQ; ++i) {
+    const u64 y2 = mul2u(acc[i], scale2);
     const int nv = dec_valid(i, p);
-    const float y0 = k0 + j0 < nv ? lo_f(y2) : -INFINITY;
-    const float y1 = k0 + j0 + 1 < nv ? hi_f(y2) : -INFINITY;
-    const size_t row = (size_t)bh * p.n_q + i;
-    *reinterpret_cast<float2*>(a.scores + row * ((size_t)a.n_ch * DC_CK) + k0 + j0) = make_float2(y0, y1);
+    const float y0 = k0 + t < nv ? lo_f(y2) : -INFINITY;
+    const float y1 = k0 + t + DC_T < nv ? hi_f(y2) : -INFINITY;
+    const size_t row = (size_t)bh * NQ + i;
+    float* yrow = a.scores + row * ((size_t)a.n_ch * DC_CK) + k0;
+    yrow[t] = y0;
+    yrow[t + DC_T] = y1;
     // chunk statistics: maximum, first argmax, and the sum over the other keys
-    const float lm = fmaxf(y0, y1);
-    const float m = block_max(lm, redf);
+    const float m = block_max(fmaxf(y0, y1), redf);
     int li = 0x7FFFFFFF;
-    if (m > -INFINITY) li = y0 == m ? k0 + j0 : (y1 == m ? k0 + j0 + 1 : 0x7FFFFFFF);
+    if (m > -INFINITY) li = y0 == m ? k0 + t : (y1 == m ? k0 + t + DC_T : 0x7FFFFFFF);
     const int am = block_min_i(li, redi);
     double sl = 0.0;
     if (m > -INFINITY) {
-      if (k0 + j0 != am) sl += (double)expf(__fsub_rn(y0, m));
-      if (k0 + j0 + 1 != am) sl += (double)expf(__fsub_rn(y1, m));
+      if (k0 + t != am) sl += (double)expf(__fsub_rn(y0, m));
+      if (k0 + t + DC_T != am) sl += (double)expf(__fsub_rn(y1, m));
     }
     const double sc = block_sum_d(sl, redd);
     if (t == 0) {
@@ -227,7 +302,7 @@ __device__ __forceinline__ float dec_recompute(const float* qf, const uint16_t* 
 }
 
 template <int D, int VAR>
-__global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a, int rnd) {
+__global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a) {
   constexpr int G = DC_T / (D / 2);  // key groups of the partial P.V
   __shared__ float ys[DC_CK];        // mixed scores of the chunk (current row)
   __shared__ float ps[DC_CK];        // softmax numerators against the chunk maximum
@@ -241,14 +316,19 @@ __global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a, int r
   const int c = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
   const int k0 = c * DC_CK;
   const int nwords = (p.n_k + 31) >> 5;
-  const bool fast = (rnd != kRndExact) && head_fast_ok(a.stats + (size_t)bh * a.nchunk * 4, a.nchunk,
-                                                        p.emax_sum_limit);
+  const bool fast = a.cfast[(size_t)bh * a.n_ch + c] != 0;
   const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = 8e-6f * p.tau;
   const float tlo = refine_ok ? p.tau - band : INFINITY;
   const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
   const uint16_t* Kh = p.K + (size_t)bh * p.n_k * D;
   const uint16_t* Vh = p.V + (size_t)bh * p.n_k * D;
+  if (t == 0) {  // the chunk's V rows towards L2 while the selection runs
+    const int nk = min(DC_CK, p.n_k - k0);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(Vh + (size_t)k0 * D), "r"(nk * D * 2) : "memory");
+  }
+  __shared__ float wgt[DC_T];  // combine: chunk weights
+  __shared__ int last;
   long long nsel = 0;
   for (int i = 0; i < p.n_q; ++i) {
     const size_t row = (size_t)bh * p.n_q + i;
@@ -371,14 +451,25 @@ __global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a, int r
     {
       const int dp = t % (D / 2), gq = t / (D / 2);
       const int kend = min(DC_CK, nv - k0);
+      const uint32_t* vcol = reinterpret_cast<const uint32_t*>(Vh + (size_t)k0 * D) + dp;
       float o0 = 0.f, o1 = 0.f;
-      for (int j = gq; j < kend; j += G) {
-        const float pj = ps[j];
-        if (pj != 0.f) {
-          const uint32_t v2 = __ldg(reinterpret_cast<const uint32_t*>(Vh + (size_t)(k0 + j) * D) + dp);
-          o0 = fmaf(pj, bf16_lo(v2), o0);
-          o1 = fmaf(pj, bf16_hi(v2), o1);
+      // eight independent loads in flight per thread (V is read once: HBM bound)
+      int j = gq;
+      for (; j + 7 * G < kend; j += 8 * G) {
+        uint32_t v2[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v2[u] = __ldg(vcol + (size_t)(j + u * G) * (D / 2));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float pj = ps[j + u * G];
+          o0 = fmaf(pj, bf16_lo(v2[u]), o0);
+          o1 = fmaf(pj, bf16_hi(v2[u]), o1);
         }
+      }
+      for (; j < kend; j += G) {
+        const uint32_t v2 = __ldg(vcol + (size_t)j * (D / 2));
+        o0 = fmaf(ps[j], bf16_lo(v2), o0);
+        o1 = fmaf(ps[j], bf16_hi(v2), o1);
       }
       ro[gq][2 * dp] = o0;
       ro[gq][2 * dp + 1] = o1;
@@ -395,65 +486,79 @@ __global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a, int r
       pr[0] = mc;
       pr[1] = lc;
     }
+    // the last chunk of the row to finish adds up the row's partials (chunk order)
+    __threadfence();
+    __syncthreads();
+    if (t == 0) last = atomicAdd(a.rowdone + row, 1u) == (unsigned)(a.n_ch - 1);
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      const float* p0 = a.part + row * a.n_ch * (2 + D);
+      float lm = -INFINITY;
+      for (int cc = t; cc < a.n_ch; cc += DC_T) lm = fmaxf(lm, __ldcg(p0 + (size_t)cc * (2 + D)));
+      const float m = block_max(lm, redf);
+      float l = 0.f, o = 0.f;
+      for (int c0 = 0; c0 < a.n_ch; c0 += DC_T) {
+        const int nc = min(DC_T, a.n_ch - c0);
+        __syncthreads();
+        if (t < nc) {
+          const float mcc = __ldcg(p0 + (size_t)(c0 + t) * (2 + D));
+          wgt[t] = (m == -INFINITY || mcc == -INFINITY) ? 0.f : expf(__fsub_rn(mcc, m));
+        }
+        __syncthreads();
+        if (t < D) {
+#pragma unroll 8
+          for (int cc = 0; cc < nc; ++cc) {
+            const float* q = p0 + (size_t)(c0 + cc) * (2 + D);
+            l = fmaf(__ldcg(q + 1), wgt[cc], l);
+            o = fmaf(__ldcg(q + 2 + t), wgt[cc], o);
+          }
+        }
+      }
+      if (t < D) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float v = o * inv;
+        p.out[row * D + t] = f32_to_bf16_rne(v);
+        if (p.out_f32) p.out_f32[row * D + t] = v;
+        if (t == 0 && p.lse_out) p.lse_out[row] = nv > 0 ? m + logf(l) : -INFINITY;
+      }
+    }
     __syncthreads();  // shared arrays are reused by the next row
   }
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
 }
 
-// ---------------------------------------------------------------------------
-// 3. Combine: per row, the chunk partials rescaled to the row maximum, summed in
-// chunk order, divided by the normaliser. grid (B*H*n_q), D threads.
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(D) dec_combine_kernel(const DecArgs a) {
-  const Problem& p = a.p;
-  const size_t row = blockIdx.x;
-  const int t = threadIdx.x;
-  const float* pr = a.part + row * a.n_ch * (2 + D);
-  float m = -INFINITY;
-  for (int c = 0; c < a.n_ch; ++c) m = fmaxf(m, pr[(size_t)c * (2 + D)]);
-  float l = 0.f, o = 0.f;
-  if (m > -INFINITY) {
-    for (int c = 0; c < a.n_ch; ++c) {
-      const float* q = pr + (size_t)c * (2 + D);
-      if (q[0] == -INFINITY) continue;
-      const float wgt = expf(__fsub_rn(q[0], m));
-      l = fmaf(q[1], wgt, l);
-      o = fmaf(q[2 + t], wgt, o);
-    }
-  }
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  const float v = o * inv;
-  p.out[row * D + t] = f32_to_bf16_rne(v);
-  if (p.out_f32) p.out_f32[row * D + t] = v;
-  if (t == 0 && p.lse_out) {
-    const int i = (int)(row % p.n_q);
-    p.lse_out[row] = dec_valid(i, p) > 0 ? m + logf(l) : -INFINITY;
+template <int D, int RND, int NQ>
+cudaError_t dec_launch_scores(const DecArgs& a, dim3 grid, cudaStream_t st) {
+  const size_t smem = dec_scores_smem<D>();
+  cudaError_t e = cudaFuncSetAttribute(dec_scores_kernel<D, RND, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dec_scores_kernel<D, RND, NQ><<<grid, DC_T, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int RND>
+cudaError_t dec_launch_rnd(const DecArgs& a, dim3 grid, cudaStream_t st) {
+  switch (a.p.n_q) {
+    case 1: return dec_launch_scores<D, RND, 1>(a, grid, st);
+    case 2: return dec_launch_scores<D, RND, 2>(a, grid, st);
+    case 3: return dec_launch_scores<D, RND, 3>(a, grid, st);
+    default: return dec_launch_scores<D, RND, 4>(a, grid, st);
   }
 }
 
 template <int D>
 cudaError_t dec_launch(const DecArgs& a, int rnd, cudaStream_t st) {
   const dim3 grid((unsigned)a.n_ch, (unsigned)(a.p.B * a.p.H));
-  const size_t smem1 = dec_scores_smem<D>();
   cudaError_t e;
-  if (rnd == kRndFast) {
-    e = cudaFuncSetAttribute(dec_scores_kernel<D, kRndFast>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-    if (e == cudaSuccess) dec_scores_kernel<D, kRndFast><<<grid, DC_T, smem1, st>>>(a);
-  } else if (rnd == kRndNone) {
-    e = cudaFuncSetAttribute(dec_scores_kernel<D, kRndNone>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-    if (e == cudaSuccess) dec_scores_kernel<D, kRndNone><<<grid, DC_T, smem1, st>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(dec_scores_kernel<D, kRndExact>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-    if (e == cudaSuccess) dec_scores_kernel<D, kRndExact><<<grid, DC_T, smem1, st>>>(a);
-  }
+  if (rnd == kRndFast) e = dec_launch_rnd<D, kRndFast>(a, grid, st);
+  else if (rnd == kRndNone) e = dec_launch_rnd<D, kRndNone>(a, grid, st);
+  else e = dec_launch_rnd<D, kRndExact>(a, grid, st);
   if (e != cudaSuccess) return e;
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (a.p.variant == LAMP_STRICT) dec_select_kernel<D, LAMP_STRICT><<<grid, DC_T, 0, st>>>(a, rnd);
-  else if (a.p.variant == LAMP_RELAXED) dec_select_kernel<D, LAMP_RELAXED><<<grid, DC_T, 0, st>>>(a, rnd);
-  else dec_select_kernel<D, LAMP_GIVEN_MASK><<<grid, DC_T, 0, st>>>(a, rnd);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dec_combine_kernel<D><<<(unsigned)(a.p.B * a.p.H * a.p.n_q), D, 0, st>>>(a);
+  if (a.p.variant == LAMP_STRICT) dec_select_kernel<D, LAMP_STRICT><<<grid, DC_T, 0, st>>>(a);
+  else if (a.p.variant == LAMP_RELAXED) dec_select_kernel<D, LAMP_RELAXED><<<grid, DC_T, 0, st>>>(a);
+  else dec_select_kernel<D, LAMP_GIVEN_MASK><<<grid, DC_T, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -462,12 +567,12 @@ cudaError_t dec_launch(const DecArgs& a, int rnd, cudaStream_t st) {
 cudaError_t launch_decode(const Problem& p, const Workspace& ws, char* base, cudaStream_t st) {
   DecArgs a;
   a.p = p;
-  a.stats = reinterpret_cast<const int*>(base + ws.stats);
-  a.nchunk = ws.nchunk;
   a.n_ch = ws.dec_chunks;
   a.scores = reinterpret_cast<float*>(base + ws.dec_scores);
   a.cstat = reinterpret_cast<DecStat*>(base + ws.dec_stat);
   a.part = reinterpret_cast<float*>(base + ws.dec_part);
+  a.cfast = reinterpret_cast<int*>(base + ws.dec_flag);
+  a.rowdone = reinterpret_cast<unsigned*>(base + ws.dec_done);
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
   return p.d == 64 ? dec_launch<64>(a, rnd, st) : dec_launch<128>(a, rnd, st);
 }

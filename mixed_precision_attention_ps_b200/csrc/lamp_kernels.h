@@ -55,6 +55,8 @@ struct Workspace {
   size_t dec_scores;   // decode: fp32 low-precision scores [B*H][n_q][dec_chunks * 512]
   size_t dec_stat;     // decode: per (row, chunk) maximum, first argmax, S_rest (16 bytes)
   size_t dec_part;     // decode: per (row, chunk) softmax maximum, normaliser, partial output [2 + d] f32
+  size_t dec_flag;     // decode: per (b, h, chunk) int, the chunk's products are exact
+  size_t dec_done;     // decode: per row, chunks whose partials are written (the last one combines)
 };
 
 // Strict / given-mask configuration: rows per work item and threads.

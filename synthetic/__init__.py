@@ -204,5 +204,7 @@ WORKLOADS = {
     "long_1x32x16384x128": Workload(1, 32, 16384, 16384, 128),
     # a smaller case of the streamed relaxed kernel, sized for profiling captures
     "long_1x8x4096x128": Workload(1, 8, 4096, 4096, 128),
+    # decode: one new query per head against a 16K-token key/value cache
+    "decode_1x32x1x16384x128": Workload(1, 32, 1, 16384, 128),
     "outlier_4x25x4096x64": Workload(4, 25, 4096, 4096, 64, outlier_frac=0.01),
 }

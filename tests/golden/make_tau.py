@@ -39,6 +39,8 @@ PLAN = [
     ("batch8_8x25x1024x64", oracle.RELAXED, [4], [0.016], None),
     ("long_1x32x16384x128", oracle.RELAXED, [4], [0.01], 768),
     ("long_1x8x4096x128", oracle.RELAXED, [4], [0.01], None),
+    ("decode_1x32x1x16384x128", oracle.STRICT, [4], [0.016], None),
+    ("decode_1x32x1x16384x128", oracle.RELAXED, [4], [0.01], None),
     ("outlier_4x25x4096x64", oracle.STRICT, [4, 6], [0.003, 0.076], None),
 ]
 
