@@ -303,7 +303,7 @@ __device__ __forceinline__ float dec_recompute(const float* qf, const uint16_t* 
 
 template <int D, int VAR>
 __global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a) {
-  constexpr int G = DC_T / (D / 2);  // key groups of the partial P.V
+  constexpr int G = DC_T / (D / 8);  // key groups of the partial P.V (a thread: 8 value columns)
   __shared__ float ys[DC_CK];        // mixed scores of the chunk (current row)
   __shared__ float ps[DC_CK];        // softmax numerators against the chunk maximum
   __shared__ float qf[D];            // the current row of Q, binary32
@@ -447,32 +447,31 @@ __global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a) {
     ps[t + DC_T] = p1;
     const float lc = block_sum_f(p0 + p1, redf);  // its barriers also publish ps
     // partial output: key group gq of thread t takes keys gq, gq + G, ... and the
-    // value columns 2 dp, 2 dp + 1
+    // value columns 8 dq .. 8 dq + 7 (one 16-byte load per key)
     {
-      const int dp = t % (D / 2), gq = t / (D / 2);
+      const int dq = t % (D / 8), gq = t / (D / 8);
       const int kend = min(DC_CK, nv - k0);
-      const uint32_t* vcol = reinterpret_cast<const uint32_t*>(Vh + (size_t)k0 * D) + dp;
-      float o0 = 0.f, o1 = 0.f;
-      // eight independent loads in flight per thread (V is read once: HBM bound)
-      int j = gq;
-      for (; j + 7 * G < kend; j += 8 * G) {
-        uint32_t v2[8];
+      const uint4* vcol = reinterpret_cast<const uint4*>(Vh + (size_t)k0 * D) + dq;
+      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      auto add = [&](float pj, uint4 v) {
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v2[u] = __ldg(vcol + (size_t)(j + u * G) * (D / 2));
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float pj = ps[j + u * G];
-          o0 = fmaf(pj, bf16_lo(v2[u]), o0);
-          o1 = fmaf(pj, bf16_hi(v2[u]), o1);
+        for (int e = 0; e < 4; ++e) {
+          o[2 * e] = fmaf(pj, bf16_lo(w4[e]), o[2 * e]);
+          o[2 * e + 1] = fmaf(pj, bf16_hi(w4[e]), o[2 * e + 1]);
         }
+      };
+      int j = gq;
+      for (; j + 3 * G < kend; j += 4 * G) {  // four 16-byte loads in flight per thread
+        uint4 v4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v4[u] = __ldg(vcol + (size_t)(j + u * G) * (D / 8));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) add(ps[j + u * G], v4[u]);
       }
-      for (; j < kend; j += G) {
-        const uint32_t v2 = __ldg(vcol + (size_t)j * (D / 2));
-        o0 = fmaf(ps[j], bf16_lo(v2), o0);
-        o1 = fmaf(ps[j], bf16_hi(v2), o1);
-      }
-      ro[gq][2 * dp] = o0;
-      ro[gq][2 * dp + 1] = o1;
+      for (; j < kend; j += G) add(ps[j], __ldg(vcol + (size_t)j * (D / 8)));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ro[gq][8 * dq + e] = o[e];
     }
     __syncthreads();
     float* pr = a.part + (row * a.n_ch + c) * (2 + D);
