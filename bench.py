@@ -42,9 +42,6 @@ UNIT = "G-scores/s"
 TAU_FILE = os.path.join(ROOT, "tests", "golden", "tau.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["lamp_ws.cu", "lamp_ws_common.cuh", "lamp_stream.cu", "lamp_rows.cu", "lamp_strict.cu",
-                  "lamp_prep.cu", "lamp_device.cuh",
-                  "lamp_kernels.h"]
 L2_FLUSH_BYTES = 256 << 20
 N_SM = 148
 FP32_LANES_PER_SM_CLK = 128
@@ -214,23 +211,25 @@ def run_reference(a, w, variant, mu, tau, cfg):
 # ----------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------
-def kernel_source_hash() -> str:
+def source_hash(files) -> str:
+    """Hash of the named csrc files: a traffic figure is valid only for the sources it
+    was measured on."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files:
         h.update(open(os.path.join(ROOT, "mixed_precision_attention_ps_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_bytes(workload: str, variant: int, mu: int) -> float | None:
-    """DRAM bytes per launch of the row kernel from the committed ncu summary, or
-    None when the kernel sources changed since that capture."""
+    """DRAM bytes per launch of the measured kernel from the committed ncu summary,
+    or None when that kernel's sources changed since the capture."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     doc = json.load(open(TRAFFIC_FILE))
-    if doc.get("kernel_source_hash") != kernel_source_hash():
-        return None
     for e in doc.get("entries", []):
         if e["workload"] == workload and e["variant"] == variant and e["mu"] == mu:
+            if source_hash(e["sources"]) != e["source_hash"]:
+                return None
             return float(e["dram_bytes_per_launch"])
     return None
 
