@@ -90,6 +90,29 @@ def is_decode(w) -> bool:
     return w.n_q <= 4 and w.n_k >= 512
 
 
+def rank_workload(w, rank: int):
+    """Weak scaling: every rank runs the same shape on its own inputs (seed + rank)."""
+    return S.Workload(w.B, w.H, w.n_q, w.n_k, w.d, w.causal, w.outlier_frac, w.outlier_scale, seed=w.seed + rank)
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of a few floats over all ranks (the step time of a job is
+    its slowest rank's). Single process: the values themselves."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_value(world: int, valid_per_rank: int, ms: float) -> float:
+    """Whole-job throughput in G-scores/s: every rank's scores over the slowest rank's time."""
+    return world * valid_per_rank / (ms * 1e-3) / 1e9
+
+
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
 
@@ -284,7 +307,7 @@ def run_ours(a, w, variant, mu, tau, cfg):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     lamp.load()
-    wr = S.Workload(w.B, w.H, w.n_q, w.n_k, w.d, w.causal, w.outlier_frac, w.outlier_scale, seed=w.seed + rank)
+    wr = rank_workload(w, rank)
     Q, K, V = S.make_qkv(wr)
 
     def dev_t(x):
@@ -328,11 +351,7 @@ def run_ours(a, w, variant, mu, tau, cfg):
         dist.barrier()
     clk = clocks.stop()
     times = [s.elapsed_time(e) for s, e in evs]
-    ms = statistics.mean(times)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([statistics.mean(times)], dev)[0]
     launches_per_step = 4 if is_decode(w) else 2  # exponent statistics + row kernel (decode: + 3)
 
     # ---- end to end through the C ABI with host buffers ---------------------------------
@@ -418,18 +437,16 @@ def run_ours(a, w, variant, mu, tau, cfg):
         ms_e2e = t0.elapsed_time(t1) / e2e_steps
         # the pipelined outputs equal the device-resident call's
         assert torch.equal(hout[(e2e_steps - 1) & 1], out.view(torch.int16).cpu())
+    ms_e2e, ms_serial = max_over_ranks([ms_e2e, ms_serial], dev)
     if world > 1:
-        t = torch.tensor([ms_e2e, ms_serial], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e, ms_serial = float(t[0].item()), float(t[1].item())
         dist.barrier()
     h2d = Q.nbytes + K.nbytes + V.nbytes
     d2h = out.numel() * 2 + mask.numel() * 4
 
     result = None
     if rank == 0:
-        value = world * valid / (ms * 1e-3) / 1e9
-        value_e2e = world * valid / (ms_e2e * 1e-3) / 1e9
+        value = job_value(world, valid, ms)
+        value_e2e = job_value(world, valid, ms_e2e)
         # roofline: ALU issue. 4 d lane-ops per valid score (1 multiply-add + 3 integer
         # ops of the round-to-nearest-even to mu bits, per accumulation step), against
         # 128 FP32/INT32 lanes per SM per clock x 148 SMs x the maximum SM clock.
