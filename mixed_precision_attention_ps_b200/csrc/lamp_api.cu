@@ -222,9 +222,22 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
     return w;
   }
   w.use_ws = ws_fits(p.d, p.n_k, smem_optin) ? 1 : 0;
-  // the relaxed and given-mask tests need no whole row: rows too long for the
-  // whole-row kernel stream through 512-key tiles instead
-  w.use_stream = (!w.use_ws && p.variant != LAMP_STRICT && stream_smem_bytes(p.d) + kStaticSmemReserve <= smem_optin) ? 1 : 0;
+  // rows too long for the whole-row kernel stream through 512-key tiles instead
+  w.use_stream = (!w.use_ws && stream_smem_bytes(p.d) + kStaticSmemReserve <= smem_optin) ? 1 : 0;
+  if (w.use_stream && p.variant == LAMP_STRICT) {
+    // strict rows take two passes over a score slab in HBM (the strict test needs
+    // the whole row's statistics before it selects anything); past the slab cap
+    // the row kernels serve them
+    const size_t slab = (size_t)BH * p.n_q * stream_slab_ld(p.n_k) * 4;
+    if (slab > kStrictSlabCap) {
+      w.use_stream = 0;
+    } else {
+      w.st_slab = off;
+      off = align256(off + slab);
+      w.st_rows = off;
+      off = align256(off + (size_t)BH * p.n_q * 16);
+    }
+  }
   w.rows_bm = (w.use_ws || w.use_stream) ? 0 : rows_pick_bm(p.d, p.n_k, smem_optin);
   if (!w.use_ws && !w.use_stream && !w.rows_bm && strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
     const long long n_items = (long long)((p.n_q + kStrictBM - 1) / kStrictBM) * BH;

@@ -51,6 +51,8 @@ struct Workspace {
   int use_ws;          // 1: warp-specialised kernel (two 16-row buffers fit on chip)
   int use_stream;      // 1: streamed one-pass kernel (relaxed / given mask, rows too long for use_ws)
   int use_decode;      // 1: split-key decode kernels (few query rows, long rows)
+  size_t st_slab;      // strict rows on the streamed kernel: low-precision score slab [B*H][n_q][ld] f32
+  size_t st_rows;      // ... and per-row statistics (maximum, first argmax, S_rest), 16 bytes each
   int dec_chunks;      // decode: 512-key chunks per row
   size_t dec_scores;   // decode: fp32 low-precision scores [B*H][n_q][dec_chunks * 512]
   size_t dec_stat;     // decode: per (row, chunk) maximum, first argmax, S_rest (16 bytes)
@@ -80,7 +82,9 @@ cudaError_t launch_decode(const Problem& p, const Workspace& ws, char* base, cud
 constexpr int kDecodeMaxQ = 4;       // query rows per (b, h) the decode kernels take
 constexpr int kDecodeMinKeys = 512;  // shortest rows routed to them
 constexpr int kDecodeChunk = 512;    // keys per chunk (one CTA)
+constexpr size_t kStrictSlabCap = (size_t)8 << 30;  // largest score slab of the two-pass strict rows
 size_t stream_smem_bytes(int d);
+size_t stream_slab_ld(int n_k);  // slab row stride: keys rounded up to whole 512-key tiles
 int rows_nkp(int bm, int n_k);
 size_t rows_smem_bytes(int d, int bm, int n_k);
 cudaError_t launch_ps_round(const float* x, float* y, size_t n, int mu, int path, cudaStream_t st);

@@ -60,12 +60,31 @@ __host__ __device__ inline StSmem st_plan() {
   return s;
 }
 
+// Strict rows too long for whole-row buffers run in two passes of this kernel
+// (template parameter PH):
+//   PH 0: one pass (relaxed, given mask);
+//   PH 1: strict statistics: the producers compute the scores; the consumers store
+//         every tile to an HBM score slab and keep, per row, the maximum m, its
+//         first key am and S_rest = sum over the other keys of exp(y - m) online
+//         across tiles (tile maximum and sum, merged in double);
+//   PH 2: strict selection: the producers refill the tile buffers from the slab;
+//         the consumers run the strict test with the row statistics of pass 1,
+//         then recompute, online softmax and P.V as in PH 0.
+struct RowStat {
+  float m;      // maximum of the row's low-precision scores (-inf if none valid)
+  int am;       // its first key
+  double srest; // sum over the other keys of exp(y - m)
+};
+
 struct StArgs {
   Problem p;
   const int* stats;  // per-(b, h) exponent statistics
   int nchunk;
   int n_items;
   int n_rb;
+  float* slab;       // strict: low-precision scores [B*H][n_q][ld]
+  size_t ld;         // slab row stride (keys rounded up to whole tiles)
+  RowStat* rows;     // strict: [B*H][n_q]
 };
 
 __device__ __forceinline__ int st_ntiles(int kv_end) { return kv_end > 0 ? (kv_end + ST_T - 1) / ST_T : 1; }
@@ -73,7 +92,7 @@ __device__ __forceinline__ int st_ntiles(int kv_end) { return kv_end > 0 ? (kv_e
 // ---------------------------------------------------------------------------
 // Producers: every tile of every item, in the order the consumers take them.
 // ---------------------------------------------------------------------------
-template <int D, int RND>
+template <int D, int RND, int PH>
 __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem, const StSmem& L, int warp,
                                             int lane) {
   const Problem& p = a.p;
@@ -105,9 +124,26 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
         return;
       }
       float* tile = reinterpret_cast<float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
-      ws_produce_tile<D, RND>(p, it, t0, tlen, sQ, tile, ST_TS, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
-                              Kh, negc, pow2s, scale2, s);
-      deal = (deal + (tlen + WS_UNIT - 1) / WS_UNIT) % WS_NP;
+      if (PH == 2) {
+        // the tile's scores from the slab: rows of the item by cp.async, keys of the
+        // tile that the scores pass wrote; rows past the item hold -inf
+        const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;
+        const int per_row = written / 4;  // 16-byte pieces
+        for (int u = warp * 32 + lane; u < WS_BM * per_row; u += WS_NP * 32) {
+          const int r = u / per_row, c4 = u % per_row;
+          float* dst = tile + (size_t)r * ST_TS + 4 * c4;
+          if (r < it.rows)
+            cp_async16(dst, a.slab + ((size_t)it.bh * p.n_q + it.i0 + r) * a.ld + t0 + 4 * c4);
+          else
+            *reinterpret_cast<float4*>(dst) = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+      } else {
+        ws_produce_tile<D, RND>(p, it, t0, tlen, sQ, tile, ST_TS, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
+                                Kh, negc, pow2s, scale2, s);
+        deal = (deal + (tlen + WS_UNIT - 1) / WS_UNIT) % WS_NP;
+      }
       mbar_arrive(bars + buf);  // this thread's scores of the tile are in place
     }
   }
@@ -116,7 +152,7 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
 // ---------------------------------------------------------------------------
 // Consumers: selection, recompute, online softmax and P.V, tile by tile.
 // ---------------------------------------------------------------------------
-template <int D, int RND, int VAR>
+template <int D, int RND, int VAR, int PH>
 __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem, const StSmem& L, int cw,
                                             int lane) {
   constexpr int NH = D / 64;
@@ -171,10 +207,26 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
     }
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     SelRows S;
+    int am_abs[2] = {0x7FFFFFFF, 0x7FFFFFFF};  // strict: first key of each row's maximum
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
       S.live[tt] = rr_[tt] < it.rows;
       S.mrun[tt] = -INFINITY;
+      if (VAR == LAMP_STRICT) {  // the row statistics of the scores pass
+        RowStat rs;
+        rs.m = -INFINITY;
+        rs.am = 0x7FFFFFFF;
+        rs.srest = 0.0;
+        if (rr_[tt] < it.rows) rs = a.rows[grow[tt]];
+        am_abs[tt] = rs.am;
+        S.m[tt] = rs.m;
+        S.srest[tt] = rs.srest;
+        S.Sd[tt] = 1.0 + rs.srest;
+        S.Sf[tt] = (float)S.Sd[tt];
+        S.srest_f[tt] = (float)rs.srest;
+        S.c2[tt] = (float)(2.0 / (S.Sd[tt] * S.Sd[tt]));
+        S.mL[tt] = rs.m * kLog2e;
+      }
     }
     float acc[8][4];
 #pragma unroll
@@ -232,6 +284,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         S.nv[tt] = nvr[tt];
         S.word0[tt] = grow[tt] * nwords + (t0 >> 5);
         S.mx[tt] = -INFINITY;
+        if (VAR == LAMP_STRICT) S.am[tt] = am_abs[tt] == 0x7FFFFFFF ? 0x7FFFFFFF : am_abs[tt] - t0;
       }
       for (int i4 = 0; i4 < nit; ++i4)
         sel_step<VAR>(p, S, 128 * i4, written, nwords - (t0 >> 5), tlo, thi, lane, wbuf, nsel);
@@ -370,7 +423,117 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
 }
 
-template <int D, int RND, int VAR>
+// Pass 1 of the strict rows: every tile stored to the slab, and per row the
+// maximum, its first key and S_rest kept online across the tiles. A tile's
+// maximum and first key come from warp reductions and its sum of exp(y - tile
+// maximum) over the other keys from binary32 expf terms summed in double; the
+// merge is exact in double: a larger tile maximum rescales the running sum by
+// exp(m_old - m_new) with the old maximum joining it as a term 1, a smaller or
+// equal one adds (tile sum + 1) exp(m_tile - m).
+template <int D>
+__device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char* smem, const StSmem& L, int cw,
+                                                  int lane) {
+  constexpr int NCT = WS_NC * 32;
+  const Problem& p = a.p;
+  const int tidc = cw * 32 + lane;
+  const int G = gridDim.x, cta = blockIdx.x;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  float* qbase = reinterpret_cast<float*>(smem + L.q);
+  for (int k0 = 0; k0 < 2; ++k0) {
+    const int q0 = ws_item(k0, cta, G, a.n_items);
+    if (q0 < 0) break;
+    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), tidc, NCT);
+  }
+  mbar_arrive(bars + 2);
+  mbar_arrive(bars + 3);
+  int k = 0;
+  for (int ii = 0;; ++ii) {
+    const int q = ws_item(ii, cta, G, a.n_items);
+    if (q < 0) break;
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    float* sQ = qbase + (ii & 1) * ws_qfloats<D>();
+    const int nt = st_ntiles(it.kv_end);
+    int rr_[2];
+    size_t grow[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      rr_[t] = 2 * cw + t;
+      grow[t] = (size_t)it.bh * p.n_q + it.i0 + rr_[t];
+    }
+    float M[2] = {-INFINITY, -INFINITY};
+    int AM[2] = {0x7FFFFFFF, 0x7FFFFFFF};
+    double Sacc[2] = {0.0, 0.0};
+    for (int t = 0; t < nt; ++t, ++k) {
+      const int buf = k & 1;
+      const int t0 = t * ST_T;
+      const int tlen = max(0, min(ST_T, it.kv_end - t0));
+      const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;
+      const float* tile = reinterpret_cast<const float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
+      const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
+      if (named_or(BAR_CONS, NCT, !ok)) {
+        ws_timeout(p);
+        return;
+      }
+      const int nit = (written + 127) >> 7;
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        const float* row = tile + (size_t)rr_[tt] * ST_TS;
+        if (rr_[tt] < it.rows) {
+          float* dst = a.slab + grow[tt] * a.ld + t0;
+          for (int j0 = 4 * lane; j0 < written; j0 += 128)
+            *reinterpret_cast<float4*>(dst + j0) = *reinterpret_cast<const float4*>(row + j0);
+        }
+        float lm = -INFINITY;
+        int li = 0x7FFFFFFF;
+        for (int i4 = 0; i4 < nit; ++i4) {
+          const int j0 = 128 * i4 + 4 * lane;
+          const float4 v = lds4_or_ninf(row + j0, j0 < written);
+          if (v.x > lm) { lm = v.x; li = j0; }
+          if (v.y > lm) { lm = v.y; li = j0 + 1; }
+          if (v.z > lm) { lm = v.z; li = j0 + 2; }
+          if (v.w > lm) { lm = v.w; li = j0 + 3; }
+        }
+        const float mt = warp_max_redux(lm);
+        if (mt > -INFINITY) {  // warp-uniform
+          const int at = t0 + __reduce_min_sync(0xFFFFFFFFu, lm == mt ? li : 0x7FFFFFFF);
+          double sl = 0.0;
+          for (int i4 = 0; i4 < nit; ++i4) {
+            const int j0 = 128 * i4 + 4 * lane;
+            const float4 v = lds4_or_ninf(row + j0, j0 < written);
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (t0 + j0 + e != at) sl += (double)expf(__fsub_rn(vv[e], mt));
+          }
+          const double st = warp_sum_d(sl);
+          if (mt > M[tt]) {
+            Sacc[tt] = M[tt] > -INFINITY ? (Sacc[tt] + 1.0) * exp((double)M[tt] - (double)mt) + st : st;
+            M[tt] = mt;
+            AM[tt] = at;
+          } else {
+            Sacc[tt] += (st + 1.0) * exp((double)mt - (double)M[tt]);
+          }
+        }
+      }
+      if (t == nt - 1) {  // end of the item: the row statistics, then Q of item + 2
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+          if (lane == 0 && rr_[tt] < it.rows) {
+            RowStat rs;
+            rs.m = M[tt];
+            rs.am = AM[tt];
+            rs.srest = Sacc[tt];
+            a.rows[grow[tt]] = rs;
+          }
+        const int q2 = ws_item(ii + 2, cta, G, a.n_items);
+        if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
+      }
+      mbar_arrive(bars + 2 + buf);  // tile buffer free (and, after an item's last tile, Q of item + 2 staged)
+    }
+  }
+}
+
+template <int D, int RND, int VAR, int PH>
 __global__ void __launch_bounds__(WS_NP * 32 + WS_NC * 32, 1) st_kernel(const StArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const StSmem L = st_plan<D>();
@@ -384,13 +547,14 @@ __global__ void __launch_bounds__(WS_NP * 32 + WS_NC * 32, 1) st_kernel(const St
     mbar_fence_init();
   }
   __syncthreads();
-  if (warp < WS_NP) st_producer<D, RND>(a, smem, L, warp, lane);
-  else st_consumer<D, RND, VAR>(a, smem, L, warp - WS_NP, lane);
+  if (warp < WS_NP) st_producer<D, RND, PH>(a, smem, L, warp, lane);
+  else if (PH == 1) st_consumer_stats<D>(a, smem, L, warp - WS_NP, lane);
+  else st_consumer<D, RND, VAR, PH>(a, smem, L, warp - WS_NP, lane);
 }
 
-template <int D, int RND, int VAR>
+template <int D, int RND, int VAR, int PH>
 cudaError_t st_launch_one(const StArgs& a, int grid, cudaStream_t st) {
-  auto k = st_kernel<D, RND, VAR>;
+  auto k = st_kernel<D, RND, VAR, PH>;
   const size_t smem = (size_t)st_plan<D>().total;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -400,11 +564,17 @@ cudaError_t st_launch_one(const StArgs& a, int grid, cudaStream_t st) {
 
 template <int D, int RND>
 cudaError_t st_launch_var(const StArgs& a, int grid, cudaStream_t st) {
-  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK>(a, grid, st);
-  return st_launch_one<D, RND, LAMP_RELAXED>(a, grid, st);
+  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK, 0>(a, grid, st);
+  if (a.p.variant == LAMP_RELAXED) return st_launch_one<D, RND, LAMP_RELAXED, 0>(a, grid, st);
+  // strict: the scores-and-statistics pass, then the selection pass
+  cudaError_t e = st_launch_one<D, RND, LAMP_STRICT, 1>(a, grid, st);
+  if (e != cudaSuccess) return e;
+  return st_launch_one<D, RND, LAMP_STRICT, 2>(a, grid, st);
 }
 
 }  // namespace
+
+size_t stream_slab_ld(int n_k) { return (size_t)((n_k + ST_T - 1) / ST_T) * ST_T; }
 
 size_t stream_smem_bytes(int d) { return d == 64 ? (size_t)st_plan<64>().total : (size_t)st_plan<128>().total; }
 
@@ -415,6 +585,9 @@ cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int
   a.nchunk = ws.nchunk;
   a.n_rb = (p.n_q + WS_BM - 1) / WS_BM;
   a.n_items = a.n_rb * p.B * p.H;
+  a.slab = reinterpret_cast<float*>(base + ws.st_slab);
+  a.ld = stream_slab_ld(p.n_k);
+  a.rows = reinterpret_cast<RowStat*>(base + ws.st_rows);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
   if (p.d == 64) {
