@@ -79,7 +79,8 @@ enum lamp_status {
   LAMP_ERR_ARG = -1,          /* null required pointer, mu outside [1,23], tau NaN,
                                  unknown variant, a dimension <= 0, scale <= 0 or NaN */
   LAMP_ERR_UNSUPPORTED = -2,  /* d not in {64, 128}; pointer not 16-byte aligned;
-                                 strict/given-mask with n_k > LAMP_MAX_STRICT_NK;
+                                 a problem only the row kernels can serve (see
+                                 LAMP_MAX_STRICT_NK) with n_k > LAMP_MAX_STRICT_NK;
                                  B * H > 65535 */
   LAMP_ERR_WORKSPACE = -3,    /* workspace given but smaller than lamp_workspace_size() */
   LAMP_ERR_CUDA = -4,         /* a CUDA call failed (allocation, launch); see lamp_last_error() */
@@ -87,8 +88,12 @@ enum lamp_status {
   LAMP_ERR_CHECK = -6         /* reserved: a device-side check failed (reported via status_out) */
 };
 
-/* Largest n_k accepted by the strict and given-mask variants (their softmax
- * needs the whole row of scores before any probability is known). */
+/* Largest n_k of the row kernels. Relaxed and given-mask rows of any length
+ * stream through 512-key tiles, decode rows (n_q <= 4) split their keys, and
+ * strict rows longer than 1024 keys take two streamed passes over a score slab
+ * of B*H*n_q*ceil(n_k/512)*512*4 bytes in the workspace. Only a strict problem
+ * whose slab would pass 8 GiB falls to the row kernels, which need
+ * n_k <= LAMP_MAX_STRICT_NK (else LAMP_ERR_UNSUPPORTED). */
 #define LAMP_MAX_STRICT_NK 65536
 
 typedef struct {

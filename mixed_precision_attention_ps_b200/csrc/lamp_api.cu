@@ -108,8 +108,6 @@ int check_args(const lamp_args* a) {
   if (std::isnan(a->scale) || a->scale < 0.f || std::isinf(a->scale))
     return fail(LAMP_ERR_ARG, "scale must be 0 (default) or a positive finite value");
   if (d.d != 64 && d.d != 128) return fail(LAMP_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d.d);
-  if (a->variant != LAMP_RELAXED && d.n_k > LAMP_MAX_STRICT_NK)
-    return fail(LAMP_ERR_UNSUPPORTED, "strict/given-mask variants support n_k <= %d", LAMP_MAX_STRICT_NK);
   const long long rows = (long long)d.B * d.H * d.n_q;
   if ((long long)d.B * d.H > 65535 || rows > (1LL << 40))
     return fail(LAMP_ERR_UNSUPPORTED, "problem too large for the index space");
@@ -251,6 +249,20 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
 
 }  // namespace lamp
 
+// The plan's kernels must be able to serve the problem: the row kernels (strict
+// problems whose score slab would pass its cap) take rows of at most
+// LAMP_MAX_STRICT_NK keys and need their shared-memory rows or row slab.
+int check_plan(const lamp::Problem& p, const lamp::Workspace& ws, const DeviceInfo& info) {
+  if (ws.use_decode || ws.use_ws || ws.use_stream) return LAMP_OK;
+  if (p.n_k > LAMP_MAX_STRICT_NK)
+    return fail(LAMP_ERR_UNSUPPORTED,
+                "rows of %d keys: past the streamed kernel's score-slab cap the row kernels take n_k <= %d",
+                p.n_k, LAMP_MAX_STRICT_NK);
+  if (!ws.rows_bm && lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
+    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
+  return LAMP_OK;
+}
+
 extern "C" {
 
 const char* lamp_last_error(void) { return g_err; }
@@ -279,9 +291,8 @@ int lamp_attention_ex(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (!ws.use_decode && !ws.use_ws && !ws.use_stream && !ws.rows_bm &&
-      lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
-    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
+  rc = check_plan(p, ws, info);
+  if (rc != LAMP_OK) return rc;
   if (a->workspace && a->workspace_bytes < ws.total)
     return fail(LAMP_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu bytes needed",
                 a->workspace_bytes, ws.total);
@@ -314,9 +325,8 @@ int lamp_attention_noalloc(const lamp_args* a) {
   if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   lamp::Problem p = make_problem(a);
   lamp::Workspace ws = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
-  if (!ws.use_decode && !ws.use_ws && !ws.use_stream && !ws.rows_bm &&
-      lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
-    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
+  rc = check_plan(p, ws, info);
+  if (rc != LAMP_OK) return rc;
   if (ws.total > (size_t)LAMP_NOALLOC_SCRATCH_BYTES)
     return fail(LAMP_ERR_WORKSPACE,
                 "this problem needs %zu bytes of scratch, more than the %u bytes lamp_attention_noalloc "

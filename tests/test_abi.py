@@ -65,7 +65,6 @@ def call_ex(**kw):
     (dict(dims=(0, 1, 128, 128, 64)), lamp.LAMP_ERR_ARG, "positive"),
     (dict(dims=(1, 1, 128, -1, 64)), lamp.LAMP_ERR_ARG, "positive"),
     (dict(dims=(1, 1, 128, 128, 96)), lamp.LAMP_ERR_UNSUPPORTED, "d must be"),
-    (dict(dims=(1, 1, 128, 70000, 64)), lamp.LAMP_ERR_UNSUPPORTED, "n_k"),
     (dict(Q=FAKE + 8), lamp.LAMP_ERR_UNSUPPORTED, "16-byte"),
     (dict(out_f32=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
     (dict(n_selected_out=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),

@@ -103,3 +103,34 @@ def test_outlier_4x25x4096_relaxed_sampled():
     w = S.WORKLOADS["outlier_4x25x4096x64"]
     rows = P.sample_rows(w, 6, 5, seed=15)
     run_case(w, 4, 0.3, oracle.RELAXED, rows=rows)
+
+
+@pytest.mark.parametrize("n_q,variant", [
+    (20, oracle.STRICT),      # two streamed passes over the score slab
+    (20, oracle.GIVEN_MASK),  # one streamed pass with a caller-given mask
+    (3, oracle.STRICT),       # decode rows: the keys split over chunks
+])
+def test_rows_longer_than_the_row_kernel_limit(n_q, variant):
+    """Rows past LAMP_MAX_STRICT_NK keys: only the row kernels are limited."""
+    n_k = lamp.LAMP_MAX_STRICT_NK + 4501
+    w = S.Workload(1, 1, n_q, n_k, 64, causal=True, seed=16 + n_q)
+    mask = None
+    if variant == oracle.GIVEN_MASK:
+        rng = np.random.default_rng(16)
+        nv = np.array([w.valid_keys(i) for i in range(w.n_q)])
+        mask = S.random_control_mask(w, rng.integers(0, nv // 50 + 1)[None, :]).reshape(1, 1, n_q, -1)
+    g, orc, _ = run_case(w, 4, 2e-4, variant, mask_in=mask)  # z is about 1/4600 at the row maximum
+    assert g.count() == int(orc.nsel.sum()) > 0
+
+
+def test_row_kernel_limit_is_reported_before_any_launch():
+    """A strict problem whose score slab would pass 8 GiB falls to the row
+    kernels, which take at most LAMP_MAX_STRICT_NK keys: the call fails with
+    LAMP_ERR_UNSUPPORTED at planning time (the fake pointers are never used)."""
+    fake = 1 << 20
+    n_k = lamp.LAMP_MAX_STRICT_NK + 4464
+    rc = lamp.lamp_attention_ex(dims=(1, 1, 32768, n_k, 64), Q=fake, K=fake, V=fake, out=fake, mu=4,
+                                tau=0.05, variant=lamp.LAMP_STRICT, causal=1, check=False)
+    assert rc == lamp.LAMP_ERR_UNSUPPORTED and "row kernels" in lamp.lamp_last_error()
+    # the relaxed variant streams the same rows
+    assert lamp.lamp_workspace_size((1, 1, 32768, n_k, 64), lamp.LAMP_RELAXED) > 0
