@@ -1,4 +1,5 @@
-"""ctypes binding of the CPU oracle (``lamp_oracle.c``).
+"""ctypes binding of the CPU oracle (``lamp_oracle.c``: attention;
+``lamp_oracle_act.c``: GELU after a PS(mu) linear map).
 
 Test infrastructure only: the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline / reference legs use it; the CUDA library and its
@@ -17,7 +18,7 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "lamp_oracle.c")
+_SRCS = [os.path.join(_HERE, "lamp_oracle.c"), os.path.join(_HERE, "lamp_oracle_act.c")]
 _LIB = os.path.join(_HERE, "liblamp_oracle.so")
 _CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c99"]
 
@@ -28,9 +29,9 @@ _lib = None
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (plain C, no contraction of a*b+c)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(f) for f in _SRCS):
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        subprocess.run(["gcc", *_CFLAGS, *_SRCS, "-o", tmp, "-lm"], check=True)
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -63,6 +64,13 @@ def lib():
             L.lamp_oracle_row_kl.argtypes = [P, P, ctypes.c_int]
             L.lamp_oracle_kl_rows.restype = None
             L.lamp_oracle_kl_rows.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64, P]
+            L.lamp_oracle_gelu.restype = ctypes.c_double
+            L.lamp_oracle_gelu.argtypes = [ctypes.c_double]
+            L.lamp_oracle_gelu_kappa.restype = ctypes.c_double
+            L.lamp_oracle_gelu_kappa.argtypes = [ctypes.c_double]
+            L.lamp_oracle_linear_gelu_rows.restype = ctypes.c_int
+            L.lamp_oracle_linear_gelu_rows.argtypes = [P, P, P, ctypes.c_float, ctypes.c_int, ctypes.c_double,
+                                                       ctypes.c_int, P, P, ctypes.c_int64, P, P, P, P, P, P]
             _lib = L
     return _lib
 
@@ -204,3 +212,101 @@ def calibrate_tau(crit: np.ndarray, n_valid_per_row, rate: float) -> float:
     if k >= vals.size:
         return -1.0
     return float(np.partition(vals, vals.size - 1 - k)[vals.size - 1 - k])
+
+
+# --------------------------------------------------------------------------------------
+# LAMP on an elementwise activation: GELU(scale * x W^T) with a PS(mu) linear map
+# --------------------------------------------------------------------------------------
+
+def gelu(y) -> np.ndarray:
+    """GELU (tanh form) in double, elementwise."""
+    y = np.asarray(y, dtype=np.float64)
+    f = np.vectorize(lambda v: lib().lamp_oracle_gelu(float(v)), otypes=[np.float64])
+    return f(y)
+
+
+def gelu_kappa(y) -> np.ndarray:
+    """Component-wise condition number |y f'(y) / f(y)| of the tanh-form GELU, in double."""
+    y = np.asarray(y, dtype=np.float64)
+    f = np.vectorize(lambda v: lib().lamp_oracle_gelu_kappa(float(v)), otypes=[np.float64])
+    return f(y)
+
+
+class ActResult:
+    """Per-row oracle outputs of LAMP GELU(scale * x W^T) for a list of rows."""
+
+    def __init__(self, nrows, N):
+        self.ps = np.empty((nrows, N), np.float32)
+        self.mixed = np.empty((nrows, N), np.float32)
+        self.kappa = np.empty((nrows, N), np.float64)
+        self.mask = np.zeros((nrows, (N + 31) // 32), np.uint32)
+        self.out = np.empty((nrows, N), np.float64)
+        self.nsel = np.zeros(nrows, np.int64)
+
+
+def linear_gelu_rows(x, W, *, scale=1.0, mu=4, tau=0.0, variant=STRICT, mask_in=None, rows=None,
+                     threads: int = 1) -> ActResult:
+    """Oracle LAMP GELU(scale * x W^T) for selected rows of x.
+
+    x: uint16 [M, K], W: uint16 [N, K] (bf16 bit patterns). variant STRICT is the
+    kappa test; GIVEN_MASK takes mask_in [M, ceil(N/32)]. rows: row ids of x, or
+    None for every row.
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("x and W disagree on K")
+    if rows is None:
+        rows = np.arange(M, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    res = ActResult(rows.size, N)
+    dims = np.array([M, N, K], dtype=np.int64)
+    if mask_in is not None:
+        mask_in = np.ascontiguousarray(mask_in, dtype=np.uint32).reshape(M, -1)
+    L = lib()
+
+    def run(lo, hi):
+        sub = slice(lo, hi)
+        rc = L.lamp_oracle_linear_gelu_rows(
+            _ptr(dims), _ptr(x), _ptr(W), float(scale), int(mu), float(tau), int(variant), _ptr(mask_in),
+            _ptr(rows[sub]), hi - lo, _ptr(res.ps[sub]), _ptr(res.mixed[sub]), _ptr(res.kappa[sub]),
+            _ptr(res.mask[sub]), _ptr(res.out[sub]), _ptr(res.nsel[sub]))
+        if rc != 0:
+            raise ValueError(f"oracle rejected its arguments (rc={rc})")
+
+    n = rows.size
+    if threads <= 1 or n < 2 * threads:
+        run(0, n)
+    else:
+        chunk = max(1, n // (threads * 4))
+        bounds = [(lo, min(n, lo + chunk)) for lo in range(0, n, chunk)]
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda b: run(*b), bounds))
+    return res
+
+
+def act_errors(out_x, y_x, out_ref, y_ref) -> dict:
+    """Errors of activation outputs against the all-FP32 ones.
+
+    l1_rel : l1 error relative to the l1 norm of the reference outputs;
+    max_rel: the largest component-wise relative output error;
+    max_amp, p99_amp: the largest (99th percentile) realised amplification of a
+             component's relative input error into its relative output error,
+             |f(y_x) - f(y)| / |f(y)| over |y_x - y| / |y|, over the components
+             whose input differs from the FP32 one (the quantity that the
+             component-wise condition number bounds to first order).
+    """
+    a = np.asarray(out_x, dtype=np.float64)
+    r = np.asarray(out_ref, dtype=np.float64)
+    yx = np.asarray(y_x, dtype=np.float64)
+    yr = np.asarray(y_ref, dtype=np.float64)
+    diff = np.abs(a - r)
+    nz = r != 0.0
+    rel = diff[nz] / np.abs(r[nz])
+    m = (yx != yr) & nz & (yr != 0.0)
+    amp = (diff[m] / np.abs(r[m])) / (np.abs(yx[m] - yr[m]) / np.abs(yr[m]))
+    return {"l1_rel": float(diff.sum() / np.abs(r).sum()), "max_rel": float(rel.max()) if rel.size else 0.0,
+            "max_amp": float(amp.max()) if amp.size else 0.0,
+            "p99_amp": float(np.percentile(amp, 99)) if amp.size else 0.0}

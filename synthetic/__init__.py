@@ -16,7 +16,8 @@ Generator (counter based, so any element can be produced on its own):
   scaled, rounded to float32, then to bfloat16 (both round-to-nearest-even).
 
 Streams: 0 = Q, 1 = K, 2 = V, 3 = outlier channel choice, 4 = random-control
-subset keys.
+subset keys, 5 = x and 6 = W of the activation workloads (GELU after a linear
+map; x is [M, K], W is [N, K] like a linear layer's weight).
 
 The workloads stand in for GPT-2 XL activations on OpenWebText (LAMP summary,
 "Experimental results"), which are not available here: iid N(0,1) entries, and
@@ -36,6 +37,7 @@ _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
 STREAM_Q, STREAM_K, STREAM_V, STREAM_OUTLIER, STREAM_RANDOM = 0, 1, 2, 3, 4
+STREAM_X, STREAM_W = 5, 6
 
 
 def mix64(z: np.ndarray) -> np.ndarray:
@@ -207,4 +209,48 @@ WORKLOADS = {
     # decode: one new query per head against a 16K-token key/value cache
     "decode_1x32x1x16384x128": Workload(1, 32, 1, 16384, 128),
     "outlier_4x25x4096x64": Workload(4, 25, 4096, 4096, 64, outlier_frac=0.01),
+}
+
+
+@dataclass(frozen=True)
+class LinearWorkload:
+    """One synthetic activation problem: GELU(scale * x W^T), x [M, K], W [N, K],
+    iid N(0,1) bf16 entries; scale = fl32(1/sqrt(K)) makes the pre-activations
+    about N(0,1)."""
+
+    M: int
+    N: int
+    K: int
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return float(np.float32(1.0 / math.sqrt(self.K)))
+
+    def outputs(self) -> int:
+        return self.M * self.N
+
+    def as_rows(self) -> Workload:
+        """The same shape as a one-head non-causal attention workload (rows of x
+        against rows of W), for the row-wise random-control masks."""
+        return Workload(1, 1, self.M, self.N, self.K, causal=False, seed=self.seed)
+
+
+def make_linear(lw: LinearWorkload) -> tuple[np.ndarray, np.ndarray]:
+    """x [M, K] and W [N, K] as uint16 bf16 bit patterns."""
+    x = to_bf16_bits(normal_f64(lw.seed, STREAM_X, 0, lw.M * lw.K)).reshape(lw.M, lw.K)
+    W = to_bf16_bits(normal_f64(lw.seed, STREAM_W, 0, lw.N * lw.K)).reshape(lw.N, lw.K)
+    return x, W
+
+
+def linear_random_mask(lw: LinearWorkload, counts: np.ndarray) -> np.ndarray:
+    """Mask [M, ceil(N/32)] choosing ``counts[i]`` of the N outputs of row i
+    uniformly without replacement (the random control at a matched row count)."""
+    return random_control_mask(lw.as_rows(), np.asarray(counts)[None, :])[0]
+
+
+LINEAR_WORKLOADS = {
+    "gelu_small_96x300x200": LinearWorkload(96, 300, 200),
+    # GPT-2 XL's first MLP layer (1600 -> 6400) on 1024 tokens
+    "gelu_gpt2xl_fc_1024x6400x1600": LinearWorkload(1024, 6400, 1600),
 }

@@ -8,6 +8,13 @@ over the valid (query, key) entries, k = round(rate * entries); the entries
 strictly above it are selected, so the selected count is at most k (fewer when
 criterion values tie).
 
+The activation workloads (GELU after a PS(mu) linear map) calibrate on the
+condition number kappa_j of every output. Their low-precision outputs take few
+distinct values (mu = 4 keeps 5 significant bits), so kappa ties heavily; tau is
+put halfway between the (k+1)-th largest value and the next larger distinct one,
+which selects the same entries and keeps every kappa far from tau (a last-bit
+difference between two exp implementations then decides nothing).
+
 Entries are taken from the whole workload, except for the 16K-token workload,
 where the oracle evaluates a uniform random sample of query rows (seeded; the
 row count is recorded). Sampling rows uniformly keeps the entry distribution,
@@ -42,6 +49,8 @@ PLAN = [
     ("decode_1x32x1x16384x128", oracle.STRICT, [4], [0.016], None),
     ("decode_1x32x1x16384x128", oracle.RELAXED, [4], [0.01], None),
     ("outlier_4x25x4096x64", oracle.STRICT, [4, 6], [0.003, 0.076], None),
+    ("gelu_small_96x300x200", oracle.STRICT, [4], [0.016], None),
+    ("gelu_gpt2xl_fc_1024x6400x1600", oracle.STRICT, [4], [0.003, 0.016, 0.076], None),
 ]
 
 
@@ -64,7 +73,30 @@ class TopK:
         return float(s[k])
 
 
+def calibrate_linear(name, mu, rates, threads):
+    lw = S.LINEAR_WORKLOADS[name]
+    x, W = S.make_linear(lw)
+    entries = lw.outputs()
+    ks = [int(round(r * entries)) for r in rates]
+    top = TopK(max(ks) + 1)
+    chunk = max(1, int(2 ** 22 // lw.N))
+    for lo in range(0, lw.M, chunk):
+        rows = np.arange(lo, min(lw.M, lo + chunk), dtype=np.int64)
+        res = oracle.linear_gelu_rows(x, W, scale=lw.scale, mu=mu, tau=np.inf, rows=rows, threads=threads)
+        top.add(res.kappa.reshape(-1))
+    out = []
+    for rate, k in zip(rates, ks):
+        v = top.kth_largest(k)
+        above = top.vals[top.vals > v]
+        tau = 0.5 * (v + float(above.min())) if above.size else v
+        out.append({"workload": name, "variant": int(oracle.STRICT), "mu": mu, "rate": rate, "tau": tau,
+                    "k": k, "entries": entries, "selected_at_tau": int(np.sum(top.vals > tau)), "rows": "all"})
+    return out
+
+
 def calibrate(name, variant, mu, rates, sample_rows, threads):
+    if name in S.LINEAR_WORKLOADS:
+        return calibrate_linear(name, mu, rates, threads)
     w = S.WORKLOADS[name]
     Q, K, V = S.make_qkv(w)
     total_rows = w.B * w.H * w.n_q

@@ -53,3 +53,24 @@ def test_random_control_mask_counts_and_validity():
     for i in range(50):
         assert not bits[:, i, nv[i]:].any()
     assert np.array_equal(S.pack_mask(bits), m)
+
+
+def test_linear_workload_inputs():
+    lw = S.LinearWorkload(5, 40, 24, seed=2)
+    x, W = S.make_linear(lw)
+    x2, W2 = S.make_linear(lw)
+    assert x.shape == (5, 24) and W.shape == (40, 24) and x.dtype == np.uint16
+    assert np.array_equal(x, x2) and np.array_equal(W, W2)
+    assert not np.array_equal(x[0, :24], W[0, :24])          # x and W use separate streams
+    assert lw.scale == np.float32(1 / np.sqrt(24))
+    xf = S.bf16_bits_to_f32(S.make_linear(S.LinearWorkload(64, 64, 256, seed=1))[0])
+    assert abs(float(xf.mean())) < 0.02 and abs(float(xf.std()) - 1) < 0.02
+
+
+def test_linear_random_mask_counts():
+    lw = S.LinearWorkload(7, 70, 8, seed=4)
+    counts = np.array([0, 1, 5, 70, 3, 33, 2])
+    m = S.linear_random_mask(lw, counts)
+    bits = S.unpack_mask(m, lw.N)
+    assert m.shape == (7, 3) and np.array_equal(bits.sum(axis=1), counts)
+    assert int(m[:, -1].max()) >> 6 == 0                     # no bits past N
