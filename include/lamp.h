@@ -198,6 +198,62 @@ LAMP_API const char *lamp_version(void);
  * that its copy of the struct has the same layout. */
 LAMP_API size_t lamp_args_size(void);
 
+/*
+ * lamp_linear_gelu -- LAMP on an elementwise activation: out = GELU(y) with
+ * y = scale * x W^T computed in PS(mu), and the outputs whose component-wise
+ * condition number kappa_j = |y_j f'(y_j) / f(y_j)| exceeds tau recomputed in
+ * binary32 before the activation. LAMP summary (gist.science paper 2601.21623):
+ * "Theoretical basis" item 3 (for an activation the Jacobian is diagonal, so the
+ * sensitive components are found directly) and "Implementation strategy" steps
+ * 1-3. f is GELU in its tanh form (GPT-2's activation),
+ * f(y) = y/2 (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))), and
+ * kappa(y) = |1 + y u'(y) (1 - tanh u)| (1 at y = 0; +inf for a non-finite y).
+ *
+ *   M, N, K     x is [M, K], W is [N, K] (a linear layer's weight layout), out
+ *               [M, N]; all row-major. K must be a multiple of 8; M <= 4194240.
+ *   x, W        bf16 bit patterns, device pointers, 16-byte aligned.
+ *   out         bf16 [M, N] (2-byte aligned): f(y) rounded to nearest even.
+ *   mask_out    nullable: uint32 words [M][ceil(N/32)], bit j % 32 of word j / 32
+ *               set when output j of the row was recomputed; padding bits 0.
+ *   mu, tau     PS(mu) fraction bits (1..23); kappa threshold (tau < 0 recomputes
+ *               every output, +inf none; ignored for LAMP_GIVEN_MASK). NaN is
+ *               LAMP_ERR_ARG.
+ *   variant     LAMP_STRICT (the kappa test; an activation has no relaxed form,
+ *               LAMP_RELAXED is LAMP_ERR_ARG) or LAMP_GIVEN_MASK (mask_in).
+ *   scale       multiplies each finished sum once in binary32; 0 = 1.
+ *   mask_in     LAMP_GIVEN_MASK: words in the mask_out layout (bits past N ignored).
+ *   out_f32     nullable fp32 [M, N]: f(y) before the bf16 rounding.
+ *   ps_out      nullable fp32 [M, N]: the PS(mu) outputs y_hat.
+ *   mixed_out   nullable fp32 [M, N]: y after the recompute.
+ *   n_selected_out  nullable device word: set to the number of recomputed outputs.
+ * Every pointer is caller-owned device memory; the call is asynchronous on
+ * stream, allocates nothing, and launches one kernel (plus a memset of
+ * n_selected_out). Returns LAMP_OK, LAMP_ERR_ARG or LAMP_ERR_UNSUPPORTED
+ * (K % 8 != 0, misaligned pointers, M too large) before launching anything, or
+ * LAMP_ERR_CUDA when the launch fails.
+ */
+typedef struct {
+  int M, N, K;
+  const void *x, *W;
+  void *out;
+  uint32_t *mask_out;
+  int mu;
+  float tau;
+  int variant;
+  float scale;
+  const uint32_t *mask_in;
+  float *out_f32;
+  float *ps_out;
+  float *mixed_out;
+  unsigned long long *n_selected_out;
+  lamp_stream_t stream;
+} lamp_gelu_args;
+
+LAMP_API int lamp_linear_gelu(const lamp_gelu_args *args);
+
+/* sizeof(lamp_gelu_args) as compiled into the library. */
+LAMP_API size_t lamp_gelu_args_size(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,14 +18,14 @@ from ._native import (LAMP_ERR_ARG, LAMP_ERR_CHECK, LAMP_ERR_CUDA, LAMP_ERR_TIME
                       LAMP_ERR_UNSUPPORTED, LAMP_ERR_WORKSPACE, LAMP_GIVEN_MASK, LAMP_MAX_STRICT_NK,
                       LAMP_NOALLOC_SCRATCH_BYTES, LAMP_OK, LAMP_RELAXED, LAMP_STRICT, LampError, lamp_args,
                       lamp_args_size, lamp_attention, lamp_attention_ex, lamp_attention_noalloc, lamp_dims,
-                      lamp_last_error, lamp_ps_round,
-                      lamp_version, lamp_workspace_size, load, make_args)
+                      lamp_gelu_args, lamp_gelu_args_size, lamp_last_error, lamp_linear_gelu, lamp_ps_round,
+                      lamp_version, lamp_workspace_size, load, make_args, make_gelu_args)
 
 __all__ = [
     "LAMP_STRICT", "LAMP_RELAXED", "LAMP_GIVEN_MASK", "LampError", "lamp_attention", "lamp_attention_ex",
     "lamp_attention_noalloc",
     "lamp_workspace_size", "lamp_last_error", "lamp_ps_round", "lamp_version", "lamp_args_size",
-    "attention", "LampOutputs", "load",
+    "attention", "LampOutputs", "load", "lamp_linear_gelu", "lamp_gelu_args_size", "linear_gelu", "GeluOutputs",
 ]
 
 
@@ -78,4 +78,53 @@ def attention(Q, K, V, *, mu: int = 4, tau: float = 0.0, variant: int = LAMP_STR
                       tau=tau, variant=variant, causal=int(bool(causal)), stream=stream, scale=scale,
                       mask_in=mask_in, out_f32=res.out_f32, ps_scores_out=res.ps_scores,
                       mixed_scores_out=res.mixed_scores, lse_out=res.lse, n_selected_out=res.n_selected)
+    return res
+
+
+@dataclass
+class GeluOutputs:
+    out: "object"
+    mask: "object | None" = None
+    out_f32: "object | None" = None
+    ps: "object | None" = None
+    mixed: "object | None" = None
+    n_selected: "object | None" = None
+
+
+def linear_gelu(x, W, *, mu: int = 4, tau: float = 0.0, variant: int = LAMP_STRICT, scale: float = 0.0,
+                mask_in=None, want_mask: bool = True, want_out_f32: bool = False, want_scores: bool = False,
+                want_count: bool = False, stream=None) -> GeluOutputs:
+    """LAMP GELU(scale * x W^T) on torch tensors ("Theoretical basis", item 3:
+    an activation's diagonal Jacobian).
+
+    x: [M, K], W: [N, K] (a linear layer's weight), both torch.bfloat16,
+    contiguous, on one CUDA device, K a multiple of 8. Returns the bf16 output
+    [M, N] and the requested extras (mask words int32 [M, ceil(N/32)], the PS(mu)
+    and mixed pre-activations fp32 [M, N], selected count int64 [1]).
+    """
+    import torch
+
+    M, K = x.shape
+    N = W.shape[0]
+    dev = x.device
+    for t in (x, W):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != dev:
+            raise ValueError("x and W must be contiguous bfloat16 tensors on one device")
+    if W.shape[1] != K:
+        raise ValueError("x and W disagree on K")
+    res = GeluOutputs(out=torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+    if want_mask:
+        res.mask = torch.empty((M, (N + 31) // 32), dtype=torch.int32, device=dev)
+    if want_out_f32:
+        res.out_f32 = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if want_scores:
+        res.ps = torch.empty((M, N), dtype=torch.float32, device=dev)
+        res.mixed = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if want_count:
+        res.n_selected = torch.empty(1, dtype=torch.int64, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    lamp_linear_gelu(M=M, N=N, K=K, x=x, W=W, out=res.out, mask_out=res.mask, mu=mu, tau=tau, variant=variant,
+                     scale=scale, mask_in=mask_in, out_f32=res.out_f32, ps_out=res.ps, mixed_out=res.mixed,
+                     n_selected_out=res.n_selected, stream=stream)
     return res

@@ -73,6 +73,25 @@ class lamp_args(ctypes.Structure):
     ]
 
 
+class lamp_gelu_args(ctypes.Structure):
+    _fields_ = [
+        ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int),
+        ("x", _P), ("W", _P),
+        ("out", _P),
+        ("mask_out", _P),
+        ("mu", ctypes.c_int),
+        ("tau", ctypes.c_float),
+        ("variant", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("mask_in", _P),
+        ("out_f32", _P),
+        ("ps_out", _P),
+        ("mixed_out", _P),
+        ("n_selected_out", _P),
+        ("stream", _P),
+    ]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -87,6 +106,8 @@ SIGNATURES = {
     "lamp_ps_round": (ctypes.c_int, [_P, _P, ctypes.c_size_t, ctypes.c_int, ctypes.c_int, _P]),
     "lamp_version": (ctypes.c_char_p, []),
     "lamp_args_size": (ctypes.c_size_t, []),
+    "lamp_linear_gelu": (ctypes.c_int, [ctypes.POINTER(lamp_gelu_args)]),
+    "lamp_gelu_args_size": (ctypes.c_size_t, []),
 }
 
 
@@ -106,6 +127,8 @@ def load(path: str = LIB_PATH):
                 fn.argtypes = args
             if L.lamp_args_size() != ctypes.sizeof(lamp_args):
                 raise ImportError("lamp_args layout of the binding does not match liblamp.so")
+            if L.lamp_gelu_args_size() != ctypes.sizeof(lamp_gelu_args):
+                raise ImportError("lamp_gelu_args layout of the binding does not match liblamp.so")
             _lib = L
     return _lib
 
@@ -187,4 +210,24 @@ def lamp_attention_noalloc(args: lamp_args | None = None, check: bool = True, **
 
 def lamp_ps_round(x, y, n: int, mu: int, path: int = 0, stream=None, check: bool = True) -> int:
     rc = load().lamp_ps_round(_ptr(x), _ptr(y), int(n), int(mu), int(path), _stream(stream))
+    return _check(rc) if check else rc
+
+
+def lamp_gelu_args_size() -> int:
+    return int(load().lamp_gelu_args_size())
+
+
+def make_gelu_args(M, N, K, x, W, out, *, mask_out=None, mu=4, tau=0.0, variant=LAMP_STRICT, scale=0.0,
+                   mask_in=None, out_f32=None, ps_out=None, mixed_out=None, n_selected_out=None,
+                   stream=None) -> lamp_gelu_args:
+    return lamp_gelu_args(int(M), int(N), int(K), _ptr(x), _ptr(W), _ptr(out), _ptr(mask_out), int(mu),
+                          float(tau), int(variant), float(scale), _ptr(mask_in), _ptr(out_f32), _ptr(ps_out),
+                          _ptr(mixed_out), _ptr(n_selected_out), _stream(stream))
+
+
+def lamp_linear_gelu(args: lamp_gelu_args | None = None, check: bool = True, **kw) -> int:
+    """LAMP GELU(scale * x W^T): pass a lamp_gelu_args, or make_gelu_args' keyword arguments."""
+    if args is None:
+        args = make_gelu_args(**kw)
+    rc = load().lamp_linear_gelu(ctypes.byref(args))
     return _check(rc) if check else rc

@@ -353,6 +353,50 @@ int lamp_attention(const lamp_dims* dims, const void* Q, const void* K, const vo
   return lamp_attention_ex(&a);
 }
 
+size_t lamp_gelu_args_size(void) { return sizeof(lamp_gelu_args); }
+
+int lamp_linear_gelu(const lamp_gelu_args* a) {
+  if (!a) return fail(LAMP_ERR_ARG, "args is NULL");
+  if (a->M <= 0 || a->N <= 0 || a->K <= 0)
+    return fail(LAMP_ERR_ARG, "dimensions must be positive (M=%d N=%d K=%d)", a->M, a->N, a->K);
+  if (!a->x || !a->W || !a->out) return fail(LAMP_ERR_ARG, "x, W and out must be non-NULL");
+  if (a->mu < 1 || a->mu > 23) return fail(LAMP_ERR_ARG, "mu must be in [1, 23] (got %d)", a->mu);
+  if (a->variant == LAMP_RELAXED)
+    return fail(LAMP_ERR_ARG, "an activation's kappa test is exact per output; there is no relaxed variant");
+  if (a->variant != LAMP_STRICT && a->variant != LAMP_GIVEN_MASK)
+    return fail(LAMP_ERR_ARG, "unknown variant %d", a->variant);
+  if (a->variant == LAMP_STRICT && std::isnan(a->tau)) return fail(LAMP_ERR_ARG, "tau is NaN");
+  if (a->variant == LAMP_GIVEN_MASK && !a->mask_in) return fail(LAMP_ERR_ARG, "LAMP_GIVEN_MASK needs mask_in");
+  if (std::isnan(a->scale) || a->scale < 0.f || std::isinf(a->scale))
+    return fail(LAMP_ERR_ARG, "scale must be 0 (default 1) or a positive finite value");
+  if (a->K % 8) return fail(LAMP_ERR_UNSUPPORTED, "K must be a multiple of 8 (got %d)", a->K);
+  if (a->M > lamp::gelu_max_rows()) return fail(LAMP_ERR_UNSUPPORTED, "M must be at most %d", lamp::gelu_max_rows());
+  if (!aligned(a->x, 16) || !aligned(a->W, 16)) return fail(LAMP_ERR_UNSUPPORTED, "x and W must be 16-byte aligned");
+  if (!aligned(a->out, 2) || (a->mask_out && !aligned(a->mask_out, 4)) || (a->mask_in && !aligned(a->mask_in, 4)) ||
+      (a->out_f32 && !aligned(a->out_f32, 4)) || (a->ps_out && !aligned(a->ps_out, 4)) ||
+      (a->mixed_out && !aligned(a->mixed_out, 4)) || (a->n_selected_out && !aligned(a->n_selected_out, 8)))
+    return fail(LAMP_ERR_UNSUPPORTED, "outputs must be naturally aligned");
+  lamp::GeluProblem g;
+  g.M = a->M; g.N = a->N; g.K = a->K;
+  g.mu = a->mu;
+  g.tau = a->variant == LAMP_GIVEN_MASK ? 0.f : a->tau;
+  g.scale = a->scale == 0.f ? 1.f : a->scale;
+  g.variant = a->variant;
+  g.x = static_cast<const uint16_t*>(a->x);
+  g.W = static_cast<const uint16_t*>(a->W);
+  g.out = static_cast<uint16_t*>(a->out);
+  g.mask_out = a->mask_out;
+  g.mask_in = a->mask_in;
+  g.out_f32 = a->out_f32;
+  g.ps_out = a->ps_out;
+  g.mixed_out = a->mixed_out;
+  g.nsel_out = a->n_selected_out;
+  g.emax_sum_limit = emax_sum_limit(a->mu, a->K);
+  cudaError_t e = lamp::launch_gelu(g, reinterpret_cast<cudaStream_t>(a->stream));
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 int lamp_ps_round(const float* x, float* y, size_t n, int mu, int path, lamp_stream_t stream) {
   if ((!x || !y) && n) return fail(LAMP_ERR_ARG, "x and y must be non-NULL");
   if (mu < 1 || mu > 23) return fail(LAMP_ERR_ARG, "mu must be in [1, 23] (got %d)", mu);

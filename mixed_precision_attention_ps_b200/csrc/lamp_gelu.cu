@@ -1,0 +1,343 @@
+// LAMP on an elementwise activation: out = GELU(y), y = scale * x W^T with the
+// linear map accumulated in PS(mu), and the outputs whose component-wise
+// condition number exceeds tau recomputed in binary32 before the activation.
+// LAMP summary (gist.science paper 2601.21623): "Theoretical basis" item 3 (an
+// activation has a diagonal Jacobian, so each output's sensitivity is its own
+// condition number kappa_j = |y_j f'(y_j) / f(y_j)|) and "Implementation
+// strategy" steps 1-3 (low-precision g, look-ahead selection, recompute).
+//
+// One CTA of 256 threads computes a 64 x 128 tile of outputs over the whole K:
+// warp w owns rows 8w .. 8w+7 of the tile, lane l the columns l + 32m (m < 4),
+// so that a ballot over a (row, m) is one mask word. Slices of 32 dimensions of
+// x and W are staged global -> registers -> shared memory as binary32 (W as
+// (w, w) pairs), one slice ahead; a step is packed over two rows: fma.rn.f32x2
+// of the exact bf16 products, then the PS(mu) rounding of the pair.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "lamp.h"
+#include "lamp_device.cuh"
+#include "lamp_kernels.h"
+
+namespace lamp {
+namespace {
+
+constexpr int GL_BM = 64, GL_BN = 128, GL_KS = 32, GL_T = 256;
+constexpr float kGeluC = 0.7978845608028654f;   // sqrt(2 / pi)
+constexpr float kGeluA = 0.044715f;
+constexpr double kGeluCd = 0.7978845608028654;  // sqrt(2 / pi) in double
+constexpr double kGeluAd = 0.044715;
+// |kappa_f32 - kappa| <= 2e-5 (1 + |v|) for the binary32 evaluation below (v the
+// term added to 1): inside twice that band the test is taken again in double.
+constexpr float kKappaBand = 4e-5f;
+
+struct GeluSmem {
+  float xs[2][GL_KS][GL_BM];  // x slice: [dim][row], so a row pair is one 8-byte word
+  u64 ws[2][GL_KS][GL_BN];    // W slice: [dim][col] as (w, w)
+};
+
+struct GeluArgs {
+  GeluProblem p;
+  u64 negc, pow2s;  // the two-instruction rounding's constants, as pairs
+  int s;            // 23 - mu
+};
+
+__device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// bf16 bits -> binary32 bits, for the low and high halves of a word
+__device__ __forceinline__ uint32_t lo_bits(uint32_t w) { return w << 16; }
+__device__ __forceinline__ uint32_t hi_bits(uint32_t w) { return w & 0xFFFF0000u; }
+
+// Largest magnitude and (smallest nonzero magnitude - 1) of the staged values, as
+// binary32 bit patterns compared as integers (a zero wraps to 0xFFFFFFFF).
+__device__ __forceinline__ void fold(uint32_t& mx, uint32_t& mn, uint32_t bits) {
+  const uint32_t a = bits & 0x7FFFFFFFu;
+  mx = max(mx, a);
+  mn = min(mn, a - 1u);
+}
+
+// kappa(y) = |1 + y u'(y) (1 - tanh u)|, u = c (y + a y^3), in double, with the
+// operations in the order of the definition (no contraction).
+__device__ __noinline__ double kappa_d(float yf) {
+  const double y = (double)yf;
+  const double y2 = __dmul_rn(y, y);
+  const double u = __dmul_rn(kGeluCd, __dadd_rn(y, __dmul_rn(__dmul_rn(kGeluAd, y), y2)));
+  const double du = __dmul_rn(kGeluCd, __dadd_rn(1.0, __dmul_rn(__dmul_rn(3.0 * kGeluAd, y), y)));
+  const double omt = 2.0 / __dadd_rn(1.0, exp(__dmul_rn(2.0, u)));
+  return fabs(__dadd_rn(1.0, __dmul_rn(__dmul_rn(y, du), omt)));
+}
+
+// The same in binary32: returns kappa and the term v (kappa = |1 + v|).
+__device__ __forceinline__ float kappa_f(float y, float& v) {
+  const float y2 = y * y;
+  const float u = kGeluC * fmaf(kGeluA * y2, y, y);
+  const float du = kGeluC * fmaf(3.f * kGeluA, y2, 1.f);
+  const float omt = 2.f / (1.f + expf(2.f * u));
+  v = y * du * omt;
+  return fabsf(1.f + v);
+}
+
+__device__ __forceinline__ float gelu_f(float y) {
+  const float u = kGeluC * fmaf(kGeluA * y * y, y, y);
+  return 0.5f * y * (1.f + tanhf(u));
+}
+
+// The K loop: acc[p][m] accumulates rows (8w + 2p, 8w + 2p + 1) of the tile
+// against column lane + 32m, in PS(mu) steps of the given mode, sequentially
+// over k. FOLD collects the operands' magnitude range for the rounding test.
+template <int MODE, bool FOLD>
+__device__ __forceinline__ void gelu_mainloop(const GeluArgs& A, GeluSmem& sm, int m0, int n0, u64 (&acc)[4][4],
+                                              uint32_t (&rng)[4]) {
+  const GeluProblem& p = A.p;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int xr = t & 63, xc = t >> 6;          // x: row xr, dims 8 xc .. 8 xc + 7 of a slice
+  const int wc = t & 127, wq = (t >> 7) * 2;   // W: col wc, dims 8 wq .. 8 wq + 15
+  const bool xin = m0 + xr < p.M, win = n0 + wc < p.N;
+  const uint16_t* xp = p.x + (size_t)(xin ? m0 + xr : 0) * p.K + 8 * xc;
+  const uint16_t* wp = p.W + (size_t)(win ? n0 + wc : 0) * p.K + 8 * wq;
+  const int nsl = (p.K + GL_KS - 1) / GL_KS;
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+  uint4 rx, rw0, rw1;
+  auto load = [&](int sl) {
+    const int k = sl * GL_KS;
+    rx = (xin && k + 8 * xc < p.K) ? ldg16(xp + k) : z4;
+    rw0 = (win && k + 8 * wq < p.K) ? ldg16(wp + k) : z4;
+    rw1 = (win && k + 8 * wq + 8 < p.K) ? ldg16(wp + k + 8) : z4;
+  };
+  auto store = [&](int buf) {
+    const uint32_t xw[4] = {rx.x, rx.y, rx.z, rx.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t a = lo_bits(xw[j]), b = hi_bits(xw[j]);
+      sm.xs[buf][8 * xc + 2 * j][xr] = __uint_as_float(a);
+      sm.xs[buf][8 * xc + 2 * j + 1][xr] = __uint_as_float(b);
+      if (FOLD) { fold(rng[0], rng[1], a); fold(rng[0], rng[1], b); }
+    }
+    const uint32_t ww[8] = {rw0.x, rw0.y, rw0.z, rw0.w, rw1.x, rw1.y, rw1.z, rw1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t a = lo_bits(ww[j]), b = hi_bits(ww[j]);
+      sm.ws[buf][8 * wq + 2 * j][wc] = ((u64)a << 32) | a;
+      sm.ws[buf][8 * wq + 2 * j + 1][wc] = ((u64)b << 32) | b;
+      if (FOLD) { fold(rng[2], rng[3], a); fold(rng[2], rng[3], b); }
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc[i][m] = 0ull;
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int sl = 0; sl < nsl; ++sl) {
+    const int buf = sl & 1;
+    if (sl + 1 < nsl) load(sl + 1);
+#pragma unroll 8
+    for (int k = 0; k < GL_KS; ++k) {
+      const ulonglong2 xa = *reinterpret_cast<const ulonglong2*>(&sm.xs[buf][k][8 * warp]);
+      const ulonglong2 xb = *reinterpret_cast<const ulonglong2*>(&sm.xs[buf][k][8 * warp + 4]);
+      const u64 xq[4] = {xa.x, xa.y, xb.x, xb.y};
+      u64 wd[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) wd[m] = sm.ws[buf][k][lane + 32 * m];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc[i][m] = ps_step<MODE>(xq[i], wd[m], acc[i][m], A.negc, A.pow2s, A.s);
+    }
+    // buf ^ 1 was last read before the barrier that ended the previous slice
+    if (sl + 1 < nsl) store(buf ^ 1);
+    __syncthreads();
+  }
+}
+
+// The two-instruction rounding is exact when every partial sum is 0 or a normal
+// number below 2^(127 - s): partial sums are multiples of the smallest product
+// grid 2^(e_x,min - 7) 2^(e_w,min - 7), and bounded by the growth limit the host
+// computes from mu and K.
+__device__ __forceinline__ bool gelu_fast_ok(const uint32_t (&r)[4], int emax_sum_limit) {
+  const int ex = (int)(r[0] >> 23), ew = (int)(r[2] >> 23);
+  if (ex >= 255 || ew >= 255) return false;  // an infinity or NaN: the exact rounding
+  if (r[1] == 0xFFFFFFFFu || r[3] == 0xFFFFFFFFu) return true;  // one operand all zero: every product is 0
+  const int lx = max((int)((r[1] + 1u) >> 23), 1) - 134, lw = max((int)((r[3] + 1u) >> 23), 1) - 134;
+  return (ex - 127) + (ew - 127) <= emax_sum_limit && lx + lw >= -126;
+}
+
+template <int RND>
+__global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  GeluSmem& sm = *reinterpret_cast<GeluSmem*>(smem_raw);
+  __shared__ uint32_t red[GL_T / 32][4];
+  __shared__ int fast_sh;
+  const GeluProblem& p = A.p;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int n0 = blockIdx.x * GL_BN, m0 = blockIdx.y * GL_BM;
+  u64 acc[4][4];
+  uint32_t rng[4] = {0u, 0xFFFFFFFFu, 0u, 0xFFFFFFFFu};
+
+  // step 1: the low-precision linear map. The fused forms (the two-instruction
+  // rounding for mu <= 10, a fused multiply-add for mu = 23) are taken first and
+  // checked against the operands' magnitude range; a tile outside it (products
+  // that are not exact in binary32, partial sums outside the rounding's domain)
+  // is computed again with one binary32 multiply, add and exact rounding a step.
+  if (RND == kRndExact) {
+    gelu_mainloop<kStepExact, false>(A, sm, m0, n0, acc, rng);
+  } else {
+    if (RND == kRndNone) gelu_mainloop<kStepF32, true>(A, sm, m0, n0, acc, rng);
+    else gelu_mainloop<kStepFast, true>(A, sm, m0, n0, acc, rng);
+    rng[0] = __reduce_max_sync(0xFFFFFFFFu, rng[0]);
+    rng[1] = __reduce_min_sync(0xFFFFFFFFu, rng[1]);
+    rng[2] = __reduce_max_sync(0xFFFFFFFFu, rng[2]);
+    rng[3] = __reduce_min_sync(0xFFFFFFFFu, rng[3]);
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[warp][i] = rng[i];
+    }
+    __syncthreads();
+    if (t == 0) {
+      uint32_t r[4] = {0u, 0xFFFFFFFFu, 0u, 0xFFFFFFFFu};
+      for (int w = 0; w < GL_T / 32; ++w) {
+        r[0] = max(r[0], red[w][0]); r[1] = min(r[1], red[w][1]);
+        r[2] = max(r[2], red[w][2]); r[3] = min(r[3], red[w][3]);
+      }
+      fast_sh = gelu_fast_ok(r, p.emax_sum_limit) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!fast_sh)  // outside the two-instruction rounding's domain: again, exactly
+      gelu_mainloop<kStepExact, false>(A, sm, m0, n0, acc, rng);
+  }
+
+  // step 2: the condition number of each output, and the selection
+  const u64 sc2 = pack2(p.scale, p.scale);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc[i][m] = mul2u(acc[i][m], sc2);
+  const int row0 = m0 + 8 * warp;
+  const int nw = (p.N + 31) >> 5;
+  uint32_t myword = 0u;  // lane 4r + m keeps the ballot of (row r, column group m)
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int row = row0 + r;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int col = n0 + lane + 32 * m;
+      const float y = (r & 1) ? hi_f(acc[r >> 1][m]) : lo_f(acc[r >> 1][m]);
+      const bool valid = row < p.M && col < p.N;
+      bool sel;
+      if (p.variant == LAMP_GIVEN_MASK) {
+        sel = valid && ((__ldg(p.mask_in + (size_t)row * nw + (col >> 5)) >> lane) & 1u);
+      } else if (!isfinite(y)) {
+        sel = valid && p.tau < INFINITY;  // kappa = +inf
+      } else {
+        float v;
+        const float kf = kappa_f(y, v);
+        sel = kf > p.tau;
+        if (fabsf(kf - p.tau) <= kKappaBand * (1.f + fabsf(v))) sel = kappa_d(y) > (double)p.tau;
+        sel = sel && valid;
+      }
+      const uint32_t b = __ballot_sync(0xFFFFFFFFu, sel);
+      if (lane == 4 * r + m) myword = b;
+      if (valid) {
+        const size_t o = (size_t)row * p.N + col;
+        if (p.ps_out) p.ps_out[o] = y;
+        if (!sel) {  // step 3 for the others: the activation of the low-precision output
+          if (p.mixed_out) p.mixed_out[o] = y;
+          const float f = gelu_f(y);
+          if (p.out_f32) p.out_f32[o] = f;
+          p.out[o] = f32_to_bf16_rne(f);
+        }
+      }
+    }
+  }
+  {
+    const int r = lane >> 2, m = lane & 3;
+    if (p.mask_out && row0 + r < p.M && (n0 >> 5) + m < nw) p.mask_out[(size_t)(row0 + r) * nw + (n0 >> 5) + m] = myword;
+  }
+
+  // step 3: recompute the selected outputs in binary32, 32 per round over the warp
+  const int cnt = __popc(myword);
+  int incl = cnt;  // inclusive scan of the counts over the lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  if (p.nsel_out && lane == 0 && total) atomicAdd(p.nsel_out, (unsigned long long)total);
+  for (int base = 0; base < total; base += 32) {
+    const int slot = base + lane;
+    // the word holding this slot: the first lane whose inclusive count passes it
+    int lo = 0, hi = 31;
+#pragma unroll
+    for (int it = 0; it < 5; ++it) {
+      const int mid = (lo + hi) >> 1;
+      const int v = __shfl_sync(0xFFFFFFFFu, incl, mid);
+      if (v > slot) hi = mid; else lo = mid + 1;
+    }
+    const int owner = lo;
+    const uint32_t word = __shfl_sync(0xFFFFFFFFu, myword, owner);
+    const int before = __shfl_sync(0xFFFFFFFFu, incl - cnt, owner);
+    if (slot < total) {
+      const int c = __fns(word, 0, slot - before + 1);
+      const int r = owner >> 2, m = owner & 3;
+      const int row = row0 + r, col = n0 + c + 32 * m;
+      const uint4* xq = reinterpret_cast<const uint4*>(p.x + (size_t)row * p.K);
+      const uint4* wq = reinterpret_cast<const uint4*>(p.W + (size_t)col * p.K);
+      float s = 0.f;  // the sequential binary32 dot: one multiply and one add a step
+#pragma unroll 4
+      for (int k = 0; k < (p.K >> 3); ++k) {
+        const uint4 a = __ldg(xq + k), b = __ldg(wq + k);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          s = __fadd_rn(s, __fmul_rn(__uint_as_float(lo_bits(aw[j])), __uint_as_float(lo_bits(bw[j]))));
+          s = __fadd_rn(s, __fmul_rn(__uint_as_float(hi_bits(aw[j])), __uint_as_float(hi_bits(bw[j]))));
+        }
+      }
+      const float y = __fmul_rn(p.scale, s);
+      const size_t o = (size_t)row * p.N + col;
+      if (p.mixed_out) p.mixed_out[o] = y;
+      const float f = gelu_f(y);
+      if (p.out_f32) p.out_f32[o] = f;
+      p.out[o] = f32_to_bf16_rne(f);
+    }
+  }
+}
+
+template <int RND>
+cudaError_t gelu_launch_one(const GeluArgs& A, cudaStream_t st) {
+  const size_t smem = sizeof(GeluSmem);
+  cudaError_t e = cudaFuncSetAttribute(gelu_kernel<RND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((A.p.N + GL_BN - 1) / GL_BN, (A.p.M + GL_BM - 1) / GL_BM);
+  gelu_kernel<RND><<<grid, GL_T, smem, st>>>(A);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int gelu_max_rows() { return 65535 * GL_BM; }
+
+cudaError_t launch_gelu(const GeluProblem& p, cudaStream_t st) {
+  if (p.nsel_out) {
+    cudaError_t e = cudaMemsetAsync(p.nsel_out, 0, sizeof(unsigned long long), st);
+    if (e != cudaSuccess) return e;
+  }
+  GeluArgs A;
+  A.p = p;
+  A.s = 23 - p.mu;
+  const float c = -(float)((1 << A.s) - 1), q = (float)(1 << A.s);
+  uint32_t cb, qb;
+  std::memcpy(&cb, &c, 4);
+  std::memcpy(&qb, &q, 4);
+  A.negc = ((u64)cb << 32) | cb;
+  A.pow2s = ((u64)qb << 32) | qb;
+  if (p.mu == 23) return gelu_launch_one<kRndNone>(A, st);
+  if (p.mu <= 10) return gelu_launch_one<kRndFast>(A, st);
+  return gelu_launch_one<kRndExact>(A, st);
+}
+
+}  // namespace lamp

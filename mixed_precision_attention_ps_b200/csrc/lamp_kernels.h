@@ -91,4 +91,25 @@ cudaError_t launch_ps_round(const float* x, float* y, size_t n, int mu, int path
 
 size_t strict_smem_bytes(int d, int nkp, bool rows_on_chip);
 
+// LAMP GELU(scale * x W^T): x [M, K], W [N, K] bf16, out [M, N].
+struct GeluProblem {
+  int M, N, K;
+  int mu;
+  float tau;
+  float scale;
+  int variant;  // LAMP_STRICT (the kappa test) or LAMP_GIVEN_MASK
+  const uint16_t* x;
+  const uint16_t* W;
+  uint16_t* out;
+  uint32_t* mask_out;
+  const uint32_t* mask_in;
+  float* out_f32;
+  float* ps_out;
+  float* mixed_out;
+  unsigned long long* nsel_out;
+  int emax_sum_limit;  // largest e_x + e_w for which the two-instruction rounding is exact
+};
+cudaError_t launch_gelu(const GeluProblem& p, cudaStream_t st);
+int gelu_max_rows();
+
 }  // namespace lamp

@@ -38,6 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_struct_layout_matches(lib):
     assert lamp.lamp_args_size() == ctypes.sizeof(_native.lamp_args) == 168
+    assert lamp.lamp_gelu_args_size() == ctypes.sizeof(_native.lamp_gelu_args) == 112
     assert lamp.lamp_version().startswith("lamp-b200")
 
 
@@ -106,3 +107,35 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_native, "_lib", None)
     with pytest.raises(ImportError, match="no fallback"):
         _native.load(str(tmp_path / "liblamp.so"))
+
+
+def call_gelu(**kw):
+    base = dict(M=4, N=40, K=16, x=FAKE, W=FAKE, out=FAKE, mu=4, tau=1.0)
+    base.update(kw)
+    return lamp.lamp_linear_gelu(check=False, **base)
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(x=None), lamp.LAMP_ERR_ARG, "non-NULL"),
+    (dict(out=None), lamp.LAMP_ERR_ARG, "non-NULL"),
+    (dict(M=0), lamp.LAMP_ERR_ARG, "positive"),
+    (dict(K=-8), lamp.LAMP_ERR_ARG, "positive"),
+    (dict(mu=24), lamp.LAMP_ERR_ARG, "mu"),
+    (dict(variant=lamp.LAMP_RELAXED), lamp.LAMP_ERR_ARG, "relaxed"),
+    (dict(variant=5), lamp.LAMP_ERR_ARG, "variant"),
+    (dict(tau=float("nan")), lamp.LAMP_ERR_ARG, "tau"),
+    (dict(variant=lamp.LAMP_GIVEN_MASK), lamp.LAMP_ERR_ARG, "mask_in"),
+    (dict(scale=float("inf")), lamp.LAMP_ERR_ARG, "scale"),
+    (dict(K=12), lamp.LAMP_ERR_UNSUPPORTED, "multiple of 8"),
+    (dict(M=65535 * 64 + 1), lamp.LAMP_ERR_UNSUPPORTED, "at most"),
+    (dict(W=FAKE + 8), lamp.LAMP_ERR_UNSUPPORTED, "16-byte"),
+    (dict(out=FAKE + 1), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
+    (dict(n_selected_out=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
+])
+def test_gelu_argument_checks(lib, kw, code, msg):
+    assert call_gelu(**kw) == code
+    assert msg in lamp.lamp_last_error()
+
+
+def test_gelu_null_args(lib):
+    assert _native.load().lamp_linear_gelu(None) == lamp.LAMP_ERR_ARG
