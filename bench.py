@@ -17,6 +17,9 @@ between steps outside the events; the max over ranks is reported.
 
 --impl reference times the CPU oracle (the plain C definition of the method)
 on this host's cores on a bounded sample of the same workload.
+
+The gelu_* workloads time LAMP on an elementwise activation instead (GELU after
+a PS(mu) linear map), with the same contract.
 """
 from __future__ import annotations
 
@@ -54,7 +57,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gpt2xl_1x25x1024x64", choices=sorted(S.WORKLOADS))
+    ap.add_argument("--workload", default="gpt2xl_1x25x1024x64", choices=sorted(S.WORKLOADS) + sorted(S.LINEAR_WORKLOADS))
     ap.add_argument("--variant", type=int, default=None, help="0 strict, 1 relaxed (default: per workload)")
     ap.add_argument("--mu", type=int, default=4)
     ap.add_argument("--rate", type=float, default=None, help="target recompute rate (tau from tau.json)")
@@ -72,6 +75,8 @@ DEFAULTS = {  # workload -> (variant, rate)
     "decode_1x32x1x16384x128": (0, 0.016),
     "outlier_4x25x4096x64": (0, 0.003),
     "single_head_128": (0, None),
+    "gelu_gpt2xl_fc_1024x6400x1600": (0, 0.016),
+    "gelu_small_96x300x200": (0, 0.016),
 }
 
 
@@ -516,8 +521,253 @@ def cpu_baseline(w, Q, K, V, mu, tau, variant) -> dict:
     return {"value": n_scores / t_all / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
 
 
+# ----------------------------------------------------------------------------------------
+# LAMP on an elementwise activation: GELU(scale * x W^T), the linear map in PS(mu)
+# ----------------------------------------------------------------------------------------
+def gelu_metric(lw, mu) -> str:
+    return f"LAMP GELU(x W^T) G-outputs/s at {lw.M}x{lw.N}x{lw.K} mu={mu}; % of roofline"
+
+
+GELU_UNIT = "G-outputs/s"
+
+
+def gelu_oracle_pass(lw, x, W, mu, tau, rows, threads) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.linear_gelu_rows(x, W, scale=lw.scale, mu=mu, tau=tau, rows=rows, threads=threads)
+    return time.perf_counter() - t0
+
+
+def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0) -> dict:
+    """The activation oracle as it stands, on the host's cores, over a row sample
+    repeated until about `seconds` of work have run."""
+    threads = os.cpu_count() or 1
+    m = max(1, lw.M // max(1, int(1.5e8 // (lw.N * lw.K))))
+    rows = np.arange(0, lw.M, m, dtype=np.int64)
+    t_all, n_out, passes = 0.0, 0, 0
+    while t_all < seconds and passes < 20:
+        t_all += gelu_oracle_pass(lw, x, W, mu, tau, rows, threads)
+        n_out += rows.size * lw.N
+        passes += 1
+    return {"value": n_out / t_all / 1e9, "unit": GELU_UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{passes} pass(es) over {rows.size} of {lw.M} rows (every {m}th, {rows.size * lw.N} "
+                      f"outputs each), {t_all:.1f} s"}
+
+
+def gelu_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream) -> dict:
+    """Errors against the all-FP32 outputs (tau < 0) for no recompute, LAMP at tau and
+    a random choice of the same per-row count, on a row sample (outside the timed region)."""
+    import oracle
+
+    def run(**kw):
+        r = lamp.linear_gelu(xd, Wd, mu=mu, scale=lw.scale, want_scores=True, want_out_f32=True,
+                             want_count=True, stream=stream, **kw)
+        torch.cuda.synchronize()
+        return r
+
+    rows = torch.arange(0, lw.M, 8, device=xd.device)
+    pick = lambda t: t.index_select(0, rows).cpu().numpy()  # noqa: E731
+    ref = run(tau=-1.0)
+    base = run(tau=float("inf"))
+    lr = run(tau=tau)
+    words = lr.mask.cpu().numpy().view(np.uint32)
+    per_row = np.unpackbits(words.view(np.uint8), axis=-1).sum(-1)
+    rmask = S.linear_random_mask(lw, per_row)
+    rr = run(tau=0.0, variant=2, mask_in=torch.from_numpy(rmask.view(np.int32)).to(xd.device))
+    r_out, r_y = pick(ref.out_f32), pick(ref.mixed)
+    err = {k: oracle.act_errors(pick(v.out_f32), pick(v.mixed), r_out, r_y)
+           for k, v in (("ps_only", base), ("lamp", lr), ("random_same_count", rr))}
+    return {"recompute_rate": lr.n_selected.item() / lw.outputs(), "rows_sampled": int(rows.numel()),
+            "errors_vs_fp32": err,
+            "max_amp_reduction_lamp": err["ps_only"]["max_amp"] / max(err["lamp"]["max_amp"], 1e-300),
+            "max_amp_reduction_random": err["ps_only"]["max_amp"] / max(err["random_same_count"]["max_amp"], 1e-300)}
+
+
+def run_gelu_reference(a, lw, mu, tau, cfg):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    x, W = S.make_linear(lw)
+    m = max(1, lw.M // max(1, int(1.6e8 // (lw.N * lw.K))))
+    rows = np.arange(0, lw.M, m, dtype=np.int64)
+    for _ in range(a.warmup):
+        gelu_oracle_pass(lw, x, W, mu, tau, rows, threads)
+    times = [gelu_oracle_pass(lw, x, W, mu, tau, rows, threads) for _ in range(a.steps)]
+    ms = 1e3 * statistics.mean(times)
+    value = rows.size * lw.N / (ms * 1e-3) / 1e9
+    sample = f"{rows.size} of {lw.M} rows (every {m}th), {rows.size * lw.N} outputs per step"
+    line = {"metric": gelu_metric(lw, mu), "value": value, "unit": GELU_UNIT, "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": GELU_UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": GELU_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gelu_ours(a, lw, mu, tau, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import mixed_precision_attention_ps_b200 as lamp
+
+    rank, local, world = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lamp.load()
+    lwr = S.LinearWorkload(lw.M, lw.N, lw.K, seed=lw.seed + rank)  # weak scaling: own inputs per rank
+    x, W = S.make_linear(lwr)
+
+    def dev_t(v):
+        return torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    xd, Wd = dev_t(x), dev_t(W)
+    out = torch.empty((lw.M, lw.N), dtype=torch.bfloat16, device=dev)
+    mask = torch.empty((lw.M, (lw.N + 31) // 32), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    args = lamp.make_gelu_args(lw.M, lw.N, lw.K, xd, Wd, out, mask_out=mask, mu=mu, tau=tau, scale=lw.scale,
+                               stream=stream)
+    call = lambda: lamp.lamp_linear_gelu(args)  # noqa: E731
+
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(getattr(props, "uuid", None) and ("GPU-" + str(props.uuid)))
+    clocks.start()
+    for _ in range(a.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    for s, e in evs:
+        flush.zero_()
+        s.record(stream)
+        call()
+        e.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    times = [s.elapsed_time(e) for s, e in evs]
+    ms = max_over_ranks([statistics.mean(times)], dev)[0]
+
+    # end to end through the C ABI with host buffers, pipelined as for attention: two
+    # device buffer sets, H2D / compute / D2H streams ordered by events
+    hx, hW = (torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).pin_memory() for v in (x, W))
+    hout = [torch.empty(out.shape, dtype=torch.int16).pin_memory() for _ in range(2)]
+    hmask = [torch.empty(mask.shape, dtype=torch.int32).pin_memory() for _ in range(2)]
+    e2e_steps = 0 if a.no_e2e else max(3, min(a.steps, 200))
+    ms_e2e = float("nan")
+    if e2e_steps:
+        sets = [(torch.empty_like(xd), torch.empty_like(Wd), torch.empty_like(out), torch.empty_like(mask))
+                for _ in range(2)]
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        bargs = [lamp.make_gelu_args(lw.M, lw.N, lw.K, st[0], st[1], st[2], mask_out=st[3], mu=mu, tau=tau,
+                                     scale=lw.scale, stream=s_cmp) for st in sets]
+
+        def pipeline(n):
+            done_in = [torch.cuda.Event() for _ in range(n)]
+            done_cmp = [torch.cuda.Event() for _ in range(n)]
+            done_out = [torch.cuda.Event() for _ in range(n)]
+            for i in range(n):
+                b = i & 1
+                bx, bW, bo, bm = sets[b]
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(done_cmp[i - 2])
+                    bx.view(torch.int16).copy_(hx, non_blocking=True)
+                    bW.view(torch.int16).copy_(hW, non_blocking=True)
+                    done_in[i].record(s_in)
+                s_cmp.wait_event(done_in[i])
+                if i >= 2:
+                    s_cmp.wait_event(done_out[i - 2])
+                lamp.lamp_linear_gelu(bargs[b])
+                done_cmp[i].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(done_cmp[i])
+                    hout[b].copy_(bo.view(torch.int16), non_blocking=True)
+                    hmask[b].copy_(bm, non_blocking=True)
+                    done_out[i].record(s_out)
+            return done_out[n - 1]
+
+        pipeline(4)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(s_in)
+        last = pipeline(e2e_steps)
+        s_out.wait_event(last)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        ms_e2e = t0.elapsed_time(t1) / e2e_steps
+        assert torch.equal(hout[(e2e_steps - 1) & 1], out.view(torch.int16).cpu())
+    ms_e2e = max_over_ranks([ms_e2e], dev)[0]
+    if world > 1:
+        dist.barrier()
+    result = None
+    if rank == 0:
+        n_out = lw.outputs()
+        value = job_value(world, n_out, ms)
+        peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
+        f_max = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+        peak = N_SM * FP32_LANES_PER_SM_CLK * f_max / 1e12
+        achieved = 4.0 * lw.K * n_out / (ms * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s", "frac": achieved / peak,
+                "traffic": traffic_bytes(a.workload, 0, mu),
+                "kernel": "gelu_kernel (one launch per call)",
+                "peak_basis": f"148 SMs x 128 lanes/clk x {f_max / 1e6:.0f} MHz (max SM clock); 4 K lane-ops "
+                              "per output (K steps of 1 multiply-add + 3 integer ops of the rounding)"}
+        result = {"metric": gelu_metric(lw, mu), "value": value, "unit": GELU_UNIT, "n_gpus": world, "steps": a.steps,
+                  "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                  "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg, "clocks": clk,
+                  "roofline": roof, "gpu_launches": a.steps,
+                  "e2e": {"value": job_value(world, n_out, ms_e2e), "unit": GELU_UNIT,
+                          "h2d_bytes_per_step": x.nbytes + W.nbytes,
+                          "d2h_bytes_per_step": out.numel() * 2 + mask.numel() * 4, "ms_per_step": ms_e2e,
+                          "form": "pipelined: 2 buffer sets, H2D / compute / D2H streams"},
+                  "ms_p10_p90": [float(np.percentile(times, 10)), float(np.percentile(times, 90))]}
+        if not a.no_kl:
+            result["accuracy"] = gelu_accuracy(lamp, torch, lwr, xd, Wd, mu, tau, stream)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not a.no_cpu_baseline and world == 1:
+            result["cpu_baseline"] = gelu_cpu_baseline(lwr, x, W, mu, tau)
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main_gelu(a):
+    lw = S.LINEAR_WORKLOADS[a.workload]
+    _, drate = DEFAULTS[a.workload]
+    rate = drate if a.rate is None else a.rate
+    tau, rate = lookup_tau(a.workload, 0, a.mu, rate)
+    cfg = {"workload": a.workload, "M": lw.M, "N": lw.N, "K": lw.K, "op": "GELU (tanh form) of scale * x W^T",
+           "scale": lw.scale, "variant": "kappa test", "mu": a.mu, "tau": tau, "target_recompute_rate": rate,
+           "inputs": "bf16 N(0,1) x and W (SplitMix64 + Box-Muller), seed = rank",
+           "l2": "flushed between steps (256 MB write)", "outputs_per_step_per_gpu": lw.outputs()}
+    if a.impl == "reference":
+        return run_gelu_reference(a, lw, a.mu, tau, cfg)
+    return run_gelu_ours(a, lw, a.mu, tau, cfg)
+
+
 def main():
     a = parse()
+    if a.workload in S.LINEAR_WORKLOADS:
+        return main_gelu(a)
     w = S.WORKLOADS[a.workload]
     dv, drate = DEFAULTS[a.workload]
     variant = dv if a.variant is None else a.variant
