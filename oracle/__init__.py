@@ -1,5 +1,6 @@
 """ctypes binding of the CPU oracle (``lamp_oracle.c``: attention;
-``lamp_oracle_act.c``: GELU after a PS(mu) linear map).
+``lamp_oracle_act.c``: GELU after a PS(mu) linear map; ``lamp_oracle_ln.c``:
+LayerNorm after a PS(mu) linear map).
 
 Test infrastructure only: the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline / reference legs use it; the CUDA library and its
@@ -18,7 +19,7 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, "lamp_oracle.c"), os.path.join(_HERE, "lamp_oracle_act.c")]
+_SRCS = [os.path.join(_HERE, f) for f in ("lamp_oracle.c", "lamp_oracle_act.c", "lamp_oracle_ln.c")]
 _LIB = os.path.join(_HERE, "liblamp_oracle.so")
 _CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c99"]
 
@@ -68,6 +69,16 @@ def lib():
             L.lamp_oracle_gelu.argtypes = [ctypes.c_double]
             L.lamp_oracle_gelu_kappa.restype = ctypes.c_double
             L.lamp_oracle_gelu_kappa.argtypes = [ctypes.c_double]
+            L.lamp_oracle_layernorm.restype = ctypes.c_double
+            L.lamp_oracle_layernorm.argtypes = [P, ctypes.c_int64, ctypes.c_double, P]
+            L.lamp_oracle_ln_select.restype = ctypes.c_int64
+            L.lamp_oracle_ln_select.argtypes = [P, ctypes.c_int64, ctypes.c_double, ctypes.c_double, P, P]
+            L.lamp_oracle_ln_thresholds.restype = None
+            L.lamp_oracle_ln_thresholds.argtypes = [P, ctypes.c_int64, ctypes.c_double, P]
+            L.lamp_oracle_linear_ln_rows.restype = ctypes.c_int
+            L.lamp_oracle_linear_ln_rows.argtypes = [P, P, P, ctypes.c_float, ctypes.c_int, ctypes.c_double,
+                                                     ctypes.c_double, ctypes.c_int, P, P, ctypes.c_int64, P, P, P,
+                                                     P, P, P, P]
             L.lamp_oracle_linear_gelu_rows.restype = ctypes.c_int
             L.lamp_oracle_linear_gelu_rows.argtypes = [P, P, P, ctypes.c_float, ctypes.c_int, ctypes.c_double,
                                                        ctypes.c_int, P, P, ctypes.c_int64, P, P, P, P, P, P]
@@ -310,3 +321,94 @@ def act_errors(out_x, y_x, out_ref, y_ref) -> dict:
     return {"l1_rel": float(diff.sum() / np.abs(r).sum()), "max_rel": float(rel.max()) if rel.size else 0.0,
             "max_amp": float(amp.max()) if amp.size else 0.0,
             "p99_amp": float(np.percentile(amp, 99)) if amp.size else 0.0}
+
+
+# --------------------------------------------------------------------------------------
+# LAMP on LayerNorm: LN(scale * x W^T) with a PS(mu) linear map
+# --------------------------------------------------------------------------------------
+LN_EPS = 1e-5  # GPT-2's layer-norm epsilon
+
+
+def layernorm(y, eps: float = LN_EPS):
+    """LayerNorm of one row (no affine part) in double. Returns (out, sigma)."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty_like(y)
+    sigma = lib().lamp_oracle_layernorm(_ptr(y), y.size, float(eps), _ptr(out))
+    return out, sigma
+
+
+def ln_select(ps_row, tau: float, eps: float = LN_EPS):
+    """Greedy selection of one row: (0/1 int32 mask, k, unselected sum of squares)."""
+    ps_row = np.ascontiguousarray(ps_row, dtype=np.float32)
+    sel = np.zeros(ps_row.size, dtype=np.int32)
+    rest = np.zeros(1, dtype=np.float64)
+    k = lib().lamp_oracle_ln_select(_ptr(ps_row), ps_row.size, float(eps), float(tau), _ptr(sel), _ptr(rest))
+    return sel, int(k), float(rest[0])
+
+
+def ln_thresholds(ps_row, eps: float = LN_EPS) -> np.ndarray:
+    """The tau values at which one row's greedy count changes (non-decreasing)."""
+    ps_row = np.ascontiguousarray(ps_row, dtype=np.float32)
+    t = np.empty(ps_row.size, dtype=np.float64)
+    lib().lamp_oracle_ln_thresholds(_ptr(ps_row), ps_row.size, float(eps), _ptr(t))
+    return t
+
+
+class LnResult:
+    """Per-row oracle outputs of LAMP LayerNorm(scale * x W^T)."""
+
+    def __init__(self, nrows, N):
+        self.ps = np.empty((nrows, N), np.float32)
+        self.mixed = np.empty((nrows, N), np.float32)
+        self.out = np.empty((nrows, N), np.float64)
+        self.mask = np.zeros((nrows, (N + 31) // 32), np.uint32)
+        self.nsel = np.zeros(nrows, np.int64)
+        self.sigma = np.zeros(nrows, np.float64)
+        self.rest = np.zeros(nrows, np.float64)
+
+
+def linear_ln_rows(x, W, *, scale=1.0, mu=4, tau=0.0, eps=LN_EPS, variant=STRICT, mask_in=None, rows=None,
+                   threads: int = 1) -> LnResult:
+    """Oracle LAMP LayerNorm(scale * x W^T) for selected rows of x (x [M, K],
+    W [N, K] bf16 bits). variant STRICT is the greedy selection; GIVEN_MASK
+    takes mask_in [M, ceil(N/32)]."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("x and W disagree on K")
+    if rows is None:
+        rows = np.arange(M, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    res = LnResult(rows.size, N)
+    dims = np.array([M, N, K], dtype=np.int64)
+    if mask_in is not None:
+        mask_in = np.ascontiguousarray(mask_in, dtype=np.uint32).reshape(M, -1)
+    L = lib()
+
+    def run(lo, hi):
+        sub = slice(lo, hi)
+        rc = L.lamp_oracle_linear_ln_rows(
+            _ptr(dims), _ptr(x), _ptr(W), float(scale), int(mu), float(tau), float(eps), int(variant),
+            _ptr(mask_in), _ptr(rows[sub]), hi - lo, _ptr(res.ps[sub]), _ptr(res.mixed[sub]), _ptr(res.out[sub]),
+            _ptr(res.mask[sub]), _ptr(res.nsel[sub]), _ptr(res.sigma[sub]), _ptr(res.rest[sub]))
+        if rc != 0:
+            raise ValueError(f"oracle rejected its arguments (rc={rc})")
+
+    n = rows.size
+    if threads <= 1 or n < 2 * threads:
+        run(0, n)
+    else:
+        chunk = max(1, n // (threads * 4))
+        bounds = [(lo, min(n, lo + chunk)) for lo in range(0, n, chunk)]
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda b: run(*b), bounds))
+    return res
+
+
+def ln_errors(out_x, out_ref) -> dict:
+    """Row errors of LayerNorm outputs against the all-FP32 ones: the mean and the
+    largest l2 error of a row (the quantity the norm-wise bound controls)."""
+    d = np.linalg.norm(np.asarray(out_x, np.float64) - np.asarray(out_ref, np.float64), axis=-1)
+    return {"mean_l2": float(d.mean()), "max_l2": float(d.max())}

@@ -253,4 +253,8 @@ LINEAR_WORKLOADS = {
     "gelu_small_96x300x200": LinearWorkload(96, 300, 200),
     # GPT-2 XL's first MLP layer (1600 -> 6400) on 1024 tokens
     "gelu_gpt2xl_fc_1024x6400x1600": LinearWorkload(1024, 6400, 1600),
+    # LayerNorm after a linear map
+    "ln_small_64x300x128": LinearWorkload(64, 300, 128),
+    # GPT-2 XL's attention output projection (1600 -> 1600) on 1024 tokens
+    "ln_gpt2xl_proj_1024x1600x1600": LinearWorkload(1024, 1600, 1600),
 }

@@ -15,6 +15,12 @@ put halfway between the (k+1)-th largest value and the next larger distinct one,
 which selects the same entries and keeps every kappa far from tau (a last-bit
 difference between two exp implementations then decides nothing).
 
+The LayerNorm workloads select per row greedily (the largest magnitudes until
+the rest meets the bound); a row's count changes at the oracle's threshold
+values sqrt(sum of the m smallest squares) / sigma, so tau is put halfway between
+the two consecutive distinct thresholds (over all rows) that give k recomputed
+outputs in total.
+
 Entries are taken from the whole workload, except for the 16K-token workload,
 where the oracle evaluates a uniform random sample of query rows (seeded; the
 row count is recorded). Sampling rows uniformly keeps the entry distribution,
@@ -51,6 +57,8 @@ PLAN = [
     ("outlier_4x25x4096x64", oracle.STRICT, [4, 6], [0.003, 0.076], None),
     ("gelu_small_96x300x200", oracle.STRICT, [4], [0.016], None),
     ("gelu_gpt2xl_fc_1024x6400x1600", oracle.STRICT, [4], [0.003, 0.016, 0.076], None),
+    ("ln_small_64x300x128", oracle.STRICT, [4], [0.016], None),
+    ("ln_gpt2xl_proj_1024x1600x1600", oracle.STRICT, [4], [0.003, 0.016, 0.076], None),
 ]
 
 
@@ -94,7 +102,27 @@ def calibrate_linear(name, mu, rates, threads):
     return out
 
 
+def calibrate_ln(name, mu, rates, threads):
+    lw = S.LINEAR_WORKLOADS[name]
+    x, W = S.make_linear(lw)
+    res = oracle.linear_ln_rows(x, W, scale=lw.scale, mu=mu, tau=np.inf, threads=threads)
+    t = np.sort(np.concatenate([oracle.ln_thresholds(res.ps[r]) for r in range(lw.M)]))
+    entries = lw.outputs()
+    out = []
+    for rate in rates:
+        k = int(round(rate * entries))
+        lo = t[entries - k - 1]          # the (entries - k)-th smallest threshold: met
+        above = t[t > lo]
+        tau = 0.5 * (lo + float(above.min())) if above.size else float(lo)
+        sel = int(entries - np.searchsorted(t, tau, side="right"))
+        out.append({"workload": name, "variant": int(oracle.STRICT), "mu": mu, "rate": rate, "tau": tau,
+                    "k": k, "entries": entries, "selected_at_tau": sel, "rows": "all"})
+    return out
+
+
 def calibrate(name, variant, mu, rates, sample_rows, threads):
+    if name.startswith("ln_"):
+        return calibrate_ln(name, mu, rates, threads)
     if name in S.LINEAR_WORKLOADS:
         return calibrate_linear(name, mu, rates, threads)
     w = S.WORKLOADS[name]
