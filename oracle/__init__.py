@@ -326,7 +326,7 @@ def act_errors(out_x, y_x, out_ref, y_ref) -> dict:
 # --------------------------------------------------------------------------------------
 # LAMP on LayerNorm: LN(scale * x W^T) with a PS(mu) linear map
 # --------------------------------------------------------------------------------------
-LN_EPS = 1e-5  # GPT-2's layer-norm epsilon
+LN_EPS = float(np.float32(1e-5))  # GPT-2's layer-norm epsilon, as the binary32 the C ABI takes
 
 
 def layernorm(y, eps: float = LN_EPS):

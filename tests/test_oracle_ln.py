@@ -71,7 +71,9 @@ def test_greedy_is_a_sparsest_feasible_set(seed):
     rng = np.random.default_rng(100 + seed)
     y = (rng.standard_normal(10) * 1.5).astype(np.float32)
     t = oracle.ln_thresholds(y)
-    for tau in (0.0, 0.5, 1.0, 2.0, 3.0, float(t[4]), float(t[8]) + 1e-9, 100.0):
+    # away from the threshold values themselves, where the two sides of the
+    # comparison differ only by rounding
+    for tau in (0.0, 0.5, 1.0, 2.0, 3.0, 0.5 * float(t[4] + t[5]), float(t[8]) * (1 + 1e-9), 100.0):
         sel, k, rest = oracle.ln_select(y, tau)
         assert k == brute_force_min_count(y, tau)
         # the set is the k largest magnitudes
