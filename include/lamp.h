@@ -254,6 +254,58 @@ LAMP_API int lamp_linear_gelu(const lamp_gelu_args *args);
 /* sizeof(lamp_gelu_args) as compiled into the library. */
 LAMP_API size_t lamp_gelu_args_size(void);
 
+/*
+ * lamp_linear_layernorm -- LAMP on LayerNorm: out = LN(y) over each row of
+ * y = scale * x W^T, with y computed in PS(mu) and, per row, the largest
+ * magnitudes recomputed in binary32 until ||(1 - q) o y_hat||_2 / sigma_hat <= tau
+ * (sigma_hat the low-precision row's sqrt(var + eps)). LAMP summary
+ * (gist.science paper 2601.21623): "Theoretical basis" item 3 (layer
+ * normalisation: a nearly sparsest set by sorting the input magnitudes) and
+ * "Implementation strategy" steps 1-3. LN has no affine part:
+ * LN(y)_j = (y_j - mean(y)) / sqrt(var(y) + eps), var the biased variance.
+ *
+ *   M, N, K, x, W, out, mask_out, mu, scale, mask_in, out_f32, ps_out,
+ *   mixed_out, n_selected_out: as for lamp_linear_gelu; N <= 8192.
+ *   tau         the bound on ||(1 - q) o y_hat||_2 / sigma_hat (tau < 0 recomputes
+ *               every output, +inf none). Equal magnitudes are taken in
+ *               ascending column order. NaN is LAMP_ERR_ARG.
+ *   variant     LAMP_STRICT (the greedy selection) or LAMP_GIVEN_MASK.
+ *   eps         LayerNorm's epsilon; 0 = 1e-5.
+ *   workspace   device scratch for y_hat of lamp_ln_workspace_size(M, N) bytes,
+ *               or NULL: then ps_out holds y_hat when given, else the library's
+ *               per-device pool (as lamp_attention_ex) provides it.
+ * Asynchronous on stream; two kernels (the linear map, then one warp per row).
+ * Returns LAMP_OK, LAMP_ERR_ARG / LAMP_ERR_UNSUPPORTED / LAMP_ERR_WORKSPACE
+ * before launching anything, or LAMP_ERR_CUDA.
+ */
+typedef struct {
+  int M, N, K;
+  const void *x, *W;
+  void *out;
+  uint32_t *mask_out;
+  int mu;
+  float tau;
+  int variant;
+  float scale;
+  float eps;
+  const uint32_t *mask_in;
+  float *out_f32;
+  float *ps_out;
+  float *mixed_out;
+  unsigned long long *n_selected_out;
+  void *workspace;
+  size_t workspace_bytes;
+  lamp_stream_t stream;
+} lamp_ln_args;
+
+LAMP_API int lamp_linear_layernorm(const lamp_ln_args *args);
+
+/* Bytes of scratch lamp_linear_layernorm needs when ps_out is NULL (M * N * 4). */
+LAMP_API size_t lamp_ln_workspace_size(int M, int N);
+
+/* sizeof(lamp_ln_args) as compiled into the library. */
+LAMP_API size_t lamp_ln_args_size(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,14 +18,16 @@ from ._native import (LAMP_ERR_ARG, LAMP_ERR_CHECK, LAMP_ERR_CUDA, LAMP_ERR_TIME
                       LAMP_ERR_UNSUPPORTED, LAMP_ERR_WORKSPACE, LAMP_GIVEN_MASK, LAMP_MAX_STRICT_NK,
                       LAMP_NOALLOC_SCRATCH_BYTES, LAMP_OK, LAMP_RELAXED, LAMP_STRICT, LampError, lamp_args,
                       lamp_args_size, lamp_attention, lamp_attention_ex, lamp_attention_noalloc, lamp_dims,
-                      lamp_gelu_args, lamp_gelu_args_size, lamp_last_error, lamp_linear_gelu, lamp_ps_round,
-                      lamp_version, lamp_workspace_size, load, make_args, make_gelu_args)
+                      lamp_gelu_args, lamp_gelu_args_size, lamp_last_error, lamp_linear_gelu,
+                      lamp_linear_layernorm, lamp_ln_args, lamp_ln_args_size, lamp_ln_workspace_size, lamp_ps_round,
+                      lamp_version, lamp_workspace_size, load, make_args, make_gelu_args, make_ln_args)
 
 __all__ = [
     "LAMP_STRICT", "LAMP_RELAXED", "LAMP_GIVEN_MASK", "LampError", "lamp_attention", "lamp_attention_ex",
     "lamp_attention_noalloc",
     "lamp_workspace_size", "lamp_last_error", "lamp_ps_round", "lamp_version", "lamp_args_size",
     "attention", "LampOutputs", "load", "lamp_linear_gelu", "lamp_gelu_args_size", "linear_gelu", "GeluOutputs",
+    "lamp_linear_layernorm", "lamp_ln_args_size", "lamp_ln_workspace_size", "linear_layernorm",
 ]
 
 
@@ -127,4 +129,39 @@ def linear_gelu(x, W, *, mu: int = 4, tau: float = 0.0, variant: int = LAMP_STRI
     lamp_linear_gelu(M=M, N=N, K=K, x=x, W=W, out=res.out, mask_out=res.mask, mu=mu, tau=tau, variant=variant,
                      scale=scale, mask_in=mask_in, out_f32=res.out_f32, ps_out=res.ps, mixed_out=res.mixed,
                      n_selected_out=res.n_selected, stream=stream)
+    return res
+
+
+def linear_layernorm(x, W, *, mu: int = 4, tau: float = 0.0, variant: int = LAMP_STRICT, scale: float = 0.0,
+                     eps: float = 0.0, mask_in=None, want_mask: bool = True, want_out_f32: bool = False,
+                     want_scores: bool = False, want_count: bool = False, stream=None) -> GeluOutputs:
+    """LAMP LayerNorm(scale * x W^T) on torch tensors ("Theoretical basis", item 3:
+    layer normalisation, greedy by sorted magnitude). Shapes and extras as for
+    linear_gelu; N <= 8192. y_hat goes to the returned ps tensor when want_scores,
+    else to the library's scratch pool."""
+    import torch
+
+    M, K = x.shape
+    N = W.shape[0]
+    dev = x.device
+    for t in (x, W):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != dev:
+            raise ValueError("x and W must be contiguous bfloat16 tensors on one device")
+    if W.shape[1] != K:
+        raise ValueError("x and W disagree on K")
+    res = GeluOutputs(out=torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+    if want_mask:
+        res.mask = torch.empty((M, (N + 31) // 32), dtype=torch.int32, device=dev)
+    if want_out_f32:
+        res.out_f32 = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if want_scores:
+        res.ps = torch.empty((M, N), dtype=torch.float32, device=dev)
+        res.mixed = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if want_count:
+        res.n_selected = torch.empty(1, dtype=torch.int64, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    lamp_linear_layernorm(M=M, N=N, K=K, x=x, W=W, out=res.out, mask_out=res.mask, mu=mu, tau=tau,
+                          variant=variant, scale=scale, eps=eps, mask_in=mask_in, out_f32=res.out_f32,
+                          ps_out=res.ps, mixed_out=res.mixed, n_selected_out=res.n_selected, stream=stream)
     return res

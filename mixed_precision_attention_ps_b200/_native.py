@@ -92,6 +92,28 @@ class lamp_gelu_args(ctypes.Structure):
     ]
 
 
+class lamp_ln_args(ctypes.Structure):
+    _fields_ = [
+        ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int),
+        ("x", _P), ("W", _P),
+        ("out", _P),
+        ("mask_out", _P),
+        ("mu", ctypes.c_int),
+        ("tau", ctypes.c_float),
+        ("variant", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("mask_in", _P),
+        ("out_f32", _P),
+        ("ps_out", _P),
+        ("mixed_out", _P),
+        ("n_selected_out", _P),
+        ("workspace", _P),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("stream", _P),
+    ]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -108,6 +130,9 @@ SIGNATURES = {
     "lamp_args_size": (ctypes.c_size_t, []),
     "lamp_linear_gelu": (ctypes.c_int, [ctypes.POINTER(lamp_gelu_args)]),
     "lamp_gelu_args_size": (ctypes.c_size_t, []),
+    "lamp_linear_layernorm": (ctypes.c_int, [ctypes.POINTER(lamp_ln_args)]),
+    "lamp_ln_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
+    "lamp_ln_args_size": (ctypes.c_size_t, []),
 }
 
 
@@ -129,6 +154,8 @@ def load(path: str = LIB_PATH):
                 raise ImportError("lamp_args layout of the binding does not match liblamp.so")
             if L.lamp_gelu_args_size() != ctypes.sizeof(lamp_gelu_args):
                 raise ImportError("lamp_gelu_args layout of the binding does not match liblamp.so")
+            if L.lamp_ln_args_size() != ctypes.sizeof(lamp_ln_args):
+                raise ImportError("lamp_ln_args layout of the binding does not match liblamp.so")
             _lib = L
     return _lib
 
@@ -230,4 +257,29 @@ def lamp_linear_gelu(args: lamp_gelu_args | None = None, check: bool = True, **k
     if args is None:
         args = make_gelu_args(**kw)
     rc = load().lamp_linear_gelu(ctypes.byref(args))
+    return _check(rc) if check else rc
+
+
+def lamp_ln_args_size() -> int:
+    return int(load().lamp_ln_args_size())
+
+
+def lamp_ln_workspace_size(M: int, N: int) -> int:
+    return int(load().lamp_ln_workspace_size(int(M), int(N)))
+
+
+def make_ln_args(M, N, K, x, W, out, *, mask_out=None, mu=4, tau=0.0, variant=LAMP_STRICT, scale=0.0, eps=0.0,
+                 mask_in=None, out_f32=None, ps_out=None, mixed_out=None, n_selected_out=None, workspace=None,
+                 workspace_bytes=0, stream=None) -> lamp_ln_args:
+    return lamp_ln_args(int(M), int(N), int(K), _ptr(x), _ptr(W), _ptr(out), _ptr(mask_out), int(mu), float(tau),
+                        int(variant), float(scale), float(eps), _ptr(mask_in), _ptr(out_f32), _ptr(ps_out),
+                        _ptr(mixed_out), _ptr(n_selected_out), _ptr(workspace), int(workspace_bytes),
+                        _stream(stream))
+
+
+def lamp_linear_layernorm(args: lamp_ln_args | None = None, check: bool = True, **kw) -> int:
+    """LAMP LayerNorm(scale * x W^T): pass a lamp_ln_args, or make_ln_args' keyword arguments."""
+    if args is None:
+        args = make_ln_args(**kw)
+    rc = load().lamp_linear_layernorm(ctypes.byref(args))
     return _check(rc) if check else rc

@@ -397,6 +397,86 @@ int lamp_linear_gelu(const lamp_gelu_args* a) {
   return ok();
 }
 
+size_t lamp_ln_args_size(void) { return sizeof(lamp_ln_args); }
+
+size_t lamp_ln_workspace_size(int M, int N) { return (M > 0 && N > 0) ? (size_t)M * (size_t)N * 4 : 0; }
+
+int lamp_linear_layernorm(const lamp_ln_args* a) {
+  if (!a) return fail(LAMP_ERR_ARG, "args is NULL");
+  if (a->M <= 0 || a->N <= 0 || a->K <= 0)
+    return fail(LAMP_ERR_ARG, "dimensions must be positive (M=%d N=%d K=%d)", a->M, a->N, a->K);
+  if (!a->x || !a->W || !a->out) return fail(LAMP_ERR_ARG, "x, W and out must be non-NULL");
+  if (a->mu < 1 || a->mu > 23) return fail(LAMP_ERR_ARG, "mu must be in [1, 23] (got %d)", a->mu);
+  if (a->variant == LAMP_RELAXED) return fail(LAMP_ERR_ARG, "LayerNorm's selection has no relaxed variant");
+  if (a->variant != LAMP_STRICT && a->variant != LAMP_GIVEN_MASK)
+    return fail(LAMP_ERR_ARG, "unknown variant %d", a->variant);
+  if (a->variant == LAMP_STRICT && std::isnan(a->tau)) return fail(LAMP_ERR_ARG, "tau is NaN");
+  if (a->variant == LAMP_GIVEN_MASK && !a->mask_in) return fail(LAMP_ERR_ARG, "LAMP_GIVEN_MASK needs mask_in");
+  if (std::isnan(a->scale) || a->scale < 0.f || std::isinf(a->scale))
+    return fail(LAMP_ERR_ARG, "scale must be 0 (default 1) or a positive finite value");
+  if (std::isnan(a->eps) || a->eps < 0.f || std::isinf(a->eps))
+    return fail(LAMP_ERR_ARG, "eps must be 0 (default 1e-5) or a positive finite value");
+  if (a->K % 8) return fail(LAMP_ERR_UNSUPPORTED, "K must be a multiple of 8 (got %d)", a->K);
+  if (a->N > lamp::kLnMaxN) return fail(LAMP_ERR_UNSUPPORTED, "N must be at most %d", lamp::kLnMaxN);
+  if (a->M > lamp::gelu_max_rows()) return fail(LAMP_ERR_UNSUPPORTED, "M must be at most %d", lamp::gelu_max_rows());
+  if (!aligned(a->x, 16) || !aligned(a->W, 16)) return fail(LAMP_ERR_UNSUPPORTED, "x and W must be 16-byte aligned");
+  if (!aligned(a->out, 2) || (a->mask_out && !aligned(a->mask_out, 4)) || (a->mask_in && !aligned(a->mask_in, 4)) ||
+      (a->out_f32 && !aligned(a->out_f32, 4)) || (a->ps_out && !aligned(a->ps_out, 4)) ||
+      (a->mixed_out && !aligned(a->mixed_out, 4)) || (a->n_selected_out && !aligned(a->n_selected_out, 8)) ||
+      (a->workspace && !aligned(a->workspace, 4)))
+    return fail(LAMP_ERR_UNSUPPORTED, "outputs and workspace must be naturally aligned");
+  const size_t need = lamp_ln_workspace_size(a->M, a->N);
+  if (a->workspace && a->workspace_bytes < need)
+    return fail(LAMP_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu bytes needed", a->workspace_bytes,
+                need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  float* yhat = a->ps_out ? a->ps_out : static_cast<float*>(a->workspace);
+  bool owned = false;
+  if (!yhat) {
+    DeviceInfo info;
+    cudaError_t e = device_info(info);
+    if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
+    cudaMemPool_t pool = nullptr;
+    e = scratch_pool(info.dev, pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&yhat), need, pool, st);
+    if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "workspace allocation failed: %s", cudaGetErrorString(e));
+    owned = true;
+  }
+  lamp::GeluProblem g{};
+  g.M = a->M; g.N = a->N; g.K = a->K;
+  g.mu = a->mu;
+  g.scale = a->scale == 0.f ? 1.f : a->scale;
+  g.variant = LAMP_STRICT;
+  g.x = static_cast<const uint16_t*>(a->x);
+  g.W = static_cast<const uint16_t*>(a->W);
+  g.ps_out = yhat;
+  g.emax_sum_limit = emax_sum_limit(a->mu, a->K);
+  lamp::LnProblem l{};
+  l.M = a->M; l.N = a->N; l.K = a->K;
+  l.tau = a->variant == LAMP_GIVEN_MASK ? 0.f : a->tau;
+  l.scale = g.scale;
+  l.eps = a->eps == 0.f ? 1e-5f : a->eps;
+  l.variant = a->variant;
+  l.x = g.x; l.W = g.W;
+  l.yhat = yhat;
+  l.out = static_cast<uint16_t*>(a->out);
+  l.mask_out = a->mask_out;
+  l.mask_in = a->mask_in;
+  l.out_f32 = a->out_f32;
+  l.mixed_out = a->mixed_out;
+  l.nsel_out = a->n_selected_out;
+  cudaError_t e = cudaSuccess;
+  if (a->n_selected_out) e = cudaMemsetAsync(a->n_selected_out, 0, sizeof(unsigned long long), st);
+  if (e == cudaSuccess) e = lamp::launch_linear_ps(g, st);
+  if (e == cudaSuccess) e = lamp::launch_ln_rows(l, st);
+  if (owned) {
+    cudaError_t fe = cudaFreeAsync(yhat, st);
+    if (e == cudaSuccess) e = fe;
+  }
+  if (e != cudaSuccess) return fail(LAMP_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 int lamp_ps_round(const float* x, float* y, size_t n, int mu, int path, lamp_stream_t stream) {
   if ((!x || !y) && n) return fail(LAMP_ERR_ARG, "x and y must be non-NULL");
   if (mu < 1 || mu > 23) return fail(LAMP_ERR_ARG, "mu must be in [1, 23] (got %d)", mu);

@@ -101,6 +101,25 @@ __device__ __forceinline__ void split_bf16(float p, uint16_t& hi, uint16_t& lo) 
   lo = f32_to_bf16_rne(r);
 }
 
+// The sequential binary32 dot of two bf16 rows of K values (K a multiple of 8,
+// rows 16-byte aligned): one binary32 multiply and one add a step, in order.
+__device__ __forceinline__ float fp32_dot_bf16(const uint16_t* a, const uint16_t* b, int K) {
+  const uint4* aq = reinterpret_cast<const uint4*>(a);
+  const uint4* bq = reinterpret_cast<const uint4*>(b);
+  float s = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < (K >> 3); ++k) {
+    const uint4 u = __ldg(aq + k), v = __ldg(bq + k);
+    const uint32_t uw[4] = {u.x, u.y, u.z, u.w}, vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      s = __fadd_rn(s, __fmul_rn(__uint_as_float(uw[j] << 16), __uint_as_float(vw[j] << 16)));
+      s = __fadd_rn(s, __fmul_rn(__uint_as_float(uw[j] & 0xFFFF0000u), __uint_as_float(vw[j] & 0xFFFF0000u)));
+    }
+  }
+  return s;
+}
+
 // ---------------------------------------------------------------------------
 // Warp reductions.
 // ---------------------------------------------------------------------------

@@ -165,7 +165,11 @@ __device__ __forceinline__ bool gelu_fast_ok(const uint32_t (&r)[4], int emax_su
   return (ex - 127) + (ew - 127) <= emax_sum_limit && lx + lw >= -126;
 }
 
-template <int RND>
+// EPI_GELU: the whole LAMP GELU op. EPI_STORE: only the PS(mu) linear map, its
+// outputs written to p.ps_out (the first half of the LayerNorm op).
+enum { EPI_GELU = 0, EPI_STORE = 1 };
+
+template <int RND, int EPI>
 __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   GeluSmem& sm = *reinterpret_cast<GeluSmem*>(smem_raw);
@@ -216,6 +220,17 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) acc[i][m] = mul2u(acc[i][m], sc2);
   const int row0 = m0 + 8 * warp;
+  if (EPI == EPI_STORE) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int row = row0 + r, col = n0 + lane + 32 * m;
+        if (row < p.M && col < p.N)
+          p.ps_out[(size_t)row * p.N + col] = (r & 1) ? hi_f(acc[r >> 1][m]) : lo_f(acc[r >> 1][m]);
+      }
+    return;
+  }
   const int nw = (p.N + 31) >> 5;
   uint32_t myword = 0u;  // lane 4r + m keeps the ballot of (row r, column group m)
 #pragma unroll
@@ -284,19 +299,7 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
       const int c = __fns(word, 0, slot - before + 1);
       const int r = owner >> 2, m = owner & 3;
       const int row = row0 + r, col = n0 + c + 32 * m;
-      const uint4* xq = reinterpret_cast<const uint4*>(p.x + (size_t)row * p.K);
-      const uint4* wq = reinterpret_cast<const uint4*>(p.W + (size_t)col * p.K);
-      float s = 0.f;  // the sequential binary32 dot: one multiply and one add a step
-#pragma unroll 4
-      for (int k = 0; k < (p.K >> 3); ++k) {
-        const uint4 a = __ldg(xq + k), b = __ldg(wq + k);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          s = __fadd_rn(s, __fmul_rn(__uint_as_float(lo_bits(aw[j])), __uint_as_float(lo_bits(bw[j]))));
-          s = __fadd_rn(s, __fmul_rn(__uint_as_float(hi_bits(aw[j])), __uint_as_float(hi_bits(bw[j]))));
-        }
-      }
+      const float s = fp32_dot_bf16(p.x + (size_t)row * p.K, p.W + (size_t)col * p.K, p.K);
       const float y = __fmul_rn(p.scale, s);
       const size_t o = (size_t)row * p.N + col;
       if (p.mixed_out) p.mixed_out[o] = y;
@@ -307,14 +310,31 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
   }
 }
 
-template <int RND>
+template <int RND, int EPI>
 cudaError_t gelu_launch_one(const GeluArgs& A, cudaStream_t st) {
   const size_t smem = sizeof(GeluSmem);
-  cudaError_t e = cudaFuncSetAttribute(gelu_kernel<RND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(gelu_kernel<RND, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((A.p.N + GL_BN - 1) / GL_BN, (A.p.M + GL_BM - 1) / GL_BM);
-  gelu_kernel<RND><<<grid, GL_T, smem, st>>>(A);
+  gelu_kernel<RND, EPI><<<grid, GL_T, smem, st>>>(A);
   return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t gelu_launch(const GeluProblem& p, cudaStream_t st) {
+  GeluArgs A;
+  A.p = p;
+  A.s = 23 - p.mu;
+  const float c = -(float)((1 << A.s) - 1), q = (float)(1 << A.s);
+  uint32_t cb, qb;
+  std::memcpy(&cb, &c, 4);
+  std::memcpy(&qb, &q, 4);
+  A.negc = ((u64)cb << 32) | cb;
+  A.pow2s = ((u64)qb << 32) | qb;
+  if (p.mu == 23) return gelu_launch_one<kRndNone, EPI>(A, st);
+  if (p.mu <= 10) return gelu_launch_one<kRndFast, EPI>(A, st);
+  return gelu_launch_one<kRndExact, EPI>(A, st);
 }
 
 }  // namespace
@@ -326,18 +346,9 @@ cudaError_t launch_gelu(const GeluProblem& p, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(p.nsel_out, 0, sizeof(unsigned long long), st);
     if (e != cudaSuccess) return e;
   }
-  GeluArgs A;
-  A.p = p;
-  A.s = 23 - p.mu;
-  const float c = -(float)((1 << A.s) - 1), q = (float)(1 << A.s);
-  uint32_t cb, qb;
-  std::memcpy(&cb, &c, 4);
-  std::memcpy(&qb, &q, 4);
-  A.negc = ((u64)cb << 32) | cb;
-  A.pow2s = ((u64)qb << 32) | qb;
-  if (p.mu == 23) return gelu_launch_one<kRndNone>(A, st);
-  if (p.mu <= 10) return gelu_launch_one<kRndFast>(A, st);
-  return gelu_launch_one<kRndExact>(A, st);
+  return gelu_launch<EPI_GELU>(p, st);
 }
+
+cudaError_t launch_linear_ps(const GeluProblem& p, cudaStream_t st) { return gelu_launch<EPI_STORE>(p, st); }
 
 }  // namespace lamp

@@ -110,6 +110,30 @@ struct GeluProblem {
   int emax_sum_limit;  // largest e_x + e_w for which the two-instruction rounding is exact
 };
 cudaError_t launch_gelu(const GeluProblem& p, cudaStream_t st);
+// The PS(mu) linear map alone: fl32(scale * x W^T) written to p.ps_out [M, N].
+cudaError_t launch_linear_ps(const GeluProblem& p, cudaStream_t st);
 int gelu_max_rows();
+
+// LAMP LayerNorm((y_hat -> greedy recompute) of scale * x W^T), per row, after
+// launch_linear_ps has written y_hat.
+struct LnProblem {
+  int M, N, K;
+  float tau;
+  float scale;
+  float eps;
+  int variant;  // LAMP_STRICT (the greedy selection) or LAMP_GIVEN_MASK
+  const uint16_t* x;
+  const uint16_t* W;
+  const float* yhat;  // [M, N], written by launch_linear_ps
+  uint16_t* out;
+  uint32_t* mask_out;
+  const uint32_t* mask_in;
+  float* out_f32;
+  float* ps_out;      // the caller's copy of y_hat, when it is not yhat itself
+  float* mixed_out;
+  unsigned long long* nsel_out;
+};
+cudaError_t launch_ln_rows(const LnProblem& p, cudaStream_t st);
+constexpr int kLnMaxN = 8192;
 
 }  // namespace lamp

@@ -39,6 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_struct_layout_matches(lib):
     assert lamp.lamp_args_size() == ctypes.sizeof(_native.lamp_args) == 168
     assert lamp.lamp_gelu_args_size() == ctypes.sizeof(_native.lamp_gelu_args) == 112
+    assert lamp.lamp_ln_args_size() == ctypes.sizeof(_native.lamp_ln_args) == 136
     assert lamp.lamp_version().startswith("lamp-b200")
 
 
@@ -139,3 +140,34 @@ def test_gelu_argument_checks(lib, kw, code, msg):
 
 def test_gelu_null_args(lib):
     assert _native.load().lamp_linear_gelu(None) == lamp.LAMP_ERR_ARG
+
+
+def call_ln(**kw):
+    base = dict(M=4, N=40, K=16, x=FAKE, W=FAKE, out=FAKE, mu=4, tau=1.0)
+    base.update(kw)
+    return lamp.lamp_linear_layernorm(check=False, **base)
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(W=None), lamp.LAMP_ERR_ARG, "non-NULL"),
+    (dict(N=0), lamp.LAMP_ERR_ARG, "positive"),
+    (dict(mu=0), lamp.LAMP_ERR_ARG, "mu"),
+    (dict(variant=lamp.LAMP_RELAXED), lamp.LAMP_ERR_ARG, "relaxed"),
+    (dict(tau=float("nan")), lamp.LAMP_ERR_ARG, "tau"),
+    (dict(variant=lamp.LAMP_GIVEN_MASK), lamp.LAMP_ERR_ARG, "mask_in"),
+    (dict(eps=-1.0), lamp.LAMP_ERR_ARG, "eps"),
+    (dict(scale=float("nan")), lamp.LAMP_ERR_ARG, "scale"),
+    (dict(K=20), lamp.LAMP_ERR_UNSUPPORTED, "multiple of 8"),
+    (dict(N=8193), lamp.LAMP_ERR_UNSUPPORTED, "at most 8192"),
+    (dict(x=FAKE + 2), lamp.LAMP_ERR_UNSUPPORTED, "16-byte"),
+    (dict(workspace=FAKE + 2), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
+    (dict(workspace=FAKE, workspace_bytes=4 * 40 * 4 - 1), lamp.LAMP_ERR_WORKSPACE, "smaller"),
+])
+def test_ln_argument_checks(lib, kw, code, msg):
+    assert call_ln(**kw) == code
+    assert msg in lamp.lamp_last_error()
+
+
+def test_ln_workspace_size(lib):
+    assert lamp.lamp_ln_workspace_size(1024, 1600) == 1024 * 1600 * 4
+    assert lamp.lamp_ln_workspace_size(0, 5) == 0
