@@ -18,8 +18,9 @@ between steps outside the events; the max over ranks is reported.
 --impl reference times the CPU oracle (the plain C definition of the method)
 on this host's cores on a bounded sample of the same workload.
 
-The gelu_* workloads time LAMP on an elementwise activation instead (GELU after
-a PS(mu) linear map), with the same contract.
+The gelu_* and ln_* workloads time LAMP on an elementwise activation (GELU after
+a PS(mu) linear map) and on LayerNorm after a PS(mu) linear map, with the same
+contract.
 """
 from __future__ import annotations
 
@@ -77,6 +78,8 @@ DEFAULTS = {  # workload -> (variant, rate)
     "single_head_128": (0, None),
     "gelu_gpt2xl_fc_1024x6400x1600": (0, 0.016),
     "gelu_small_96x300x200": (0, 0.016),
+    "ln_gpt2xl_proj_1024x1600x1600": (0, 0.016),
+    "ln_small_64x300x128": (0, 0.016),
 }
 
 
@@ -524,21 +527,25 @@ def cpu_baseline(w, Q, K, V, mu, tau, variant) -> dict:
 # ----------------------------------------------------------------------------------------
 # LAMP on an elementwise activation: GELU(scale * x W^T), the linear map in PS(mu)
 # ----------------------------------------------------------------------------------------
-def gelu_metric(lw, mu) -> str:
-    return f"LAMP GELU(x W^T) G-outputs/s at {lw.M}x{lw.N}x{lw.K} mu={mu}; % of roofline"
+def gelu_metric(lw, mu, op="gelu") -> str:
+    name = "LayerNorm" if op == "ln" else "GELU"
+    return f"LAMP {name}(x W^T) G-outputs/s at {lw.M}x{lw.N}x{lw.K} mu={mu}; % of roofline"
 
 
 GELU_UNIT = "G-outputs/s"
 
 
-def gelu_oracle_pass(lw, x, W, mu, tau, rows, threads) -> float:
+def gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op="gelu") -> float:
     import oracle
     t0 = time.perf_counter()
-    oracle.linear_gelu_rows(x, W, scale=lw.scale, mu=mu, tau=tau, rows=rows, threads=threads)
+    if op == "ln":
+        oracle.linear_ln_rows(x, W, scale=lw.scale, mu=mu, tau=tau, rows=rows, threads=threads)
+    else:
+        oracle.linear_gelu_rows(x, W, scale=lw.scale, mu=mu, tau=tau, rows=rows, threads=threads)
     return time.perf_counter() - t0
 
 
-def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0) -> dict:
+def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0, op="gelu") -> dict:
     """The activation oracle as it stands, on the host's cores, over a row sample
     repeated until about `seconds` of work have run."""
     threads = os.cpu_count() or 1
@@ -546,7 +553,7 @@ def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0) -> dict:
     rows = np.arange(0, lw.M, m, dtype=np.int64)
     t_all, n_out, passes = 0.0, 0, 0
     while t_all < seconds and passes < 20:
-        t_all += gelu_oracle_pass(lw, x, W, mu, tau, rows, threads)
+        t_all += gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op)
         n_out += rows.size * lw.N
         passes += 1
     return {"value": n_out / t_all / 1e9, "unit": GELU_UNIT, "cores": threads, "kind": "oracle",
@@ -554,14 +561,16 @@ def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0) -> dict:
                       f"outputs each), {t_all:.1f} s"}
 
 
-def gelu_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream) -> dict:
+def gelu_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream, op="gelu") -> dict:
     """Errors against the all-FP32 outputs (tau < 0) for no recompute, LAMP at tau and
     a random choice of the same per-row count, on a row sample (outside the timed region)."""
     import oracle
 
+    fn = lamp.linear_layernorm if op == "ln" else lamp.linear_gelu
+
     def run(**kw):
-        r = lamp.linear_gelu(xd, Wd, mu=mu, scale=lw.scale, want_scores=True, want_out_f32=True,
-                             want_count=True, stream=stream, **kw)
+        r = fn(xd, Wd, mu=mu, scale=lw.scale, want_scores=True, want_out_f32=True, want_count=True, stream=stream,
+               **kw)
         torch.cuda.synchronize()
         return r
 
@@ -575,15 +584,20 @@ def gelu_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream) -> dict:
     rmask = S.linear_random_mask(lw, per_row)
     rr = run(tau=0.0, variant=2, mask_in=torch.from_numpy(rmask.view(np.int32)).to(xd.device))
     r_out, r_y = pick(ref.out_f32), pick(ref.mixed)
-    err = {k: oracle.act_errors(pick(v.out_f32), pick(v.mixed), r_out, r_y)
-           for k, v in (("ps_only", base), ("lamp", lr), ("random_same_count", rr))}
+    cases = (("ps_only", base), ("lamp", lr), ("random_same_count", rr))
+    if op == "ln":
+        err = {k: oracle.ln_errors(pick(v.out_f32), r_out) for k, v in cases}
+        key = "mean_l2"
+    else:
+        err = {k: oracle.act_errors(pick(v.out_f32), pick(v.mixed), r_out, r_y) for k, v in cases}
+        key = "max_amp"
     return {"recompute_rate": lr.n_selected.item() / lw.outputs(), "rows_sampled": int(rows.numel()),
             "errors_vs_fp32": err,
-            "max_amp_reduction_lamp": err["ps_only"]["max_amp"] / max(err["lamp"]["max_amp"], 1e-300),
-            "max_amp_reduction_random": err["ps_only"]["max_amp"] / max(err["random_same_count"]["max_amp"], 1e-300)}
+            f"{key}_reduction_lamp": err["ps_only"][key] / max(err["lamp"][key], 1e-300),
+            f"{key}_reduction_random": err["ps_only"][key] / max(err["random_same_count"][key], 1e-300)}
 
 
-def run_gelu_reference(a, lw, mu, tau, cfg):
+def run_gelu_reference(a, lw, mu, tau, cfg, op="gelu"):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
@@ -592,12 +606,12 @@ def run_gelu_reference(a, lw, mu, tau, cfg):
     m = max(1, lw.M // max(1, int(1.6e8 // (lw.N * lw.K))))
     rows = np.arange(0, lw.M, m, dtype=np.int64)
     for _ in range(a.warmup):
-        gelu_oracle_pass(lw, x, W, mu, tau, rows, threads)
-    times = [gelu_oracle_pass(lw, x, W, mu, tau, rows, threads) for _ in range(a.steps)]
+        gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op)
+    times = [gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op) for _ in range(a.steps)]
     ms = 1e3 * statistics.mean(times)
     value = rows.size * lw.N / (ms * 1e-3) / 1e9
     sample = f"{rows.size} of {lw.M} rows (every {m}th), {rows.size * lw.N} outputs per step"
-    line = {"metric": gelu_metric(lw, mu), "value": value, "unit": GELU_UNIT, "n_gpus": a.gpus, "steps": a.steps,
+    line = {"metric": gelu_metric(lw, mu, op), "value": value, "unit": GELU_UNIT, "n_gpus": a.gpus, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg, "impl": "reference",
             "cpu_baseline": {"value": value, "unit": GELU_UNIT, "cores": threads, "kind": "oracle", "sample": sample},
@@ -606,7 +620,7 @@ def run_gelu_reference(a, lw, mu, tau, cfg):
     return 0
 
 
-def run_gelu_ours(a, lw, mu, tau, cfg):
+def run_gelu_ours(a, lw, mu, tau, cfg, op="gelu"):
     import torch
     import torch.distributed as dist
 
@@ -632,9 +646,19 @@ def run_gelu_ours(a, lw, mu, tau, cfg):
     mask = torch.empty((lw.M, (lw.N + 31) // 32), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    args = lamp.make_gelu_args(lw.M, lw.N, lw.K, xd, Wd, out, mask_out=mask, mu=mu, tau=tau, scale=lw.scale,
-                               stream=stream)
-    call = lambda: lamp.lamp_linear_gelu(args)  # noqa: E731
+    ws_bytes = lamp.lamp_ln_workspace_size(lw.M, lw.N) if op == "ln" else 0
+
+    def make(x_, W_, out_, mask_, st_):
+        if op == "ln":  # the LayerNorm op's y_hat scratch comes from the caller here
+            wsb = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+            return (lamp.make_ln_args(lw.M, lw.N, lw.K, x_, W_, out_, mask_out=mask_, mu=mu, tau=tau,
+                                      scale=lw.scale, workspace=wsb, workspace_bytes=ws_bytes, stream=st_), wsb)
+        return lamp.make_gelu_args(lw.M, lw.N, lw.K, x_, W_, out_, mask_out=mask_, mu=mu, tau=tau, scale=lw.scale,
+                                   stream=st_), None
+
+    entry = lamp.lamp_linear_layernorm if op == "ln" else lamp.lamp_linear_gelu
+    args, keep = make(xd, Wd, out, mask, stream)
+    call = lambda: entry(args)  # noqa: E731
 
     props = torch.cuda.get_device_properties(dev)
     clocks = ClockSampler(getattr(props, "uuid", None) and ("GPU-" + str(props.uuid)))
@@ -672,8 +696,7 @@ def run_gelu_ours(a, lw, mu, tau, cfg):
         sets = [(torch.empty_like(xd), torch.empty_like(Wd), torch.empty_like(out), torch.empty_like(mask))
                 for _ in range(2)]
         s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        bargs = [lamp.make_gelu_args(lw.M, lw.N, lw.K, st[0], st[1], st[2], mask_out=st[3], mu=mu, tau=tau,
-                                     scale=lw.scale, stream=s_cmp) for st in sets]
+        bargs = [make(st[0], st[1], st[2], st[3], s_cmp) for st in sets]
 
         def pipeline(n):
             done_in = [torch.cuda.Event() for _ in range(n)]
@@ -691,7 +714,7 @@ def run_gelu_ours(a, lw, mu, tau, cfg):
                 s_cmp.wait_event(done_in[i])
                 if i >= 2:
                     s_cmp.wait_event(done_out[i - 2])
-                lamp.lamp_linear_gelu(bargs[b])
+                entry(bargs[b][0])
                 done_cmp[i].record(s_cmp)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(done_cmp[i])
@@ -726,42 +749,46 @@ def run_gelu_ours(a, lw, mu, tau, cfg):
         achieved = 4.0 * lw.K * n_out / (ms * 1e-3) / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s", "frac": achieved / peak,
                 "traffic": traffic_bytes(a.workload, 0, mu),
-                "kernel": "gelu_kernel (one launch per call)",
+                "kernel": ("one call: the linear-map kernel (gelu_kernel, store epilogue) + ln_rows_kernel"
+                           if op == "ln" else "gelu_kernel (one launch per call)"),
                 "peak_basis": f"148 SMs x 128 lanes/clk x {f_max / 1e6:.0f} MHz (max SM clock); 4 K lane-ops "
                               "per output (K steps of 1 multiply-add + 3 integer ops of the rounding)"}
-        result = {"metric": gelu_metric(lw, mu), "value": value, "unit": GELU_UNIT, "n_gpus": world, "steps": a.steps,
+        result = {"metric": gelu_metric(lw, mu, op), "value": value, "unit": GELU_UNIT, "n_gpus": world, "steps": a.steps,
                   "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                   "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg, "clocks": clk,
-                  "roofline": roof, "gpu_launches": a.steps,
+                  "roofline": roof, "gpu_launches": (2 if op == "ln" else 1) * a.steps,
                   "e2e": {"value": job_value(world, n_out, ms_e2e), "unit": GELU_UNIT,
                           "h2d_bytes_per_step": x.nbytes + W.nbytes,
                           "d2h_bytes_per_step": out.numel() * 2 + mask.numel() * 4, "ms_per_step": ms_e2e,
                           "form": "pipelined: 2 buffer sets, H2D / compute / D2H streams"},
                   "ms_p10_p90": [float(np.percentile(times, 10)), float(np.percentile(times, 90))]}
         if not a.no_kl:
-            result["accuracy"] = gelu_accuracy(lamp, torch, lwr, xd, Wd, mu, tau, stream)
+            result["accuracy"] = gelu_accuracy(lamp, torch, lwr, xd, Wd, mu, tau, stream, op)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         if not a.no_cpu_baseline and world == 1:
-            result["cpu_baseline"] = gelu_cpu_baseline(lwr, x, W, mu, tau)
+            result["cpu_baseline"] = gelu_cpu_baseline(lwr, x, W, mu, tau, op=op)
         print(json.dumps(result), flush=True)
     return 0
 
 
 def main_gelu(a):
     lw = S.LINEAR_WORKLOADS[a.workload]
+    op = "ln" if a.workload.startswith("ln_") else "gelu"
     _, drate = DEFAULTS[a.workload]
     rate = drate if a.rate is None else a.rate
     tau, rate = lookup_tau(a.workload, 0, a.mu, rate)
-    cfg = {"workload": a.workload, "M": lw.M, "N": lw.N, "K": lw.K, "op": "GELU (tanh form) of scale * x W^T",
-           "scale": lw.scale, "variant": "kappa test", "mu": a.mu, "tau": tau, "target_recompute_rate": rate,
+    cfg = {"workload": a.workload, "M": lw.M, "N": lw.N, "K": lw.K,
+           "op": ("LayerNorm (no affine, eps = 1e-5) of scale * x W^T, greedy by sorted magnitude" if op == "ln"
+                  else "GELU (tanh form) of scale * x W^T, kappa test"),
+           "scale": lw.scale, "mu": a.mu, "tau": tau, "target_recompute_rate": rate,
            "inputs": "bf16 N(0,1) x and W (SplitMix64 + Box-Muller), seed = rank",
            "l2": "flushed between steps (256 MB write)", "outputs_per_step_per_gpu": lw.outputs()}
     if a.impl == "reference":
-        return run_gelu_reference(a, lw, a.mu, tau, cfg)
-    return run_gelu_ours(a, lw, a.mu, tau, cfg)
+        return run_gelu_reference(a, lw, a.mu, tau, cfg, op)
+    return run_gelu_ours(a, lw, a.mu, tau, cfg, op)
 
 
 def main():

@@ -6,9 +6,10 @@
 // condition number kappa_j = |y_j f'(y_j) / f(y_j)|) and "Implementation
 // strategy" steps 1-3 (low-precision g, look-ahead selection, recompute).
 //
-// One CTA of 256 threads computes a 64 x 128 tile of outputs over the whole K:
-// warp w owns rows 8w .. 8w+7 of the tile, lane l the columns l + 32m (m < 4),
-// so that a ballot over a (row, m) is one mask word. Slices of 32 dimensions of
+// One CTA of 256 threads computes a 64 x (32 NM) tile of outputs over the whole
+// K (NM = 4, or 2 when 128-wide tiles would leave SMs idle): warp w owns rows
+// 8w .. 8w+7 of the tile, lane l the columns l + 32m (m < NM), so that a ballot
+// over a (row, m) is one mask word. Slices of 32 dimensions of
 // x and W are staged global -> registers -> shared memory as binary32 (W as
 // (w, w) pairs), one slice ahead; a step is packed over two rows: fma.rn.f32x2
 // of the exact bf16 products, then the PS(mu) rounding of the pair.
@@ -24,7 +25,7 @@
 namespace lamp {
 namespace {
 
-constexpr int GL_BM = 64, GL_BN = 128, GL_KS = 32, GL_T = 256;
+constexpr int GL_BM = 64, GL_KS = 32, GL_T = 256;
 constexpr float kGeluC = 0.7978845608028654f;   // sqrt(2 / pi)
 constexpr float kGeluA = 0.044715f;
 constexpr double kGeluCd = 0.7978845608028654;  // sqrt(2 / pi) in double
@@ -33,15 +34,17 @@ constexpr double kGeluAd = 0.044715;
 // term added to 1): inside twice that band the test is taken again in double.
 constexpr float kKappaBand = 4e-5f;
 
+template <int NM>
 struct GeluSmem {
-  float xs[2][GL_KS][GL_BM];  // x slice: [dim][row], so a row pair is one 8-byte word
-  u64 ws[2][GL_KS][GL_BN];    // W slice: [dim][col] as (w, w)
+  float xs[2][GL_KS][GL_BM];   // x slice: [dim][row], so a row pair is one 8-byte word
+  u64 ws[2][GL_KS][32 * NM];   // W slice: [dim][col] as (w, w)
 };
 
 struct GeluArgs {
   GeluProblem p;
   u64 negc, pow2s;  // the two-instruction rounding's constants, as pairs
   int s;            // 23 - mu
+  int num_sms;      // of the device (host side: the tile-width choice)
 };
 
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
@@ -87,24 +90,25 @@ __device__ __forceinline__ float gelu_f(float y) {
 // The K loop: acc[p][m] accumulates rows (8w + 2p, 8w + 2p + 1) of the tile
 // against column lane + 32m, in PS(mu) steps of the given mode, sequentially
 // over k. FOLD collects the operands' magnitude range for the rounding test.
-template <int MODE, bool FOLD>
-__device__ __forceinline__ void gelu_mainloop(const GeluArgs& A, GeluSmem& sm, int m0, int n0, u64 (&acc)[4][4],
-                                              uint32_t (&rng)[4]) {
+template <int MODE, bool FOLD, int NM>
+__device__ __forceinline__ void gelu_mainloop(const GeluArgs& A, GeluSmem<NM>& sm, int m0, int n0,
+                                              u64 (&acc)[4][NM], uint32_t (&rng)[4]) {
+  constexpr int BN = 32 * NM, WL = NM / 2;  // W: each thread stages WL groups of 8 dimensions
   const GeluProblem& p = A.p;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int xr = t & 63, xc = t >> 6;          // x: row xr, dims 8 xc .. 8 xc + 7 of a slice
-  const int wc = t & 127, wq = (t >> 7) * 2;   // W: col wc, dims 8 wq .. 8 wq + 15
+  const int xr = t & 63, xc = t >> 6;                // x: row xr, dims 8 xc .. 8 xc + 7 of a slice
+  const int wc = t % BN, wq = (t / BN) * WL;         // W: col wc, dims 8 wq .. 8 (wq + WL) - 1
   const bool xin = m0 + xr < p.M, win = n0 + wc < p.N;
   const uint16_t* xp = p.x + (size_t)(xin ? m0 + xr : 0) * p.K + 8 * xc;
   const uint16_t* wp = p.W + (size_t)(win ? n0 + wc : 0) * p.K + 8 * wq;
   const int nsl = (p.K + GL_KS - 1) / GL_KS;
   const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-  uint4 rx, rw0, rw1;
+  uint4 rx, rw[WL];
   auto load = [&](int sl) {
     const int k = sl * GL_KS;
     rx = (xin && k + 8 * xc < p.K) ? ldg16(xp + k) : z4;
-    rw0 = (win && k + 8 * wq < p.K) ? ldg16(wp + k) : z4;
-    rw1 = (win && k + 8 * wq + 8 < p.K) ? ldg16(wp + k + 8) : z4;
+#pragma unroll
+    for (int g = 0; g < WL; ++g) rw[g] = (win && k + 8 * (wq + g) < p.K) ? ldg16(wp + k + 8 * g) : z4;
   };
   auto store = [&](int buf) {
     const uint32_t xw[4] = {rx.x, rx.y, rx.z, rx.w};
@@ -115,19 +119,22 @@ __device__ __forceinline__ void gelu_mainloop(const GeluArgs& A, GeluSmem& sm, i
       sm.xs[buf][8 * xc + 2 * j + 1][xr] = __uint_as_float(b);
       if (FOLD) { fold(rng[0], rng[1], a); fold(rng[0], rng[1], b); }
     }
-    const uint32_t ww[8] = {rw0.x, rw0.y, rw0.z, rw0.w, rw1.x, rw1.y, rw1.z, rw1.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t a = lo_bits(ww[j]), b = hi_bits(ww[j]);
-      sm.ws[buf][8 * wq + 2 * j][wc] = ((u64)a << 32) | a;
-      sm.ws[buf][8 * wq + 2 * j + 1][wc] = ((u64)b << 32) | b;
-      if (FOLD) { fold(rng[2], rng[3], a); fold(rng[2], rng[3], b); }
+    for (int g = 0; g < WL; ++g) {
+      const uint32_t ww[4] = {rw[g].x, rw[g].y, rw[g].z, rw[g].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t a = lo_bits(ww[j]), b = hi_bits(ww[j]);
+        sm.ws[buf][8 * (wq + g) + 2 * j][wc] = ((u64)a << 32) | a;
+        sm.ws[buf][8 * (wq + g) + 2 * j + 1][wc] = ((u64)b << 32) | b;
+        if (FOLD) { fold(rng[2], rng[3], a); fold(rng[2], rng[3], b); }
+      }
     }
   };
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int m = 0; m < 4; ++m) acc[i][m] = 0ull;
+    for (int m = 0; m < NM; ++m) acc[i][m] = 0ull;
   load(0);
   store(0);
   __syncthreads();
@@ -139,13 +146,13 @@ __device__ __forceinline__ void gelu_mainloop(const GeluArgs& A, GeluSmem& sm, i
       const ulonglong2 xa = *reinterpret_cast<const ulonglong2*>(&sm.xs[buf][k][8 * warp]);
       const ulonglong2 xb = *reinterpret_cast<const ulonglong2*>(&sm.xs[buf][k][8 * warp + 4]);
       const u64 xq[4] = {xa.x, xa.y, xb.x, xb.y};
-      u64 wd[4];
+      u64 wd[NM];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) wd[m] = sm.ws[buf][k][lane + 32 * m];
+      for (int m = 0; m < NM; ++m) wd[m] = sm.ws[buf][k][lane + 32 * m];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int m = 0; m < 4; ++m) acc[i][m] = ps_step<MODE>(xq[i], wd[m], acc[i][m], A.negc, A.pow2s, A.s);
+        for (int m = 0; m < NM; ++m) acc[i][m] = ps_step<MODE>(xq[i], wd[m], acc[i][m], A.negc, A.pow2s, A.s);
     }
     // buf ^ 1 was last read before the barrier that ended the previous slice
     if (sl + 1 < nsl) store(buf ^ 1);
@@ -169,16 +176,17 @@ __device__ __forceinline__ bool gelu_fast_ok(const uint32_t (&r)[4], int emax_su
 // outputs written to p.ps_out (the first half of the LayerNorm op).
 enum { EPI_GELU = 0, EPI_STORE = 1 };
 
-template <int RND, int EPI>
-__global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
+template <int RND, int EPI, int NM>
+__global__ void __launch_bounds__(GL_T, NM == 4 ? 2 : 3) gelu_kernel(const GeluArgs A) {
+  constexpr int BN = 32 * NM;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  GeluSmem& sm = *reinterpret_cast<GeluSmem*>(smem_raw);
+  GeluSmem<NM>& sm = *reinterpret_cast<GeluSmem<NM>*>(smem_raw);
   __shared__ uint32_t red[GL_T / 32][4];
   __shared__ int fast_sh;
   const GeluProblem& p = A.p;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int n0 = blockIdx.x * GL_BN, m0 = blockIdx.y * GL_BM;
-  u64 acc[4][4];
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * GL_BM;
+  u64 acc[4][NM];
   uint32_t rng[4] = {0u, 0xFFFFFFFFu, 0u, 0xFFFFFFFFu};
 
   // step 1: the low-precision linear map. The fused forms (the two-instruction
@@ -187,10 +195,10 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
   // that are not exact in binary32, partial sums outside the rounding's domain)
   // is computed again with one binary32 multiply, add and exact rounding a step.
   if (RND == kRndExact) {
-    gelu_mainloop<kStepExact, false>(A, sm, m0, n0, acc, rng);
+    gelu_mainloop<kStepExact, false, NM>(A, sm, m0, n0, acc, rng);
   } else {
-    if (RND == kRndNone) gelu_mainloop<kStepF32, true>(A, sm, m0, n0, acc, rng);
-    else gelu_mainloop<kStepFast, true>(A, sm, m0, n0, acc, rng);
+    if (RND == kRndNone) gelu_mainloop<kStepF32, true, NM>(A, sm, m0, n0, acc, rng);
+    else gelu_mainloop<kStepFast, true, NM>(A, sm, m0, n0, acc, rng);
     rng[0] = __reduce_max_sync(0xFFFFFFFFu, rng[0]);
     rng[1] = __reduce_min_sync(0xFFFFFFFFu, rng[1]);
     rng[2] = __reduce_max_sync(0xFFFFFFFFu, rng[2]);
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
     }
     __syncthreads();
     if (!fast_sh)  // outside the two-instruction rounding's domain: again, exactly
-      gelu_mainloop<kStepExact, false>(A, sm, m0, n0, acc, rng);
+      gelu_mainloop<kStepExact, false, NM>(A, sm, m0, n0, acc, rng);
   }
 
   // step 2: the condition number of each output, and the selection
@@ -218,13 +226,13 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int m = 0; m < 4; ++m) acc[i][m] = mul2u(acc[i][m], sc2);
+    for (int m = 0; m < NM; ++m) acc[i][m] = mul2u(acc[i][m], sc2);
   const int row0 = m0 + 8 * warp;
   if (EPI == EPI_STORE) {
 #pragma unroll
     for (int r = 0; r < 8; ++r)
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
+      for (int m = 0; m < NM; ++m) {
         const int row = row0 + r, col = n0 + lane + 32 * m;
         if (row < p.M && col < p.N)
           p.ps_out[(size_t)row * p.N + col] = (r & 1) ? hi_f(acc[r >> 1][m]) : lo_f(acc[r >> 1][m]);
@@ -232,12 +240,12 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
     return;
   }
   const int nw = (p.N + 31) >> 5;
-  uint32_t myword = 0u;  // lane 4r + m keeps the ballot of (row r, column group m)
+  uint32_t myword = 0u;  // lane NM r + m keeps the ballot of (row r, column group m)
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
     const int row = row0 + r;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
+    for (int m = 0; m < NM; ++m) {
       const int col = n0 + lane + 32 * m;
       const float y = (r & 1) ? hi_f(acc[r >> 1][m]) : lo_f(acc[r >> 1][m]);
       const bool valid = row < p.M && col < p.N;
@@ -254,7 +262,7 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
         sel = sel && valid;
       }
       const uint32_t b = __ballot_sync(0xFFFFFFFFu, sel);
-      if (lane == 4 * r + m) myword = b;
+      if (lane == NM * r + m) myword = b;
       if (valid) {
         const size_t o = (size_t)row * p.N + col;
         if (p.ps_out) p.ps_out[o] = y;
@@ -268,8 +276,9 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
     }
   }
   {
-    const int r = lane >> 2, m = lane & 3;
-    if (p.mask_out && row0 + r < p.M && (n0 >> 5) + m < nw) p.mask_out[(size_t)(row0 + r) * nw + (n0 >> 5) + m] = myword;
+    const int r = lane / NM, m = lane % NM;
+    if (p.mask_out && lane < 8 * NM && row0 + r < p.M && (n0 >> 5) + m < nw)
+      p.mask_out[(size_t)(row0 + r) * nw + (n0 >> 5) + m] = myword;
   }
 
   // step 3: recompute the selected outputs in binary32, 32 per round over the warp
@@ -297,9 +306,9 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
     const int before = __shfl_sync(0xFFFFFFFFu, incl - cnt, owner);
     if (slot < total) {
       const int c = __fns(word, 0, slot - before + 1);
-      const int r = owner >> 2, m = owner & 3;
+      const int r = owner / NM, m = owner % NM;
       const int row = row0 + r, col = n0 + c + 32 * m;
-      const float s = fp32_dot_bf16(p.x + (size_t)row * p.K, p.W + (size_t)col * p.K, p.K);
+      const float s = fp32_dot_bf16<0>(p.x + (size_t)row * p.K, p.W + (size_t)col * p.K, p.K);
       const float y = __fmul_rn(p.scale, s);
       const size_t o = (size_t)row * p.N + col;
       if (p.mixed_out) p.mixed_out[o] = y;
@@ -310,15 +319,26 @@ __global__ void __launch_bounds__(GL_T, 2) gelu_kernel(const GeluArgs A) {
   }
 }
 
+template <int RND, int EPI, int NM>
+cudaError_t gelu_launch_nm(const GeluArgs& A, cudaStream_t st) {
+  const size_t smem = sizeof(GeluSmem<NM>);
+  cudaError_t e =
+      cudaFuncSetAttribute(gelu_kernel<RND, EPI, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((A.p.N + 32 * NM - 1) / (32 * NM), (A.p.M + GL_BM - 1) / GL_BM);
+  gelu_kernel<RND, EPI, NM><<<grid, GL_T, smem, st>>>(A);
+  return cudaGetLastError();
+}
+
+// Tile width: the narrower tiles when they cut the largest per-SM share of the
+// outputs (whole tiles a SM runs, times the tile's size) by an eighth or more.
 template <int RND, int EPI>
 cudaError_t gelu_launch_one(const GeluArgs& A, cudaStream_t st) {
-  const size_t smem = sizeof(GeluSmem);
-  cudaError_t e =
-      cudaFuncSetAttribute(gelu_kernel<RND, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  const dim3 grid((A.p.N + GL_BN - 1) / GL_BN, (A.p.M + GL_BM - 1) / GL_BM);
-  gelu_kernel<RND, EPI><<<grid, GL_T, smem, st>>>(A);
-  return cudaGetLastError();
+  const long long rt = (A.p.M + GL_BM - 1) / GL_BM;
+  const long long t4 = rt * ((A.p.N + 127) / 128), t2 = rt * ((A.p.N + 63) / 64);
+  const long long share4 = (t4 + A.num_sms - 1) / A.num_sms * 2, share2 = (t2 + A.num_sms - 1) / A.num_sms;
+  if (8 * share2 <= 7 * share4) return gelu_launch_nm<RND, EPI, 2>(A, st);
+  return gelu_launch_nm<RND, EPI, 4>(A, st);
 }
 
 template <int EPI>
@@ -326,6 +346,9 @@ cudaError_t gelu_launch(const GeluProblem& p, cudaStream_t st) {
   GeluArgs A;
   A.p = p;
   A.s = 23 - p.mu;
+  int dev = 0;
+  A.num_sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&A.num_sms, cudaDevAttrMultiProcessorCount, dev);
   const float c = -(float)((1 << A.s) - 1), q = (float)(1 << A.s);
   uint32_t cb, qb;
   std::memcpy(&cb, &c, 4);

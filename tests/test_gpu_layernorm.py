@@ -199,3 +199,12 @@ def test_ln_gpt2xl_proj_sampled(rate):
     rows = np.sort(np.random.default_rng(66).choice(lw.M, size=24, replace=False))
     g, orc, nsel = run_case(lw, 4, e["tau"], rows=rows)
     assert g.count() == e["selected_at_tau"]
+
+
+def test_ln_wide_tiles_of_the_linear_map():
+    """A shape whose linear map takes the 128-wide tiles (800 of them) and rows of
+    6400 outputs; sampled rows."""
+    lw = S.LinearWorkload(1024, 6400, 64, seed=67)
+    rows = np.array([0, 1, 63, 64, 500, 1023])
+    g, orc, nsel = run_case(lw, 4, 72.0, rows=rows)
+    assert 0 < nsel
