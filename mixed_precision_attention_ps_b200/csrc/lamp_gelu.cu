@@ -45,6 +45,8 @@ struct GeluArgs {
   u64 negc, pow2s;  // the two-instruction rounding's constants, as pairs
   int s;            // 23 - mu
   int num_sms;      // of the device (host side: the tile-width choice)
+  long long tile0;  // first tile of this launch, in row-major (row tile, column tile) order
+  int ctiles;       // column tiles per row tile at this launch's width
 };
 
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
@@ -185,7 +187,8 @@ __global__ void __launch_bounds__(GL_T, NM == 4 ? 2 : 3) gelu_kernel(const GeluA
   __shared__ int fast_sh;
   const GeluProblem& p = A.p;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * GL_BM;
+  const long long tile = A.tile0 + blockIdx.x;
+  const int n0 = (int)(tile % A.ctiles) * BN, m0 = (int)(tile / A.ctiles) * GL_BM;
   u64 acc[4][NM];
   uint32_t rng[4] = {0u, 0xFFFFFFFFu, 0u, 0xFFFFFFFFu};
 
@@ -320,25 +323,39 @@ __global__ void __launch_bounds__(GL_T, NM == 4 ? 2 : 3) gelu_kernel(const GeluA
 }
 
 template <int RND, int EPI, int NM>
-cudaError_t gelu_launch_nm(const GeluArgs& A, cudaStream_t st) {
+cudaError_t gelu_launch_nm(GeluArgs A, long long t_begin, long long t_end, cudaStream_t st) {
   const size_t smem = sizeof(GeluSmem<NM>);
   cudaError_t e =
       cudaFuncSetAttribute(gelu_kernel<RND, EPI, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((A.p.N + 32 * NM - 1) / (32 * NM), (A.p.M + GL_BM - 1) / GL_BM);
-  gelu_kernel<RND, EPI, NM><<<grid, GL_T, smem, st>>>(A);
+  A.tile0 = t_begin;
+  A.ctiles = (A.p.N + 32 * NM - 1) / (32 * NM);
+  gelu_kernel<RND, EPI, NM><<<(unsigned)(t_end - t_begin), GL_T, smem, st>>>(A);
   return cudaGetLastError();
 }
 
-// Tile width: the narrower tiles when they cut the largest per-SM share of the
-// outputs (whole tiles a SM runs, times the tile's size) by an eighth or more.
+// Tile width. The 128-wide tiles run two CTAs per SM, the 64-wide ones three at
+// about 8 % less work per output. Whole problems take the narrower tiles when
+// they cut the largest per-SM share of the outputs (whole tiles a SM runs, times
+// the tile's size) by an eighth or more. Otherwise the 128-wide tiles fill whole
+// rounds of 2 x num_sms CTAs and, when a last partial round would be left, its
+// outputs go to a second launch of 64-wide tiles, which spreads them over three
+// CTAs per SM (the same rows and columns, so the two launches write disjoint
+// outputs).
 template <int RND, int EPI>
 cudaError_t gelu_launch_one(const GeluArgs& A, cudaStream_t st) {
   const long long rt = (A.p.M + GL_BM - 1) / GL_BM;
-  const long long t4 = rt * ((A.p.N + 127) / 128), t2 = rt * ((A.p.N + 63) / 64);
+  const long long c4 = (A.p.N + 127) / 128, c2 = (A.p.N + 63) / 64;
+  const long long t4 = rt * c4, t2 = rt * c2;
   const long long share4 = (t4 + A.num_sms - 1) / A.num_sms * 2, share2 = (t2 + A.num_sms - 1) / A.num_sms;
-  if (8 * share2 <= 7 * share4) return gelu_launch_nm<RND, EPI, 2>(A, st);
-  return gelu_launch_nm<RND, EPI, 4>(A, st);
+  if (8 * share2 <= 7 * share4) return gelu_launch_nm<RND, EPI, 2>(A, 0, t2, st);
+  const long long round4 = 2LL * A.num_sms, full = t4 / round4 * round4, rest = t4 - full;
+  if (full > 0 && rest > 0 && rest < round4 && c2 == 2 * c4) {
+    cudaError_t e = gelu_launch_nm<RND, EPI, 4>(A, 0, full, st);
+    if (e != cudaSuccess) return e;
+    return gelu_launch_nm<RND, EPI, 2>(A, 2 * full, t2, st);
+  }
+  return gelu_launch_nm<RND, EPI, 4>(A, 0, t4, st);
 }
 
 template <int EPI>

@@ -206,3 +206,13 @@ def test_gelu_gpt2xl_fc_sampled(rate):
     rows = np.sort(np.random.default_rng(56).choice(lw.M, size=12, replace=False))
     g, orc, nsel = run_case(lw, 4, e["tau"], rows=rows)
     assert g.count() == e["selected_at_tau"]
+
+
+def test_gelu_rows_on_both_sides_of_the_tile_split():
+    """800 tiles of 128 columns: two full rounds of 128-wide tiles, the rest as
+    64-wide tiles in a second launch. Rows from both, and from the row tile
+    that the split cuts (row tile 11: columns below and above 5376)."""
+    lw = S.LinearWorkload(1024, 6400, 64, seed=57)
+    rows = np.array([0, 703, 704, 705, 767, 768, 1000, 1023])
+    g, orc, nsel = run_case(lw, 4, 2.0, rows=rows)
+    assert nsel > 0
