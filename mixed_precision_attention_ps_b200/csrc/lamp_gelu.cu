@@ -21,6 +21,7 @@
 #include "lamp.h"
 #include "lamp_device.cuh"
 #include "lamp_kernels.h"
+#include "lamp_linear.cuh"
 
 namespace lamp {
 namespace {

@@ -20,6 +20,7 @@
 #include "lamp.h"
 #include "lamp_device.cuh"
 #include "lamp_kernels.h"
+#include "lamp_linear.cuh"
 
 namespace lamp {
 namespace {
