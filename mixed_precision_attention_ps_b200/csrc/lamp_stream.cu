@@ -426,7 +426,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
 // Pass 1 of the strict rows: every tile stored to the slab, and per row the
 // maximum, its first key and S_rest kept online across the tiles. A tile's
 // maximum and first key come from warp reductions and its sum of exp(y - tile
-// maximum) over the other keys from binary32 expf terms summed in double; the
+// maximum) over the other keys from binary32 exp terms (ex2.approx) summed in double; the
 // merge is exact in double: a larger tile maximum rescales the running sum by
 // exp(m_old - m_new) with the old maximum joining it as a term 1, a smaller or
 // equal one adds (tile sum + 1) exp(m_tile - m).
@@ -497,13 +497,17 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
         if (mt > -INFINITY) {  // warp-uniform
           const int at = t0 + __reduce_min_sync(0xFFFFFFFFu, lm == mt ? li : 0x7FFFFFFF);
           double sl = 0.0;
+          const float ml = mt * kLog2e;  // exp(y - mt) on the special-function unit, as in the selection
           for (int i4 = 0; i4 < nit; ++i4) {
             const int j0 = 128 * i4 + 4 * lane;
             const float4 v = lds4_or_ninf(row + j0, j0 < written);
             const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (t0 + j0 + e != at) sl += (double)expf(__fsub_rn(vv[e], mt));
+            for (int e = 0; e < 4; ++e) {
+              float ex;
+              asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(fmaf(vv[e], kLog2e, -ml)));
+              if (t0 + j0 + e != at) sl += (double)ex;
+            }
           }
           const double st = warp_sum_d(sl);
           if (mt > M[tt]) {

@@ -249,8 +249,17 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
             else if (e == 2) v.z = -INFINITY;
             else v.w = -INFINITY;
           }
-          sa[t] += (double)expf(__fsub_rn(v.x, m[t])) + (double)expf(__fsub_rn(v.y, m[t]));
-          sb[t] += (double)expf(__fsub_rn(v.z, m[t])) + (double)expf(__fsub_rn(v.w, m[t]));
+          // exp(y - m) as 2^(y log2 e - m log2 e) on the special-function unit
+          // (relative error about 2^-22, the selection pass's form): S_rest then
+          // carries a few 1e-7 relative error, inside the criterion's double band
+          const float ml = m[t] * kLog2e;
+          float e0, e1, e2, e3;
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(fmaf(v.x, kLog2e, -ml)));
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(fmaf(v.y, kLog2e, -ml)));
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e2) : "f"(fmaf(v.z, kLog2e, -ml)));
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e3) : "f"(fmaf(v.w, kLog2e, -ml)));
+          sa[t] += (double)e0 + (double)e1;
+          sb[t] += (double)e2 + (double)e3;
         }
       }
 #pragma unroll
