@@ -525,17 +525,32 @@ def cpu_baseline(w, Q, K, V, mu, tau, variant) -> dict:
 
 
 # ----------------------------------------------------------------------------------------
-# LAMP on an elementwise activation: GELU(scale * x W^T), the linear map in PS(mu)
+# LAMP on the operators after a PS(mu) linear map: GELU(scale * x W^T) (op "gelu")
+# and LayerNorm(scale * x W^T) (op "ln")
 # ----------------------------------------------------------------------------------------
-def gelu_metric(lw, mu, op="gelu") -> str:
+def linear_metric(lw, mu, op="gelu") -> str:
     name = "LayerNorm" if op == "ln" else "GELU"
     return f"LAMP {name}(x W^T) G-outputs/s at {lw.M}x{lw.N}x{lw.K} mu={mu}; % of roofline"
 
 
-GELU_UNIT = "G-outputs/s"
+LINEAR_UNIT = "G-outputs/s"
 
 
-def gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op="gelu") -> float:
+def linear_map_launches(M: int, N: int, num_sms: int) -> int:
+    """Kernel launches of the library's linear map for an M x N output (its tile-width
+    rule: 64-wide tiles for the whole problem, or 128-wide tiles in whole rounds of
+    2 x num_sms CTAs plus a second launch of 64-wide tiles for a last partial round)."""
+    rt = (M + 63) // 64
+    c4, c2 = (N + 127) // 128, (N + 63) // 64
+    t4, t2 = rt * c4, rt * c2
+    share4, share2 = (t4 + num_sms - 1) // num_sms * 2, (t2 + num_sms - 1) // num_sms
+    if 8 * share2 <= 7 * share4:
+        return 1
+    full = t4 // (2 * num_sms) * (2 * num_sms)
+    return 2 if (full > 0 and 0 < t4 - full < 2 * num_sms and c2 == 2 * c4) else 1
+
+
+def linear_oracle_pass(lw, x, W, mu, tau, rows, threads, op="gelu") -> float:
     import oracle
     t0 = time.perf_counter()
     if op == "ln":
@@ -545,7 +560,7 @@ def gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op="gelu") -> float:
     return time.perf_counter() - t0
 
 
-def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0, op="gelu") -> dict:
+def linear_cpu_baseline(lw, x, W, mu, tau, seconds=10.0, op="gelu") -> dict:
     """The activation oracle as it stands, on the host's cores, over a row sample
     repeated until about `seconds` of work have run."""
     threads = os.cpu_count() or 1
@@ -553,15 +568,15 @@ def gelu_cpu_baseline(lw, x, W, mu, tau, seconds=10.0, op="gelu") -> dict:
     rows = np.arange(0, lw.M, m, dtype=np.int64)
     t_all, n_out, passes = 0.0, 0, 0
     while t_all < seconds and passes < 20:
-        t_all += gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op)
+        t_all += linear_oracle_pass(lw, x, W, mu, tau, rows, threads, op)
         n_out += rows.size * lw.N
         passes += 1
-    return {"value": n_out / t_all / 1e9, "unit": GELU_UNIT, "cores": threads, "kind": "oracle",
+    return {"value": n_out / t_all / 1e9, "unit": LINEAR_UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{passes} pass(es) over {rows.size} of {lw.M} rows (every {m}th, {rows.size * lw.N} "
                       f"outputs each), {t_all:.1f} s"}
 
 
-def gelu_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream, op="gelu") -> dict:
+def linear_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream, op="gelu") -> dict:
     """Errors against the all-FP32 outputs (tau < 0) for no recompute, LAMP at tau and
     a random choice of the same per-row count, on a row sample (outside the timed region)."""
     import oracle
@@ -597,7 +612,7 @@ def gelu_accuracy(lamp, torch, lw, xd, Wd, mu, tau, stream, op="gelu") -> dict:
             f"{key}_reduction_random": err["ps_only"][key] / max(err["random_same_count"][key], 1e-300)}
 
 
-def run_gelu_reference(a, lw, mu, tau, cfg, op="gelu"):
+def run_linear_reference(a, lw, mu, tau, cfg, op="gelu"):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
@@ -606,21 +621,21 @@ def run_gelu_reference(a, lw, mu, tau, cfg, op="gelu"):
     m = max(1, lw.M // max(1, int(1.6e8 // (lw.N * lw.K))))
     rows = np.arange(0, lw.M, m, dtype=np.int64)
     for _ in range(a.warmup):
-        gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op)
-    times = [gelu_oracle_pass(lw, x, W, mu, tau, rows, threads, op) for _ in range(a.steps)]
+        linear_oracle_pass(lw, x, W, mu, tau, rows, threads, op)
+    times = [linear_oracle_pass(lw, x, W, mu, tau, rows, threads, op) for _ in range(a.steps)]
     ms = 1e3 * statistics.mean(times)
     value = rows.size * lw.N / (ms * 1e-3) / 1e9
     sample = f"{rows.size} of {lw.M} rows (every {m}th), {rows.size * lw.N} outputs per step"
-    line = {"metric": gelu_metric(lw, mu, op), "value": value, "unit": GELU_UNIT, "n_gpus": a.gpus, "steps": a.steps,
+    line = {"metric": linear_metric(lw, mu, op), "value": value, "unit": LINEAR_UNIT, "n_gpus": a.gpus, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg, "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": GELU_UNIT, "cores": threads, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": GELU_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": value, "unit": LINEAR_UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": LINEAR_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def run_gelu_ours(a, lw, mu, tau, cfg, op="gelu"):
+def run_linear_ours(a, lw, mu, tau, cfg, op="gelu"):
     import torch
     import torch.distributed as dist
 
@@ -750,31 +765,34 @@ def run_gelu_ours(a, lw, mu, tau, cfg, op="gelu"):
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s", "frac": achieved / peak,
                 "traffic": traffic_bytes(a.workload, 0, mu),
                 "kernel": ("one call: the linear-map kernel (gelu_kernel, store epilogue) + ln_rows_kernel"
-                           if op == "ln" else "gelu_kernel (one launch per call)"),
+                           if op == "ln" else "one call: gelu_kernel (128-wide tiles, then 64-wide tiles "
+                                              "for a last partial round)"),
                 "peak_basis": f"148 SMs x 128 lanes/clk x {f_max / 1e6:.0f} MHz (max SM clock); 4 K lane-ops "
                               "per output (K steps of 1 multiply-add + 3 integer ops of the rounding)"}
-        result = {"metric": gelu_metric(lw, mu, op), "value": value, "unit": GELU_UNIT, "n_gpus": world, "steps": a.steps,
+        result = {"metric": linear_metric(lw, mu, op), "value": value, "unit": LINEAR_UNIT, "n_gpus": world, "steps": a.steps,
                   "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                   "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg, "clocks": clk,
-                  "roofline": roof, "gpu_launches": (2 if op == "ln" else 1) * a.steps,
-                  "e2e": {"value": job_value(world, n_out, ms_e2e), "unit": GELU_UNIT,
+                  "roofline": roof,
+                  "gpu_launches": (linear_map_launches(lw.M, lw.N, props.multi_processor_count)
+                                   + (1 if op == "ln" else 0)) * a.steps,
+                  "e2e": {"value": job_value(world, n_out, ms_e2e), "unit": LINEAR_UNIT,
                           "h2d_bytes_per_step": x.nbytes + W.nbytes,
                           "d2h_bytes_per_step": out.numel() * 2 + mask.numel() * 4, "ms_per_step": ms_e2e,
                           "form": "pipelined: 2 buffer sets, H2D / compute / D2H streams"},
                   "ms_p10_p90": [float(np.percentile(times, 10)), float(np.percentile(times, 90))]}
         if not a.no_kl:
-            result["accuracy"] = gelu_accuracy(lamp, torch, lwr, xd, Wd, mu, tau, stream, op)
+            result["accuracy"] = linear_accuracy(lamp, torch, lwr, xd, Wd, mu, tau, stream, op)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         if not a.no_cpu_baseline and world == 1:
-            result["cpu_baseline"] = gelu_cpu_baseline(lwr, x, W, mu, tau, op=op)
+            result["cpu_baseline"] = linear_cpu_baseline(lwr, x, W, mu, tau, op=op)
         print(json.dumps(result), flush=True)
     return 0
 
 
-def main_gelu(a):
+def main_linear(a):
     lw = S.LINEAR_WORKLOADS[a.workload]
     op = "ln" if a.workload.startswith("ln_") else "gelu"
     _, drate = DEFAULTS[a.workload]
@@ -787,14 +805,14 @@ def main_gelu(a):
            "inputs": "bf16 N(0,1) x and W (SplitMix64 + Box-Muller), seed = rank",
            "l2": "flushed between steps (256 MB write)", "outputs_per_step_per_gpu": lw.outputs()}
     if a.impl == "reference":
-        return run_gelu_reference(a, lw, a.mu, tau, cfg, op)
-    return run_gelu_ours(a, lw, a.mu, tau, cfg, op)
+        return run_linear_reference(a, lw, a.mu, tau, cfg, op)
+    return run_linear_ours(a, lw, a.mu, tau, cfg, op)
 
 
 def main():
     a = parse()
     if a.workload in S.LINEAR_WORKLOADS:
-        return main_gelu(a)
+        return main_linear(a)
     w = S.WORKLOADS[a.workload]
     dv, drate = DEFAULTS[a.workload]
     variant = dv if a.variant is None else a.variant

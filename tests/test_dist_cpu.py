@@ -103,3 +103,13 @@ def test_operator_reference_arms_under_torchrun(workload):
     assert d["impl"] == "reference" and d["unit"] == "G-outputs/s" and d["value"] > 0
     assert d["config"]["workload"] == workload and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_linear_map_launch_count_follows_the_tile_rule():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.linear_map_launches(1024, 6400, 148) == 2   # 592 wide tiles, then 416 narrow ones
+    assert bench.linear_map_launches(1024, 1600, 148) == 1   # narrow tiles for the whole problem
+    assert bench.linear_map_launches(96, 300, 148) == 1
+    assert bench.linear_map_launches(1024, 6400 - 32, 148) == 1  # 100 -> 99 narrow columns: no split
