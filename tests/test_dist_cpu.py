@@ -112,4 +112,4 @@ def test_linear_map_launch_count_follows_the_tile_rule():
     assert bench.linear_map_launches(1024, 6400, 148) == 2   # 592 wide tiles, then 416 narrow ones
     assert bench.linear_map_launches(1024, 1600, 148) == 1   # narrow tiles for the whole problem
     assert bench.linear_map_launches(96, 300, 148) == 1
-    assert bench.linear_map_launches(1024, 6400 - 32, 148) == 1  # 100 -> 99 narrow columns: no split
+    assert bench.linear_map_launches(1024, 6304, 148) == 1  # 50 wide but 99 narrow column tiles: no split
