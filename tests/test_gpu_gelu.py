@@ -216,3 +216,12 @@ def test_gelu_rows_on_both_sides_of_the_tile_split():
     rows = np.array([0, 703, 704, 705, 767, 768, 1000, 1023])
     g, orc, nsel = run_case(lw, 4, 2.0, rows=rows)
     assert nsel > 0
+
+
+def test_gelu_width_whose_narrow_tiles_do_not_pair():
+    """N = 6304: 50 column tiles of 128 but 99 of 64, so no split launch; the
+    last wide tile is a quarter full. Sampled rows."""
+    lw = S.LinearWorkload(1024, 6304, 32, seed=58)
+    rows = np.array([0, 511, 767, 1023])
+    g, orc, nsel = run_case(lw, 4, 2.0, rows=rows)
+    assert nsel > 0
