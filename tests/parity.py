@@ -31,7 +31,7 @@ def to_device(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-class GpuRun:
+class GpuCall:
     """One call of lamp_attention_ex with every optional output switched on."""
 
     def __init__(self, w: S.Workload, Qd, Kd, Vd, *, mu, tau, variant, mask_in=None, scale=0.0,

@@ -25,7 +25,7 @@ def _device():
 
 def run_case(w, mu, tau, variant, rows=None, mask_in=None, scale=0.0, threads=8):
     Q, K, V = S.make_qkv(w)
-    g = P.GpuRun(w, P.to_device(Q), P.to_device(K), P.to_device(V), mu=mu, tau=tau, variant=variant,
+    g = P.GpuCall(w, P.to_device(Q), P.to_device(K), P.to_device(V), mu=mu, tau=tau, variant=variant,
                  mask_in=None if mask_in is None else torch.from_numpy(mask_in.view(np.int32)).cuda(),
                  scale=scale)
     if rows is None:
@@ -93,8 +93,8 @@ def test_tau_below_zero_and_mu23_are_fp32_attention():
     w = S.Workload(1, 2, 100, 100, 64, seed=4)
     Q, K, V = S.make_qkv(w)
     Qd, Kd, Vd = P.to_device(Q), P.to_device(K), P.to_device(V)
-    a = P.GpuRun(w, Qd, Kd, Vd, mu=4, tau=-1.0, variant=oracle.STRICT)
-    b = P.GpuRun(w, Qd, Kd, Vd, mu=23, tau=float("inf"), variant=oracle.STRICT)
+    a = P.GpuCall(w, Qd, Kd, Vd, mu=4, tau=-1.0, variant=oracle.STRICT)
+    b = P.GpuCall(w, Qd, Kd, Vd, mu=23, tau=float("inf"), variant=oracle.STRICT)
     rows = np.arange(w.B * w.H * w.n_q)
     ra, rb = a.rows(rows), b.rows(rows)
     assert np.array_equal(ra["mixed"].view(np.uint32), rb["mixed"].view(np.uint32))
@@ -142,7 +142,7 @@ def test_nonfinite_free_extreme_inputs_take_the_exact_path():
     Q2 = S.to_bf16_bits(Qf.astype(np.float64)).reshape(Q.shape)
     K2 = S.to_bf16_bits(Kf.astype(np.float64)).reshape(K.shape)
     for mu in (4, 10, 23):
-        g = P.GpuRun(w, P.to_device(Q2), P.to_device(K2), P.to_device(V), mu=mu, tau=0.05,
+        g = P.GpuCall(w, P.to_device(Q2), P.to_device(K2), P.to_device(V), mu=mu, tau=0.05,
                      variant=oracle.STRICT, scale=1.0)
         rows = np.arange(w.B * w.H * w.n_q)
         orc = oracle.attention_rows(Q2, K2, V, causal=False, scale=1.0, mu=mu, tau=0.05, rows=rows,

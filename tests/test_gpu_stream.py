@@ -79,8 +79,8 @@ def test_stream_tau_below_zero_and_mu23_agree():
     w = S.Workload(1, 2, 30, 1800, 64, causal=False, seed=13)
     Q, K, V = S.make_qkv(w)
     Qd, Kd, Vd = P.to_device(Q), P.to_device(K), P.to_device(V)
-    a = P.GpuRun(w, Qd, Kd, Vd, mu=4, tau=-1.0, variant=oracle.RELAXED)
-    b = P.GpuRun(w, Qd, Kd, Vd, mu=23, tau=float("inf"), variant=oracle.RELAXED)
+    a = P.GpuCall(w, Qd, Kd, Vd, mu=4, tau=-1.0, variant=oracle.RELAXED)
+    b = P.GpuCall(w, Qd, Kd, Vd, mu=23, tau=float("inf"), variant=oracle.RELAXED)
     rows = np.arange(w.B * w.H * w.n_q)
     ra, rb = a.rows(rows), b.rows(rows)
     assert np.array_equal(ra["mixed"].view(np.uint32), rb["mixed"].view(np.uint32))
