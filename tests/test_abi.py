@@ -171,3 +171,23 @@ def test_ln_argument_checks(lib, kw, code, msg):
 def test_ln_workspace_size(lib):
     assert lamp.lamp_ln_workspace_size(1024, 1600) == 1024 * 1600 * 4
     assert lamp.lamp_ln_workspace_size(0, 5) == 0
+
+
+def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
+    """A C program that includes only include/lamp.h links against liblamp.so and
+    gets the documented errors back without a GPU."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.dirname(_native.LIB_PATH)
+    exe = str(tmp_path / "abi_client")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c_abi", "abi_client.c"), "-L", pkg, "-llamp",
+                    f"-Wl,-rpath,{pkg}", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert "abi client ok" in r.stdout
