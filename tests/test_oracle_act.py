@@ -185,3 +185,19 @@ def test_amplification_falls_with_the_rate_and_adaptive_beats_random():
     assert errs[0]["max_amp"] > errs[1]["max_amp"] > errs[2]["max_amp"]
     # recomputed components carry no error, and the selections are nested
     assert e_base["l1_rel"] > errs[0]["l1_rel"] > errs[1]["l1_rel"] > errs[2]["l1_rel"]
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.floats(min_value=-8, max_value=8, allow_nan=False))
+def test_kappa_matches_autograd_on_random_inputs(y):
+    if abs(y) < 1e-6:
+        return
+    k = oracle.gelu_kappa(y)
+    ref = kappa_autograd(np.array([y]))[0]
+    f = float(torch_gelu(np.array([y]))[0])
+    if abs(f) < 1e-12:  # double GELU underflows in PyTorch's form; the decimal pin covers it
+        return
+    assert k == pytest.approx(ref, rel=1e-9, abs=1e-10)

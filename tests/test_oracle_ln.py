@@ -124,3 +124,25 @@ def test_error_falls_with_the_rate_and_greedy_beats_random():
         e_rnd = oracle.ln_errors(rnd.out, full.out)
         assert e["mean_l2"] < last and e["mean_l2"] < e_rnd["mean_l2"]
         last = e["mean_l2"]
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.lists(st.floats(min_value=-6, max_value=6, allow_nan=False, width=32), min_size=2, max_size=9),
+       st.floats(min_value=0.0, max_value=4.0))
+def test_greedy_minimality_on_random_rows(vals, tau):
+    """For any small row and tau: the greedy's count is the brute-force minimum,
+    its set is feasible, and it is the top-k by magnitude (ties by index)."""
+    y = np.array(vals, dtype=np.float32)
+    t = oracle.ln_thresholds(y)
+    if np.any(np.abs(t - tau) <= 1e-12 * max(1.0, tau)):
+        return  # a threshold value itself: only rounding decides there
+    sel, k, rest = oracle.ln_select(y, tau)
+    assert k == brute_force_min_count(y, tau)
+    order = sorted(range(y.size), key=lambda j: (-abs(float(y[j])), j))
+    assert set(np.nonzero(sel)[0]) == set(order[:k])
+    _, sigma = oracle.layernorm(y.astype(np.float64))
+    if tau >= 0 and k < y.size:
+        assert np.sqrt(rest) <= tau * sigma * (1 + 1e-12)
