@@ -15,8 +15,13 @@
  *   - section "Experimental results": PS(mu) (mu mantissa bits), the relaxed
  *     relative-threshold variant that needs no normalising constant and so fits
  *     a one-pass softmax, and the random-selection control.
+ * The same look-ahead scheme serves the two other operators of "Theoretical
+ * basis", item 3, each after a PS(mu) linear map y = scale * x W^T:
+ * lamp_linear_gelu (an activation: a diagonal Jacobian, a per-output condition
+ * number) and lamp_linear_layernorm (greedy recompute by sorted magnitude);
+ * their conventions are given with them below.
  *
- * Conventions for every entry point:
+ * Conventions for every entry point (the operator calls state their own shapes):
  *   - All tensor pointers are DEVICE pointers owned by the caller. Q is
  *     [B, H, n_q, d], K and V are [B, H, n_k, d], out is [B, H, n_q, d]; all
  *     contiguous row-major bfloat16 given as raw 16-bit patterns, 16-byte aligned.
