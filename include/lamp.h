@@ -232,7 +232,7 @@ LAMP_API size_t lamp_args_size(void);
  *   mixed_out   nullable fp32 [M, N]: y after the recompute.
  *   n_selected_out  nullable device word: set to the number of recomputed outputs.
  * Every pointer is caller-owned device memory; the call is asynchronous on
- * stream, allocates nothing, and launches one kernel (plus a memset of
+ * stream, allocates nothing, and launches one or two kernels (plus a memset of
  * n_selected_out). Returns LAMP_OK, LAMP_ERR_ARG or LAMP_ERR_UNSUPPORTED
  * (K % 8 != 0, misaligned pointers, M too large) before launching anything, or
  * LAMP_ERR_CUDA when the launch fails.
