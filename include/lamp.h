@@ -279,7 +279,7 @@ LAMP_API size_t lamp_gelu_args_size(void);
  *   workspace   device scratch for y_hat of lamp_ln_workspace_size(M, N) bytes,
  *               or NULL: then ps_out holds y_hat when given, else the library's
  *               per-device pool (as lamp_attention_ex) provides it.
- * Asynchronous on stream; two kernels (the linear map, then one warp per row).
+ * Asynchronous on stream; the linear map (one or two kernels), then one warp per row.
  * Returns LAMP_OK, LAMP_ERR_ARG / LAMP_ERR_UNSUPPORTED / LAMP_ERR_WORKSPACE
  * before launching anything, or LAMP_ERR_CUDA.
  */
