@@ -113,3 +113,16 @@ def test_linear_map_launch_count_follows_the_tile_rule():
     assert bench.linear_map_launches(1024, 1600, 148) == 1   # narrow tiles for the whole problem
     assert bench.linear_map_launches(96, 300, 148) == 1
     assert bench.linear_map_launches(1024, 6304, 148) == 1  # 50 wide but 99 narrow column tiles: no split
+
+
+def test_every_bench_default_has_a_calibrated_tau():
+    """bench.py's default (workload, variant, rate) pairs all resolve in tau.json,
+    so no GPU run stops on a missing threshold."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synthetic as S
+
+    for name, (variant, rate) in bench.DEFAULTS.items():
+        assert name in S.WORKLOADS or name in S.LINEAR_WORKLOADS
+        tau, r = bench.lookup_tau(name, variant, 4, rate)
+        assert tau == tau and (rate is None or r == rate)
