@@ -84,22 +84,22 @@ enum lamp_status {
   LAMP_ERR_ARG = -1,          /* null required pointer, mu outside [1,23], tau NaN,
                                  unknown variant, a dimension <= 0, scale <= 0 or NaN */
   LAMP_ERR_UNSUPPORTED = -2,  /* d not in {64, 128}; pointer not 16-byte aligned;
-                                 a problem only the row kernels can serve (see
-                                 LAMP_MAX_STRICT_NK) with n_k > LAMP_MAX_STRICT_NK;
-                                 B * H > 65535 */
+                                 a strict problem whose score slab would pass
+                                 LAMP_MAX_SCORE_SLAB_BYTES; B * H > 65535 */
   LAMP_ERR_WORKSPACE = -3,    /* workspace given but smaller than lamp_workspace_size() */
   LAMP_ERR_CUDA = -4,         /* a CUDA call failed (allocation, launch); see lamp_last_error() */
   LAMP_ERR_TIMEOUT = -5,      /* written to status_out by a kernel whose bounded wait gave up */
   LAMP_ERR_CHECK = -6         /* reserved: a device-side check failed (reported via status_out) */
 };
 
-/* Largest n_k of the row kernels. Relaxed and given-mask rows of any length
- * stream through 512-key tiles, decode rows (n_q <= 4) split their keys, and
- * strict rows longer than 1024 keys take two streamed passes over a score slab
- * of B*H*n_q*ceil(n_k/512)*512*4 bytes in the workspace. Only a strict problem
- * whose slab would pass 8 GiB falls to the row kernels, which need
- * n_k <= LAMP_MAX_STRICT_NK (else LAMP_ERR_UNSUPPORTED). */
-#define LAMP_MAX_STRICT_NK 65536
+/* Largest score slab of a strict call. Whole rows of up to 1024 keys (d = 64;
+ * 896 at d = 128) stay in shared memory, relaxed and given-mask rows of any
+ * length stream through 512-key tiles, and decode rows (n_q <= 4) split their
+ * keys. Strict rows longer than that take two streamed passes over a score slab
+ * of B*H*n_q*ceil(n_k/512)*512*4 bytes in the workspace; a problem whose slab
+ * would be larger than this is LAMP_ERR_UNSUPPORTED (lamp_workspace_size
+ * returns 0 for it). */
+#define LAMP_MAX_SCORE_SLAB_BYTES (64ull << 30)
 
 typedef struct {
   int B, H, n_q, n_k, d;

@@ -23,7 +23,7 @@ LAMP_ERR_WORKSPACE = -3
 LAMP_ERR_CUDA = -4
 LAMP_ERR_TIMEOUT = -5
 LAMP_ERR_CHECK = -6
-LAMP_MAX_STRICT_NK = 65536
+LAMP_MAX_SCORE_SLAB_BYTES = 64 << 30
 LAMP_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 STATUS_NAMES = {

@@ -147,7 +147,8 @@ lamp::Problem make_problem(const lamp_args* a) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// The launch sequence of one call: exponent statistics, then the row kernel.
+// The launch sequence of one call: exponent statistics, then the whole-row or
+// the streamed kernel (or the two decode kernels on their own).
 cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char* base, const DeviceInfo& info,
                         cudaStream_t st) {
   // the decode kernels fold their own exponent statistics and reset the count
@@ -155,9 +156,7 @@ cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char*
   cudaError_t e = lamp::launch_prep(p, ws, base, st);
   if (e != cudaSuccess) return e;
   if (ws.use_ws) return lamp::launch_ws(p, ws, base, info.num_sms, st);
-  if (ws.use_stream) return lamp::launch_stream(p, ws, base, info.num_sms, st);
-  if (ws.rows_bm) return lamp::launch_rows(p, ws, base, info.num_sms, st);
-  return lamp::launch_strict(p, ws, base, info.num_sms, info.smem_optin, st);
+  return lamp::launch_stream(p, ws, base, info.num_sms, st);
 }
 
 // Scratch of lamp_attention_noalloc: one fixed array in the device memory of
@@ -197,10 +196,6 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
   w.counters = 0;
   w.stats = 256;
   size_t off = align256(w.stats + (size_t)BH * nchunk * 16);
-  w.nkp = ((p.n_k + 127) / 128) * 128 + 4;
-  w.spill = off;
-  w.spill_rows = 0;
-  w.grid = 0;
   // decode shapes (a few query rows per head, long rows): split over the keys
   if (p.n_q <= kDecodeMaxQ && p.n_k >= kDecodeMinKeys) {
     w.use_decode = 1;
@@ -224,11 +219,11 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
   w.use_stream = (!w.use_ws && stream_smem_bytes(p.d) + kStaticSmemReserve <= smem_optin) ? 1 : 0;
   if (w.use_stream && p.variant == LAMP_STRICT) {
     // strict rows take two passes over a score slab in HBM (the strict test needs
-    // the whole row's statistics before it selects anything); past the slab cap
-    // the row kernels serve them
+    // the whole row's statistics before it selects anything)
     const size_t slab = (size_t)BH * p.n_q * stream_slab_ld(p.n_k) * 4;
+    w.st_slab_bytes = slab;
     if (slab > kStrictSlabCap) {
-      w.use_stream = 0;
+      w.slab_too_large = 1;
     } else {
       w.st_slab = off;
       off = align256(off + slab);
@@ -236,30 +231,24 @@ Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin) {
       off = align256(off + (size_t)BH * p.n_q * 16);
     }
   }
-  w.rows_bm = (w.use_ws || w.use_stream) ? 0 : rows_pick_bm(p.d, p.n_k, smem_optin);
-  if (!w.use_ws && !w.use_stream && !w.rows_bm && strict_smem_bytes(p.d, w.nkp, true) + kStaticSmemReserve > smem_optin) {
-    const long long n_items = (long long)((p.n_q + kStrictBM - 1) / kStrictBM) * BH;
-    w.grid = (int)(n_items < num_sms ? n_items : num_sms);
-    w.spill_rows = 1;
-    off = align256(off + (size_t)w.grid * kStrictBM * w.nkp * 4);
-  }
   w.total = off;
   return w;
 }
 
 }  // namespace lamp
 
-// The plan's kernels must be able to serve the problem: the row kernels (strict
-// problems whose score slab would pass its cap) take rows of at most
-// LAMP_MAX_STRICT_NK keys and need their shared-memory rows or row slab.
+// The plan's kernels must be able to serve the problem: a strict problem's
+// two-pass score slab must stay within LAMP_MAX_SCORE_SLAB_BYTES, and the
+// kernel's shared memory must fit the device.
 int check_plan(const lamp::Problem& p, const lamp::Workspace& ws, const DeviceInfo& info) {
-  if (ws.use_decode || ws.use_ws || ws.use_stream) return LAMP_OK;
-  if (p.n_k > LAMP_MAX_STRICT_NK)
+  (void)info;
+  if (ws.slab_too_large)
     return fail(LAMP_ERR_UNSUPPORTED,
-                "rows of %d keys: past the streamed kernel's score-slab cap the row kernels take n_k <= %d",
-                p.n_k, LAMP_MAX_STRICT_NK);
-  if (!ws.rows_bm && lamp::strict_smem_bytes(p.d, ws.nkp, !ws.spill_rows) + lamp::kStaticSmemReserve > info.smem_optin)
-    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small");
+                "strict rows of %d keys need a two-pass score slab of %zu bytes, more than "
+                "LAMP_MAX_SCORE_SLAB_BYTES (%llu)",
+                p.n_k, ws.st_slab_bytes, (unsigned long long)LAMP_MAX_SCORE_SLAB_BYTES);
+  if (!ws.use_decode && !ws.use_ws && !ws.use_stream)
+    return fail(LAMP_ERR_UNSUPPORTED, "device shared memory too small for the attention kernels");
   return LAMP_OK;
 }
 
@@ -280,7 +269,9 @@ size_t lamp_workspace_size(const lamp_dims* dims, int variant) {
   lamp::Problem p{};
   p.B = dims->B; p.H = dims->H; p.n_q = dims->n_q; p.n_k = dims->n_k; p.d = dims->d;
   p.variant = variant;
-  return lamp::plan_workspace(p, info.num_sms, info.smem_optin).total;
+  const lamp::Workspace w = lamp::plan_workspace(p, info.num_sms, info.smem_optin);
+  if (w.slab_too_large || (!w.use_decode && !w.use_ws && !w.use_stream)) return 0;
+  return w.total;
 }
 
 int lamp_attention_ex(const lamp_args* a) {

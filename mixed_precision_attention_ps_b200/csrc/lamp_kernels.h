@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "lamp.h"
+
 namespace lamp {
 
 // Rounding class of mu, fixed per launch:
@@ -41,17 +43,14 @@ struct Problem {
 struct Workspace {
   size_t counters;     // uint32 work counters [4]
   size_t stats;        // int32 [B*H][nchunk][4]
-  size_t spill;        // fp32 score rows [grid][BM][nkp] (strict path, when rows do not fit on chip)
   size_t total;
   int nchunk;
-  int spill_rows;      // 0 when the score rows stay in shared memory
-  int grid;            // persistent grid size used for the spill slabs
-  int nkp;             // padded row length (floats) of the global-slab kernel
-  int rows_bm;         // rows per item of the on-chip row kernel; 0 = global-slab kernel
-  int use_ws;          // 1: warp-specialised kernel (two 16-row buffers fit on chip)
-  int use_stream;      // 1: streamed one-pass kernel (relaxed / given mask, rows too long for use_ws)
+  int use_ws;          // 1: warp-specialised whole-row kernel (two 16-row buffers fit on chip)
+  int use_stream;      // 1: streamed kernel (rows too long for use_ws; strict rows in two passes)
   int use_decode;      // 1: split-key decode kernels (few query rows, long rows)
+  int slab_too_large;  // 1: strict rows whose two-pass score slab would pass kStrictSlabCap
   size_t st_slab;      // strict rows on the streamed kernel: low-precision score slab [B*H][n_q][ld] f32
+  size_t st_slab_bytes;
   size_t st_rows;      // ... and per-row statistics (maximum, first argmax, S_rest), 16 bytes each
   int dec_chunks;      // decode: 512-key chunks per row
   size_t dec_scores;   // decode: fp32 low-precision scores [B*H][n_q][dec_chunks * 512]
@@ -61,20 +60,12 @@ struct Workspace {
   size_t dec_done;     // decode: per row, chunks whose partials are written (the last one combines)
 };
 
-// Strict / given-mask configuration: rows per work item and threads.
-constexpr int kStrictBM = 32;
-constexpr int kStrictThreads = 256;
-constexpr int kRowsThreads = 256;
-constexpr int kWsThreads = 512;
+constexpr int kWsThreads = 512;  // 8 producer warps, 8 consumer warps
 // Bytes of the opt-in shared memory left for the kernels' static __shared__ data.
 constexpr size_t kStaticSmemReserve = 256;
 
 Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin);
 cudaError_t launch_prep(const Problem& p, const Workspace& ws, char* base, cudaStream_t st);
-cudaError_t launch_strict(const Problem& p, const Workspace& ws, char* base, int num_sms,
-                          size_t smem_optin, cudaStream_t st);
-cudaError_t launch_rows(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
-int rows_pick_bm(int d, int n_k, size_t smem_optin);
 cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
 bool ws_fits(int d, int n_k, size_t smem_optin);
 cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
@@ -82,14 +73,10 @@ cudaError_t launch_decode(const Problem& p, const Workspace& ws, char* base, cud
 constexpr int kDecodeMaxQ = 4;       // query rows per (b, h) the decode kernels take
 constexpr int kDecodeMinKeys = 512;  // shortest rows routed to them
 constexpr int kDecodeChunk = 512;    // keys per chunk (one CTA)
-constexpr size_t kStrictSlabCap = (size_t)8 << 30;  // largest score slab of the two-pass strict rows
+constexpr size_t kStrictSlabCap = (size_t)LAMP_MAX_SCORE_SLAB_BYTES;  // largest two-pass strict score slab
 size_t stream_smem_bytes(int d);
 size_t stream_slab_ld(int n_k);  // slab row stride: keys rounded up to whole 512-key tiles
-int rows_nkp(int bm, int n_k);
-size_t rows_smem_bytes(int d, int bm, int n_k);
 cudaError_t launch_ps_round(const float* x, float* y, size_t n, int mu, int path, cudaStream_t st);
-
-size_t strict_smem_bytes(int d, int nkp, bool rows_on_chip);
 
 // LAMP GELU(scale * x W^T): x [M, K], W [N, K] bf16, out [M, N].
 struct GeluProblem {

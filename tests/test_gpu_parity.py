@@ -58,12 +58,12 @@ def test_single_head_128_strict_mu4():
     (1, 2, 70, 257, 64, False),    # non-causal, n_k one past a tile boundary
     (1, 1, 64, 64, 128, True),     # d = 128
     (1, 2, 161, 129, 128, False),  # d = 128, ragged
-    (1, 1, 40, 1500, 64, False),   # 16 rows per work item
-    (1, 1, 33, 1100, 128, True),   # d = 128, 32 rows per work item near the shared-memory limit
-    (1, 1, 20, 3000, 64, False),   # 8 rows per work item
-    (1, 2, 19, 3000, 128, True),   # d = 128, 8 rows per work item, causal with n_k > n_q
-    (1, 1, 24, 5000, 64, False),   # rows beyond shared memory: global row slab
-    (1, 1, 9, 4700, 128, True),    # d = 128 global row slab
+    (1, 1, 40, 1500, 64, False),   # streamed: three 512-key tiles, the last one ragged
+    (1, 1, 33, 1100, 128, True),   # d = 128 streamed, just past the whole-row limit
+    (1, 1, 20, 3000, 64, False),   # streamed: six tiles
+    (1, 2, 19, 3000, 128, True),   # d = 128 streamed, causal with n_k > n_q
+    (1, 1, 24, 5000, 64, False),   # streamed: ten tiles
+    (1, 1, 9, 4700, 128, True),    # d = 128 streamed, nine tiles plus a ragged one
 ])
 @pytest.mark.parametrize("variant", [oracle.STRICT, oracle.RELAXED])
 def test_shapes(B, H, n_q, n_k, d, causal, variant):

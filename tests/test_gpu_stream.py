@@ -110,9 +110,9 @@ def test_outlier_4x25x4096_relaxed_sampled():
     (20, oracle.GIVEN_MASK),  # one streamed pass with a caller-given mask
     (3, oracle.STRICT),       # decode rows: the keys split over chunks
 ])
-def test_rows_longer_than_the_row_kernel_limit(n_q, variant):
-    """Rows past LAMP_MAX_STRICT_NK keys: only the row kernels are limited."""
-    n_k = lamp.LAMP_MAX_STRICT_NK + 4501
+def test_rows_of_seventy_thousand_keys(n_q, variant):
+    """Rows far longer than shared memory (70037 keys) on every path that takes them."""
+    n_k = 70037
     w = S.Workload(1, 1, n_q, n_k, 64, causal=True, seed=16 + n_q)
     mask = None
     if variant == oracle.GIVEN_MASK:
@@ -123,14 +123,18 @@ def test_rows_longer_than_the_row_kernel_limit(n_q, variant):
     assert g.count() == int(orc.nsel.sum()) > 0
 
 
-def test_row_kernel_limit_is_reported_before_any_launch():
-    """A strict problem whose score slab would pass 8 GiB falls to the row
-    kernels, which take at most LAMP_MAX_STRICT_NK keys: the call fails with
-    LAMP_ERR_UNSUPPORTED at planning time (the fake pointers are never used)."""
+def test_score_slab_limit_is_reported_before_any_launch():
+    """A strict problem whose two-pass score slab (B*H*n_q*ceil(n_k/512)*512*4
+    bytes) would pass LAMP_MAX_SCORE_SLAB_BYTES fails with LAMP_ERR_UNSUPPORTED
+    at planning time (the fake pointers are never used), and its workspace size
+    reads 0; the relaxed variant streams the same rows in one pass."""
     fake = 1 << 20
-    n_k = lamp.LAMP_MAX_STRICT_NK + 4464
-    rc = lamp.lamp_attention_ex(dims=(1, 1, 32768, n_k, 64), Q=fake, K=fake, V=fake, out=fake, mu=4,
-                                tau=0.05, variant=lamp.LAMP_STRICT, causal=1, check=False)
-    assert rc == lamp.LAMP_ERR_UNSUPPORTED and "row kernels" in lamp.lamp_last_error()
-    # the relaxed variant streams the same rows
-    assert lamp.lamp_workspace_size((1, 1, 32768, n_k, 64), lamp.LAMP_RELAXED) > 0
+    dims = (1, 32, 16384, 65536, 64)  # 137 GB of slab
+    assert 32 * 16384 * 65536 * 4 > lamp.LAMP_MAX_SCORE_SLAB_BYTES
+    rc = lamp.lamp_attention_ex(dims=dims, Q=fake, K=fake, V=fake, out=fake, mu=4, tau=0.05,
+                                variant=lamp.LAMP_STRICT, causal=1, check=False)
+    assert rc == lamp.LAMP_ERR_UNSUPPORTED and "LAMP_MAX_SCORE_SLAB_BYTES" in lamp.lamp_last_error()
+    assert lamp.lamp_workspace_size(dims, lamp.LAMP_STRICT) == 0
+    assert lamp.lamp_workspace_size(dims, lamp.LAMP_RELAXED) > 0
+    # the 16K-token long-context shape (34 GB of slab) is within the limit
+    assert lamp.lamp_workspace_size((1, 32, 16384, 16384, 128), lamp.LAMP_STRICT) > 32 * 16384 * 16384 * 4

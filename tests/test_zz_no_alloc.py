@@ -88,8 +88,8 @@ def test_refuses_a_workspace_and_oversized_problems():
     rc = lamp.lamp_attention_noalloc(dims=(1, 1, 16, 64, 64), Q=Qd, K=Kd, V=Vd, out=o["out"], mu=4, tau=0.1,
                                      workspace=ws, workspace_bytes=ws.numel(), check=False)
     assert rc == lamp.LAMP_ERR_ARG and "workspace" in lamp.lamp_last_error()
-    # strict rows of 6000 keys in 16 heads need global row slabs (one per resident
-    # block of 32 rows) far larger than the fixed scratch
+    # strict rows of 6000 keys in 16 heads take two streamed passes over a score
+    # slab of 16 * 32 * 6144 * 4 bytes (12.6 MB), more than the fixed scratch
     big = S.Workload(1, 16, 32, 6000, 64, causal=False, seed=25)
     dims = (big.B, big.H, big.n_q, big.n_k, big.d)
     Qb, Kb, Vb = (P.to_device(t) for t in S.make_qkv(big))
