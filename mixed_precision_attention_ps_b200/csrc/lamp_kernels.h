@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "lamp.h"
@@ -60,11 +61,31 @@ struct Workspace {
   size_t dec_done;     // decode: per row, chunks whose partials are written (the last one combines)
 };
 
-constexpr int kWsThreads = 512;  // 8 producer warps, 8 consumer warps
+// Warp-specialised kernels: 8 producer warps, 8 consumer warps and a warpgroup
+// whose first warp drives the tensor core (MMA and TMA issue), 5 warpgroups.
+constexpr int kWsThreads = 640;
+// Registers per thread after setmaxnreg, per warpgroup role. The block launches
+// with kWsLaunchRegs (65536 / 640 rounded down to a multiple of 8); the split
+// must not need more than that pool: 256 P + 256 C + 128 M <= 640 * 96.
+constexpr int kWsLaunchRegs = 96;
+constexpr int kWsProdRegs = 112, kWsConsRegs = 96, kWsMmaRegs = 64;
+static_assert(256 * kWsProdRegs + 256 * kWsConsRegs + 128 * kWsMmaRegs <= kWsThreads * kWsLaunchRegs,
+              "register split above the launch pool");
+// setmaxnreg.inc may only raise a warp's count and .dec only lower it (a lower
+// .inc target is an illegal instruction); every budget is a multiple of 8 in [24, 256].
+static_assert(kWsProdRegs >= kWsLaunchRegs && kWsConsRegs >= kWsLaunchRegs && kWsMmaRegs <= kWsLaunchRegs,
+              "setmaxnreg.inc below, or .dec above, the launch count");
+static_assert(kWsProdRegs % 8 == 0 && kWsConsRegs % 8 == 0 && kWsMmaRegs % 8 == 0 && kWsMmaRegs >= 24 &&
+                  kWsProdRegs <= 256 && kWsConsRegs <= 256,
+              "setmaxnreg counts are multiples of 8 in [24, 256]");
 // Bytes of the opt-in shared memory left for the kernels' static __shared__ data.
 constexpr size_t kStaticSmemReserve = 256;
 
 Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin);
+// Tensor map of a [bh][n][d] bf16 tensor (row-major, this GPU's memory) for TMA
+// boxes of box_x dimensions x box_y rows of one (b, h); rows past n read as zero.
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n, int bh, int box_x, int box_y,
+                           bool swizzle128);
 cudaError_t launch_prep(const Problem& p, const Workspace& ws, char* base, cudaStream_t st);
 cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
 bool ws_fits(int d, int n_k, size_t smem_optin);

@@ -1,7 +1,8 @@
-// LAMP attention, streamed one-pass kernel for the relaxed and given-mask
-// variants at any row length (the 16K-token shape): scores are produced and
-// consumed in tiles of 512 keys with an online softmax, so no complete row is
-// ever stored.
+// LAMP attention, streamed kernel for rows longer than the whole-row kernel
+// takes: the relaxed and given-mask variants in one pass at any row length (the
+// 16K-token shape), strict rows in two passes over an HBM score slab. Scores are
+// produced and consumed in tiles of 512 keys with an online softmax, so no
+// complete row is ever held on chip.
 //
 // Method ("LAMP: Look-Ahead Mixed-Precision Inference of Large Language Models",
 // technical summary, gist.science paper 2601.21623), section "Experimental
@@ -12,16 +13,27 @@
 // "Implementation strategy", steps 1-3: low-precision baseline, selection from
 // it, FP32 recompute of the selection before the softmax.
 //
-// Same organisation as the whole-row warp-specialised kernel: one persistent CTA
-// of 512 threads per SM, items (b, h, 16 query rows) in a snake order, producer
-// warps 0-7 fill tile buffers (64-key units dealt round-robin, PS(mu) steps as
-// packed binary32 pairs), consumer warps 8-15 take each tile: the relaxed
-// criterion (double re-evaluation near tau), mask words, warp-compacted FP32
-// recompute from K in global memory, then the online softmax (running maximum m
-// and normaliser l per row; the per-warp partial outputs are rescaled by
-// exp(m_old - m_new) before each tile's P.V on tensor cores). After an item's
-// last tile the partial outputs are added in a fixed order and divided by l.
-// Hand-offs per tile use mbarriers (full[b], empty[b]); every wait is bounded.
+// Same organisation as the whole-row kernel (lamp_ws.cu): one persistent CTA of
+// 640 threads per SM, items (b, h, 16 query rows) in a snake order, two tile
+// buffers in the block layout of lamp_ws_common.cuh.
+//   producers (warps 0-7): 64-key units dealt round-robin, PS(mu) steps as packed
+//     binary32 pairs; each warp's K slices arrive by TMA (bf16, 64 keys x 8
+//     dimensions) in a ring of three stages and are widened on the way to the
+//     binary32 slice buffer.
+//   consumers (warps 8-15): per tile the criterion (double re-evaluation near
+//     tau), mask words, warp-compacted FP32 recompute, then the online softmax
+//     (running maximum m and normaliser l per row, rescale factor
+//     alpha = exp(m_old - m_new)) with the numerators written in place as the
+//     bf16 hi/lo operand of P.V.
+//   tensor-core warpgroup (warps 16-19): one thread streams V tiles of 64 keys by
+//     TMA (128-byte swizzle) into a ring that runs ahead across tiles and items,
+//     and issues 4 tcgen05.mma per V tile into one of two TMEM accumulators; the
+//     four warps then fold each tile into a register accumulator,
+//     O = alpha O + P.V (a thread holds one head dimension of the item's 16
+//     rows), and after an item's last tile store O / l.
+// Every wait is bounded; a wait that gives up records LAMP_ERR_TIMEOUT in the
+// caller's status word (when given) and ends the kernel after the copies and
+// tensor-core work in flight have drained and the tensor memory is released.
 #include <cfloat>
 
 #include "lamp_ws_common.cuh"
@@ -29,34 +41,54 @@
 namespace lamp {
 namespace {
 
-constexpr int ST_T = 512;   // keys per streamed tile
-constexpr int ST_TS = ST_T + 4;  // tile row stride (floats): 16-byte steps across banks
+constexpr int ST_T = 512;  // keys per streamed tile
 
+template <int D>
+__host__ __device__ constexpr int st_vslots() { return D == 64 ? 8 : 5; }  // V tiles in the ring
+template <int D>
+__host__ __device__ constexpr int st_vtile_bytes() { return WS_VKEYS * D * 2; }
 
-struct StSmem {
-  int bars;   // mbarriers: full[2], empty[2]
-  int q;      // Q [2][D][16] f32, by item parity
+// mbarrier indices
+constexpr int SB_FULL = 0, SB_PREADY = 2, SB_EMPTY = 4, SB_TFREE = 6, SB_VFULL = 8;
+template <int D>
+__host__ __device__ constexpr int sb_vempty() { return SB_VFULL + st_vslots<D>(); }
+template <int D>
+__host__ __device__ constexpr int sb_drain() { return SB_VFULL + 2 * st_vslots<D>(); }
+template <int D>
+__host__ __device__ constexpr int sb_kring() { return sb_drain<D>() + 1; }  // [8 warps][KRING]
+template <int D>
+__host__ __device__ constexpr int sb_count() { return sb_kring<D>() + WS_NP * KRING; }
+constexpr int BAR_PROD = 2;  // named barrier of the producer group
+constexpr int BAR_EPI = 3;   // named barrier of the tensor-core warpgroup (output epilogue)
+
+struct StSmem {  // byte offsets from a 1024-byte aligned base
+  int tiles;  // score tiles [2][sw_bytes(512)] (block layout)
+  int v;      // V ring [S][D / 64][64 keys][64 dims] bf16 (128-byte swizzle)
+  int kring;  // producer K stages [8 warps][KRING][64 keys][8 dims] bf16
   int ks;     // producer K slices [8 warps][2][8][64] f32
-  int v;      // consumer V rings [8 warps][WR][8][72] bf16, later the partial outputs [KQ][16][D] f32
+  int q;      // Q [2][D][16] f32, by item parity
   int list;   // consumer mask-word buffers [8][2][32] uint32
-  int rstat;  // per row: m, l, alpha, spare [16][4] f32
-  int tiles;  // score tiles [2][16][ST_TS] f32
+  int rstat;  // per tile parity and row: m, l, alpha, spare [2][16][4] f32
+  int otile;  // output tile of an item [16][D] bf16 (epilogue)
+  int bars;   // mbarriers
+  int tmem;   // TMEM base address
   int total;
 };
 
 template <int D>
 __host__ __device__ inline StSmem st_plan() {
   StSmem s{};
-  s.bars = 0;
-  s.q = 64;
-  s.ks = s.q + 2 * ws_qfloats<D>() * 4;
-  s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
-  const int vb = WS_NC * ws_vring<D>() * 8 * WS_VSW * 2;  // per-warp V rings
-  const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;
-  s.list = s.v + (vb > ob ? vb : ob);
+  s.tiles = 0;
+  s.v = 2 * sw_bytes(ST_T);
+  s.kring = s.v + st_vslots<D>() * st_vtile_bytes<D>();
+  s.ks = s.kring + WS_NP * KRING * WS_UNIT * WS_DS * 2;
+  s.q = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
+  s.list = s.q + 2 * ws_qfloats<D>() * 4;
   s.rstat = s.list + WS_NC * 2 * SEL_WMAX * 4;
-  s.tiles = s.rstat + WS_BM * 4 * 4;
-  s.total = s.tiles + 2 * WS_BM * ST_TS * 4;
+  s.otile = s.rstat + 2 * WS_BM * 4 * 4;
+  s.bars = s.otile + WS_BM * D * 2;
+  s.tmem = s.bars + sb_count<D>() * 8;
+  s.total = s.tmem + 16;
   return s;
 }
 
@@ -66,7 +98,7 @@ __host__ __device__ inline StSmem st_plan() {
 //   PH 1: strict statistics: the producers compute the scores; the consumers store
 //         every tile to an HBM score slab and keep, per row, the maximum m, its
 //         first key am and S_rest = sum over the other keys of exp(y - m) online
-//         across tiles (tile maximum and sum, merged in double);
+//         across tiles (tile maximum and sum, merged in double); no P.V;
 //   PH 2: strict selection: the producers refill the tile buffers from the slab;
 //         the consumers run the strict test with the row statistics of pass 1,
 //         then recompute, online softmax and P.V as in PH 0.
@@ -93,16 +125,30 @@ __device__ __forceinline__ int st_ntiles(int kv_end) { return kv_end > 0 ? (kv_e
 // Producers: every tile of every item, in the order the consumers take them.
 // ---------------------------------------------------------------------------
 template <int D, int RND, int PH>
-__device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem, const StSmem& L, int warp,
-                                            int lane) {
+__device__ __forceinline__ void st_producer(const StArgs& a, const CUtensorMap* tmK, unsigned char* smem,
+                                            const StSmem& L, int warp, int lane) {
   const Problem& p = a.p;
   const int G = gridDim.x, cta = blockIdx.x;
   const int s = 23 - p.mu;
   const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
   const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
   const u64 scale2 = pack2(p.scale, p.scale);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);  // full[0], full[1], empty[0], empty[1]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
+  float* qbase = reinterpret_cast<float*>(smem + L.q);
+  uint32_t kcount = 0;
+  KTma kt;
+  kt.map = tmK;
+  kt.ring = reinterpret_cast<uint16_t*>(smem + L.kring) + warp * KRING * WS_UNIT * WS_DS;
+  kt.bar = bars + sb_kring<D>() + warp * KRING;
+  kt.count = &kcount;
+  // Q of the first two items (the consumers stage the later ones)
+  for (int k0 = 0; k0 < 2; ++k0) {
+    const int q0 = ws_item(k0, cta, G, a.n_items);
+    if (q0 < 0) break;
+    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
+  }
+  named_sync(BAR_PROD, WS_NP * 32);
   int deal = 0;  // producer warp that takes the next unit
   int k = 0;     // tile counter: buffer k & 1, phase k >> 1
   for (int ii = 0;; ++ii) {
@@ -112,26 +158,33 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
-    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + (ii & 1) * ws_qfloats<D>();
+    const float* sQ = qbase + (ii & 1) * ws_qfloats<D>();
     const int nt = st_ntiles(it.kv_end);
     for (int t = 0; t < nt; ++t, ++k) {
       const int buf = k & 1;
       const int t0 = t * ST_T;
       const int tlen = max(0, min(ST_T, it.kv_end - t0));
-      // one decision per warp: the tile routine synchronises the whole warp
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars + 2 + buf, (k >> 1) & 1))) {  // tile buffer free (and the item's Q staged)
+      const uint32_t ph = ((k - 2) >> 1) & 1;
+      // the consumers' hand-off of tile k - 2 (and, at an item's first tile, its Q
+      // staged); one decision per warp: the tile routine synchronises the warp
+      if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + SB_PREADY + buf, ph))) {
         ws_timeout(p);
         return;
       }
-      float* tile = reinterpret_cast<float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
+      float* tile = reinterpret_cast<float*>(smem + L.tiles + buf * sw_bytes(ST_T));
       if (PH == 2) {
+        // the tile buffer is free once tile k - 2's P.V has completed and been read
+        if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + SB_TFREE + buf, ph))) {
+          ws_timeout(p);
+          return;
+        }
         // the tile's scores from the slab: rows of the item by cp.async, keys of the
         // tile that the scores pass wrote; rows past the item hold -inf
         const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;
         const int per_row = written / 4;  // 16-byte pieces
         for (int u = warp * 32 + lane; u < WS_BM * per_row; u += WS_NP * 32) {
           const int r = u / per_row, c4 = u % per_row;
-          float* dst = tile + (size_t)r * ST_TS + 4 * c4;
+          float* dst = tile + sw_off(r, 4 * c4);
           if (r < it.rows)
             cp_async16(dst, a.slab + ((size_t)it.bh * p.n_q + it.i0 + r) * a.ld + t0 + 4 * c4);
           else
@@ -140,24 +193,26 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
         cp_async_commit();
         cp_async_wait<0>();
       } else {
-        ws_produce_tile<D, RND>(p, it, t0, tlen, sQ, tile, ST_TS, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
-                                Kh, negc, pow2s, scale2, s);
+        // the tile buffer is free once tile k - 2's P.V has completed and been read
+        // (tfree): the tile routine waits for that only before its first store
+        if (!ws_produce_tile<D, RND, 1>(p, it, t0, tlen, sQ, tile, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
+                                        Kh, negc, pow2s, scale2, s, kt, k >= 2 ? bars + SB_TFREE + buf : nullptr,
+                                        ph)) {
+          ws_timeout(p);
+          return;
+        }
         deal = (deal + (tlen + WS_UNIT - 1) / WS_UNIT) % WS_NP;
       }
-      mbar_arrive(bars + buf);  // this thread's scores of the tile are in place
+      mbar_arrive(bars + SB_FULL + buf);  // this thread's scores of the tile are in place
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Consumers: selection, recompute, online softmax and P.V, tile by tile.
+// Consumers: selection, recompute and the online softmax, tile by tile.
 // ---------------------------------------------------------------------------
 template <int D, int RND, int VAR, int PH>
-__device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem, const StSmem& L, int cw,
-                                            int lane) {
-  constexpr int NH = D / 64;
-  constexpr int KQ = WS_NC / NH;
-  constexpr int WR = ws_vring<D>();
+__device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem, const StSmem& L, int cw, int lane) {
   constexpr int NCT = WS_NC * 32;
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
@@ -169,23 +224,9 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   const float thi = refine_ok ? (p.tau == 0.f ? 1e-30f : p.tau + band) : -INFINITY;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
-  uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L.v);
-  float* sO = reinterpret_cast<float*>(smem + L.v);
   float* qbase = reinterpret_cast<float*>(smem + L.q);
   float* rst = reinterpret_cast<float*>(smem + L.rstat);
-  const int nh = NH == 2 ? (cw & 1) : 0;
-  const int kq = NH == 2 ? (cw >> 1) : cw;
-  const int mi = lane >> 3;
-  uint16_t* vring = sV + cw * WR * 8 * WS_VSW;
   long long nsel = 0;
-  // Q of the first two items; both tile buffers start out free
-  for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = ws_item(k0, cta, G, a.n_items);
-    if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), tidc, NCT);
-  }
-  mbar_arrive(bars + 2);
-  mbar_arrive(bars + 3);
   int k = 0;
   for (int ii = 0;; ++ii) {
     const int q = ws_item(ii, cta, G, a.n_items);
@@ -194,7 +235,6 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
-    const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
     float* sQ = qbase + (ii & 1) * ws_qfloats<D>();
     const int nt = st_ntiles(it.kv_end);
     int rr_[2], nv[2];
@@ -210,6 +250,8 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
     int am_abs[2] = {0x7FFFFFFF, 0x7FFFFFFF};  // strict: first key of each row's maximum
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
+      S.rr[tt] = rr_[tt];
+      S.off[tt] = sw_off(rr_[tt], lane);
       S.live[tt] = rr_[tt] < it.rows;
       S.mrun[tt] = -INFINITY;
       if (VAR == LAMP_STRICT) {  // the row statistics of the scores pass
@@ -228,42 +270,19 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         S.mL[tt] = rs.m * kLog2e;
       }
     }
-    float acc[8][4];
-#pragma unroll
-    for (int tt = 0; tt < 8; ++tt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
+    // keys 128 i4 + 4 lane .. + 3 of row rr_[t]: scores at ob[t] + 2048 i4, P_hi at pbo[t] + 2048 i4
+    const int ob[2] = {sw_off(rr_[0], 4 * lane), sw_off(rr_[1], 4 * lane)};
+    const int pbo[2] = {p_off(rr_[0], 4 * lane), p_off(rr_[1], 4 * lane)};
 
     for (int t = 0; t < nt; ++t, ++k) {
       const int buf = k & 1;
       const int t0 = t * ST_T;
       const int tlen = max(0, min(ST_T, it.kv_end - t0));
       const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
-      float* tile = reinterpret_cast<float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
-      float* row[2] = {tile + (size_t)rr_[0] * ST_TS, tile + (size_t)rr_[1] * ST_TS};
-      // P.V split as in the whole-row kernel: warp (kq, nh) takes the tile's 8-key
-      // steps kq, kq + KQ, ... and columns nh*64 .. nh*64 + 63, staged in its own ring
-      const int ns_all = (tlen + 7) >> 3;
-      const int nsw = ns_all > kq ? (ns_all - kq + KQ - 1) / KQ : 0;
-      auto load_step = [&](int i) {  // step i of this warp into ring slot i % WR
-        if (i < nsw) {
-          const int key0 = t0 + 8 * (kq + KQ * i);
-          uint16_t* dst = vring + (i % WR) * 8 * WS_VSW;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int c = lane + 32 * h, key = c >> 3, ch = c & 7;
-            uint16_t* dd = dst + key * WS_VSW + ch * 8;
-            if (key0 + key < p.n_k) cp_async16(dd, Vh + (size_t)(key0 + key) * D + nh * 64 + ch * 8);
-            else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-        cp_async_commit();
-      };
-      for (int i = 0; i < WR - 1; ++i) load_step(i);  // V does not depend on the scores
-      const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
+      float* tile = reinterpret_cast<float*>(smem + L.tiles + buf * sw_bytes(ST_T));
+      const bool ok = mbar_wait(bars + SB_FULL + buf, (k >> 1) & 1);
       if (named_or(BAR_CONS, NCT, !ok)) {
         ws_timeout(p);
-        cp_async_wait<0>();
         return;
       }
       int nvr[2];
@@ -275,12 +294,12 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         for (int tt = 0; tt < 2; ++tt)
           if (rr_[tt] < it.rows)
             for (int j = lane; j < ST_T && t0 + j < p.n_k; j += 32)
-              p.ps_out[grow[tt] * p.n_k + t0 + j] = j < written ? row[tt][j] : -INFINITY;
+              p.ps_out[grow[tt] * p.n_k + t0 + j] = j < written ? tile[sw_off(rr_[tt], j)] : -INFINITY;
       }
       // criterion, mask words, compaction and recompute of the selected keys
+      S.base = tile;
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
-        S.row[tt] = row[tt];
         S.nv[tt] = nvr[tt];
         S.word0[tt] = grow[tt] * nwords + (t0 >> 5);
         S.mx[tt] = -INFINITY;
@@ -290,7 +309,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         sel_step<VAR>(p, S, 128 * i4, written, nwords - (t0 >> 5), tlo, thi, lane, wbuf, nsel);
       sel_finish(p, S, wbuf, 4 * nit, min(ST_T / 32, nwords - (t0 >> 5)), lane, [&](int tt, int j) {
         const float v = ws_recompute<D>(sQ, 2 * cw + tt, Kh + (size_t)(t0 + j) * D, p.scale, fast);
-        tile[(size_t)(2 * cw + tt) * ST_TS + j] = v;
+        tile[sw_off(2 * cw + tt, j)] = v;
         if (tt == 0) S.mx[0] = fmaxf(S.mx[0], v);
         else S.mx[1] = fmaxf(S.mx[1], v);
       });
@@ -300,7 +319,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
         for (int tt = 0; tt < 2; ++tt)
           if (rr_[tt] < it.rows)
             for (int j = lane; j < ST_T && t0 + j < p.n_k; j += 32)
-              p.mixed_out[grow[tt] * p.n_k + t0 + j] = j < written ? row[tt][j] : -INFINITY;
+              p.mixed_out[grow[tt] * p.n_k + t0 + j] = j < written ? tile[sw_off(rr_[tt], j)] : -INFINITY;
       }
       // online softmax: new maximum, rescale factor, numerators of this tile in place
       const int nitw = (written + 127) >> 7;
@@ -314,93 +333,51 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
       }
       for (int i4 = 0; i4 < nitw; ++i4) {
         const int j0 = 128 * i4 + 4 * lane;
-        if (j0 >= written) continue;
+        const bool act = j0 < written;
+        float4 v[2];
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const float4 v = *reinterpret_cast<const float4*>(row[tt] + j0);
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-          uint32_t pw[4];
+        for (int tt = 0; tt < 2; ++tt) v[tt] = act ? *reinterpret_cast<const float4*>(tile + ob[tt] + 2048 * i4)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();  // the 128 keys of both rows are read before any lane overwrites them
+        if (act) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float pj;  // exp(y - m), 0 for -inf
-            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(pj) : "f"(fmaf(vv[e], kLog2e, -mL[tt])));
-            lt[tt] += pj;
-            pw[e] = p_pair_cvt(pj);
+          for (int tt = 0; tt < 2; ++tt) {
+            const float vv[4] = {v[tt].x, v[tt].y, v[tt].z, v[tt].w};
+            uint32_t pw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float pj;  // exp(y - m), 0 for -inf
+              asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(pj) : "f"(fmaf(vv[e], kLog2e, -mL[tt])));
+              lt[tt] += pj;
+              pw[e] = p_pair_cvt(pj);  // low half bf16(P), high half bf16(P - bf16(P))
+            }
+            float* dst = tile + pbo[tt] + 2048 * i4;
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(__byte_perm(pw[0], pw[1], 0x5410), __byte_perm(pw[2], pw[3], 0x5410));
+            *reinterpret_cast<uint2*>(dst + 512) =
+                make_uint2(__byte_perm(pw[0], pw[1], 0x7632), __byte_perm(pw[2], pw[3], 0x7632));
           }
-          *reinterpret_cast<uint4*>(row[tt] + j0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
       }
+      float* rs = rst + buf * WS_BM * 4;
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
         l[tt] = l[tt] * alpha[tt] + warp_sum(lt[tt]);
         if (lane == 0) {
-          rst[4 * rr_[tt]] = m[tt];
-          rst[4 * rr_[tt] + 1] = l[tt];
-          rst[4 * rr_[tt] + 2] = alpha[tt];
+          rs[4 * rr_[tt]] = m[tt];
+          rs[4 * rr_[tt] + 1] = l[tt];
+          rs[4 * rr_[tt] + 2] = alpha[tt];
         }
       }
-      named_sync(BAR_CONS, NCT);  // P of the tile and every row's rescale factor are in place
+      fence_async_smem();  // P (generic-proxy stores) becomes visible to the tensor core
+      named_sync(BAR_CONS, NCT);  // P and every row's m, l, alpha of the tile are in place
+      if (t == nt - 1) {   // Q of the item is no longer read: stage item + 2's
+        const int q2 = ws_item(ii + 2, cta, G, a.n_items);
+        if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
+      }
+      mbar_arrive(bars + SB_PREADY + buf);  // P of the tile in place (and at an item's end, Q of item + 2)
 
-      // rescale the partial outputs, then add P.V of this tile
-      {
-        const float a0 = rst[4 * (lane >> 2) + 2], a1 = rst[4 * ((lane >> 2) + 8) + 2];
-#pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-          acc[tt][0] *= a0;
-          acc[tt][1] *= a0;
-          acc[tt][2] *= a1;
-          acc[tt][3] *= a1;
-        }
-      }
-      const int ra = 8 * (mi & 1) + (lane & 7);
-      const int kl = 4 * (mi & 1) + ((lane & 7) >> 1);  // each V row serves the hi and the lo half of P
-      for (int i = 0; i < nsw; ++i) {
-        cp_async_wait<WR - 2>();  // step i has landed (this lane's copies)
-        __syncwarp();             // ... and every lane's; step i - 1's slot is free
-        load_step(i + WR - 1);
-        const int kb = 8 * (kq + KQ * i);  // relative to the tile
-        const uint16_t* vb = vring + (i % WR) * 8 * WS_VSW;
-        uint32_t af[4];
-        ldmatrix_x4(smem_u32(tile + (size_t)ra * ST_TS + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
-#pragma unroll
-        for (int nb = 0; nb < 4; ++nb) {
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(smem_u32(vb + kl * WS_VSW + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
-          mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
-          mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
-        }
-      }
-      cp_async_wait<0>();
-      named_sync(BAR_CONS, NCT);  // V stages and rescale factors are no longer read
-
-      if (t == nt - 1) {  // end of the item: add the partial outputs, divide by l
-#pragma unroll
-        for (int tt = 0; tt < 8; ++tt)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int rr = (lane >> 2) + 8 * h;
-            *reinterpret_cast<float2*>(sO + ((size_t)kq * WS_BM + rr) * D + nh * 64 + 8 * tt + 2 * (lane & 3)) =
-                make_float2(acc[tt][2 * h], acc[tt][2 * h + 1]);
-          }
-        named_sync(BAR_CONS, NCT);
-        for (int u = tidc; u < WS_BM * D / 2; u += NCT) {
-          const int rr = u / (D / 2), col = (u % (D / 2)) * 2;
-          if (rr >= it.rows) continue;
-          float2 o = *reinterpret_cast<const float2*>(sO + rr * D + col);
-#pragma unroll
-          for (int g = 1; g < KQ; ++g) {
-            const float2 v = *reinterpret_cast<const float2*>(sO + ((size_t)g * WS_BM + rr) * D + col);
-            o.x += v.x;
-            o.y += v.y;
-          }
-          const float lv = rst[4 * rr + 1];
-          const float inv = lv > 0.f ? 1.f / lv : 0.f;
-          const float v0 = o.x * inv, v1 = o.y * inv;
-          const size_t off = ((size_t)it.bh * p.n_q + it.i0 + rr) * D + col;
-          *reinterpret_cast<uint32_t*>(p.out + off) =
-              (uint32_t)f32_to_bf16_rne(v0) | ((uint32_t)f32_to_bf16_rne(v1) << 16);
-          if (p.out_f32) *reinterpret_cast<float2*>(p.out_f32 + off) = make_float2(v0, v1);
-        }
+      if (t == nt - 1) {  // end of the item: lse, and the parts of the dumps past its tiles
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
           if (rr_[tt] >= it.rows) continue;
@@ -413,11 +390,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
           if (p.mixed_out)
             for (int j = done + lane; j < p.n_k; j += 32) p.mixed_out[grow[tt] * p.n_k + j] = -INFINITY;
         }
-        named_sync(BAR_CONS, NCT);  // the output sums (V area) and this item's Q are no longer read
-        const int q2 = ws_item(ii + 2, cta, G, a.n_items);
-        if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
       }
-      mbar_arrive(bars + 2 + buf);  // tile buffer free (and, after an item's last tile, Q of item + 2 staged)
     }
   }
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
@@ -439,13 +412,6 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
   const int G = gridDim.x, cta = blockIdx.x;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* qbase = reinterpret_cast<float*>(smem + L.q);
-  for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = ws_item(k0, cta, G, a.n_items);
-    if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), tidc, NCT);
-  }
-  mbar_arrive(bars + 2);
-  mbar_arrive(bars + 3);
   int k = 0;
   for (int ii = 0;; ++ii) {
     const int q = ws_item(ii, cta, G, a.n_items);
@@ -468,8 +434,8 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
       const int t0 = t * ST_T;
       const int tlen = max(0, min(ST_T, it.kv_end - t0));
       const int written = ((tlen + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;
-      const float* tile = reinterpret_cast<const float*>(smem + L.tiles) + (size_t)buf * WS_BM * ST_TS;
-      const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
+      const float* tile = reinterpret_cast<const float*>(smem + L.tiles + buf * sw_bytes(ST_T));
+      const bool ok = mbar_wait(bars + SB_FULL + buf, (k >> 1) & 1);
       if (named_or(BAR_CONS, NCT, !ok)) {
         ws_timeout(p);
         return;
@@ -477,17 +443,18 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
       const int nit = (written + 127) >> 7;
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
-        const float* row = tile + (size_t)rr_[tt] * ST_TS;
+        const int ob = sw_off(rr_[tt], 4 * lane);  // key 128 i4 + 4 lane at ob + 2048 i4
         if (rr_[tt] < it.rows) {
           float* dst = a.slab + grow[tt] * a.ld + t0;
-          for (int j0 = 4 * lane; j0 < written; j0 += 128)
-            *reinterpret_cast<float4*>(dst + j0) = *reinterpret_cast<const float4*>(row + j0);
+          for (int i4 = 0; 128 * i4 + 4 * lane < written; ++i4)
+            *reinterpret_cast<float4*>(dst + 128 * i4 + 4 * lane) =
+                *reinterpret_cast<const float4*>(tile + ob + 2048 * i4);
         }
         float lm = -INFINITY;
         int li = 0x7FFFFFFF;
         for (int i4 = 0; i4 < nit; ++i4) {
           const int j0 = 128 * i4 + 4 * lane;
-          const float4 v = lds4_or_ninf(row + j0, j0 < written);
+          const float4 v = lds4_or_ninf(tile + ob + 2048 * i4, j0 < written);
           if (v.x > lm) { lm = v.x; li = j0; }
           if (v.y > lm) { lm = v.y; li = j0 + 1; }
           if (v.z > lm) { lm = v.z; li = j0 + 2; }
@@ -500,7 +467,7 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
           const float ml = mt * kLog2e;  // exp(y - mt) on the special-function unit, as in the selection
           for (int i4 = 0; i4 < nit; ++i4) {
             const int j0 = 128 * i4 + 4 * lane;
-            const float4 v = lds4_or_ninf(row + j0, j0 < written);
+            const float4 v = lds4_or_ninf(tile + ob + 2048 * i4, j0 < written);
             const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -529,58 +496,283 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
             rs.srest = Sacc[tt];
             a.rows[grow[tt]] = rs;
           }
+        // this pass reads no Q, and the producers are done with the item's
         const int q2 = ws_item(ii + 2, cta, G, a.n_items);
         if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
       }
-      mbar_arrive(bars + 2 + buf);  // tile buffer free (and, after an item's last tile, Q of item + 2 staged)
+      mbar_arrive(bars + SB_PREADY + buf);  // tile buffer read (and, after an item's last tile, Q of item + 2 staged)
     }
   }
 }
 
-template <int D, int RND, int VAR, int PH>
-__global__ void __launch_bounds__(WS_NP * 32 + WS_NC * 32, 1) st_kernel(const StArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const StSmem L = st_plan<D>();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-    mbar_init(bars + 0, WS_NP * 32);  // full[0]
-    mbar_init(bars + 1, WS_NP * 32);  // full[1]
-    mbar_init(bars + 2, WS_NC * 32);  // empty[0]
-    mbar_init(bars + 3, WS_NC * 32);  // empty[1]
-    mbar_fence_init();
+// ---------------------------------------------------------------------------
+// Tensor-core warpgroup (warps 16-19, ew = warp - 16). Per score tile, lane 0 of
+// warp 16 streams the V tiles by TMA and issues the tile's P.V by tcgen05.mma
+// (in the statistics pass it only hands the buffer on); then the four warps
+// (TMEM lane quarter ew: head dimensions 32 ew + lane, or 16 ew + lane in lanes
+// 0-15 for the M = 64 shape of d = 64) fold the tile into their register
+// accumulator, O = (alpha O + P_hi.V) + P_lo.V with alpha = exp(m_old - m_new)
+// of each row, release the buffer (tfree), and after an item's last tile store
+// O / l as bf16 through a shared-memory tile with 16-byte stores.
+// ---------------------------------------------------------------------------
+template <int D, int PH>
+__device__ __forceinline__ void st_tensor_warpgroup(const StArgs& a, const CUtensorMap* tmV, unsigned char* smem,
+                                                    const StSmem& L, uint32_t tbase, int ew, int lane) {
+  constexpr int S = st_vslots<D>();
+  constexpr uint32_t TB = st_vtile_bytes<D>();
+  const Problem& p = a.p;
+  const int G = gridDim.x, cta = blockIdx.x;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  unsigned char* vring = smem + L.v;
+  const uint32_t vbase = smem_u32(vring), tiles = smem_u32(smem + L.tiles);
+  const uint32_t idesc = umma_idesc_bf16(D, 32);
+  const float* rst = reinterpret_cast<const float*>(smem + L.rstat);
+  uint16_t* otile = reinterpret_cast<uint16_t*>(smem + L.otile);
+  const bool issuer = ew == 0 && lane == 0;
+  bool ok = true;
+  // V tiles form one sequence over the CTA's score tiles: V tile vt of score tile
+  // (item il, tile tl) is number gl
+  int il = 0, tl = 0, ntl = -1, bhl = 0, kvl = 0, vt = 0, nvl = -1;
+  int gl = 0, gm = 0;  // next V tile to load, next V tile to multiply
+  auto next_v = [&]() -> bool {
+    for (;;) {
+      if (ntl < 0) {  // enter item il
+        const int q = ws_item(il, cta, G, a.n_items);
+        if (q < 0) return false;
+        const ItemInfo it = ws_decode(q, p, a.n_rb);
+        ntl = st_ntiles(it.kv_end);
+        bhl = it.bh;
+        kvl = it.kv_end;
+        tl = 0;
+        nvl = -1;
+      }
+      if (tl < ntl) {
+        if (nvl < 0) {  // enter score tile tl
+          const int tlen = max(0, min(ST_T, kvl - tl * ST_T));
+          nvl = (tlen + WS_VKEYS - 1) / WS_VKEYS;
+          vt = 0;
+        }
+        if (vt < nvl) return true;
+        ++tl;
+        nvl = -1;
+        continue;
+      }
+      ++il;
+      ntl = -1;
+    }
+  };
+  auto load_upto = [&](int limit) {  // start the loads of V tiles gl .. limit - 1
+    while (ok && gl < limit && next_v()) {
+      const int slot = gl % S;
+      if (gl >= S && !mbar_wait(bars + sb_vempty<D>() + slot, ((gl / S) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      mbar_expect_tx(bars + SB_VFULL + slot, TB);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tma_load_3d(vring + slot * TB + h * 8192, tmV, 64 * h, tl * ST_T + WS_VKEYS * vt, bhl,
+                    bars + SB_VFULL + slot);
+      ++vt;
+      ++gl;
+    }
+  };
+  // P.V of score tile k (the issuing thread only)
+  auto mma_tile = [&](int k, int tlen) {
+    const int buf = k & 1;
+    const int T = (tlen + WS_VKEYS - 1) / WS_VKEYS;
+    if (PH != 1) load_upto(gm + S);
+    if (!ok || !mbar_wait(bars + SB_PREADY + buf, (k >> 1) & 1)) {
+      ok = false;
+      return;
+    }
+    if (PH == 1) {  // the statistics pass reads the tile on the CUDA cores only
+      mbar_arrive(bars + SB_EMPTY + buf);
+      return;
+    }
+    tc_fence_after();
+    const uint32_t dcol = tbase + 32 * buf;
+    const uint32_t pb = tiles + buf * sw_bytes(ST_T);
+    for (int v = 0; v < T; ++v, ++gm) {
+      load_upto(gm + S - 1);  // keep the ring full (waits for the MMAs two V tiles back)
+      const int slot = gm % S;
+      if (!ok || !mbar_wait(bars + SB_VFULL + slot, (gm / S) & 1)) {
+        ok = false;
+        return;
+      }
+      tc_fence_after();
+      const uint32_t va = vbase + slot * TB, pa = pb + v * 4096;
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) {  // 16 keys per MMA
+        const uint64_t ad = umma_desc_sw128(va + s4 * 2048, D == 128 ? 8192u : 0u, 1024);
+        const uint64_t bd = umma_desc_sw128(pa + s4 * 32, 16, 1024);
+        umma_bf16(dcol, ad, bd, idesc, (v | s4) != 0);
+      }
+      umma_commit(bars + sb_vempty<D>() + slot);
+    }
+    umma_commit(bars + SB_EMPTY + buf);  // the tile's P.V is complete
+  };
+  const int dim = D == 128 ? 32 * ew + lane : 16 * ew + lane;
+  const bool dim_ok = D == 128 || lane < 16;
+  bool good = true;
+  int k = 0;
+  for (int ii = 0; good; ++ii) {
+    const int q = ws_item(ii, cta, G, a.n_items);
+    if (q < 0) break;
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    const int nt = st_ntiles(it.kv_end);
+    float o[WS_BM];  // this thread's head dimension of the item's 16 rows
+#pragma unroll
+    for (int r = 0; r < WS_BM; ++r) o[r] = 0.f;
+    for (int t = 0; t < nt; ++t, ++k) {
+      const int buf = k & 1;
+      if (issuer && ok) mma_tile(k, max(0, min(ST_T, it.kv_end - t * ST_T)));
+      __syncwarp();
+      // a failed issue leaves the tile incomplete: the bounded wait below then
+      // gives up, and all four warps agree on it
+      const bool done = mbar_wait(bars + SB_EMPTY + buf, (k >> 1) & 1);
+      if (named_or(BAR_EPI, 128, !done)) {
+        good = false;
+        break;
+      }
+      if (PH != 1) {
+        tc_fence_after();
+        const float* rs = rst + buf * WS_BM * 4;
+        const uint32_t ta = tbase + 32 * buf + ((uint32_t)(32 * ew) << 16);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // rows 8h .. 8h + 7: O = alpha O + P_hi.V, then + P_lo.V
+          float v[8];
+          tmem_ld8(ta + 8 * h, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) o[8 * h + j] = fmaf(o[8 * h + j], rs[4 * (8 * h + j) + 2], v[j]);
+          tmem_ld8(ta + 16 + 8 * h, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) o[8 * h + j] = __fadd_rn(o[8 * h + j], v[j]);
+        }
+        if (t == nt - 1) {
+#pragma unroll
+          for (int r = 0; r < WS_BM; ++r) {
+            const float lv = rs[4 * r + 1];
+            o[r] = lv > 0.f ? o[r] * (1.f / lv) : 0.f;
+          }
+        }
+        tc_fence_before();
+      }
+      mbar_arrive(bars + SB_TFREE + buf);  // accumulator, row statistics and tile buffer are free
+      if (PH != 1 && t == nt - 1) {       // the item's output
+        if (dim_ok) {
+#pragma unroll
+          for (int r = 0; r < WS_BM; ++r) {
+            otile[r * D + dim] = f32_to_bf16_rne(o[r]);
+            if (p.out_f32 && r < it.rows) p.out_f32[((size_t)it.bh * p.n_q + it.i0 + r) * D + dim] = o[r];
+          }
+        }
+        named_sync(BAR_EPI, 128);
+        for (int c = ew * 32 + lane; c < WS_BM * D / 8; c += 128) {
+          const int r = c / (D / 8), c8 = (c % (D / 8)) * 8;
+          if (r < it.rows)
+            *reinterpret_cast<uint4*>(p.out + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8) =
+                *reinterpret_cast<const uint4*>(otile + r * D + c8);
+        }
+        named_sync(BAR_EPI, 128);  // the tile may be refilled
+      }
+    }
   }
-  __syncthreads();
-  if (warp < WS_NP) st_producer<D, RND, PH>(a, smem, L, warp, lane);
-  else if (PH == 1) st_consumer_stats<D>(a, smem, L, warp - WS_NP, lane);
-  else st_consumer<D, RND, VAR, PH>(a, smem, L, warp - WS_NP, lane);
+  if (issuer) {
+    // drain: every MMA issued and every V load in flight completes before the
+    // tensor memory is released and the CTA exits
+    umma_commit(bars + sb_drain<D>());
+    bool drained = mbar_wait(bars + sb_drain<D>(), 0);
+    for (int g = gm; g < gl; ++g) drained = mbar_wait(bars + SB_VFULL + g % S, (g / S) & 1) && drained;
+    if (!ok || !drained) good = false;
+  }
+  if (!good && lane == 0) ws_timeout(p);
 }
 
 template <int D, int RND, int VAR, int PH>
-cudaError_t st_launch_one(const StArgs& a, int grid, cudaStream_t st) {
+__global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __grid_constant__ CUtensorMap tmK,
+                                                     const __grid_constant__ CUtensorMap tmV) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + smem_align1k_pad(smem_raw);
+  const StSmem L = st_plan<D>();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.tmem);
+  if (threadIdx.x == 0) {
+    mbar_init(bars + SB_FULL + 0, WS_NP * 32);
+    mbar_init(bars + SB_FULL + 1, WS_NP * 32);
+    mbar_init(bars + SB_PREADY + 0, WS_NC * 32);
+    mbar_init(bars + SB_PREADY + 1, WS_NC * 32);
+    mbar_init(bars + SB_EMPTY + 0, 1);
+    mbar_init(bars + SB_EMPTY + 1, 1);
+    mbar_init(bars + SB_TFREE + 0, 128);
+    mbar_init(bars + SB_TFREE + 1, 128);
+    for (int i = 0; i < st_vslots<D>(); ++i) {
+      mbar_init(bars + SB_VFULL + i, 1);
+      mbar_init(bars + sb_vempty<D>() + i, 1);
+    }
+    mbar_init(bars + sb_drain<D>(), 1);
+    for (int i = 0; i < WS_NP * KRING; ++i) mbar_init(bars + sb_kring<D>() + i, 1);
+    mbar_fence_init();
+  }
+  if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  if (warp < WS_NP) {
+    regs_inc<kWsProdRegs>();
+    st_producer<D, RND, PH>(a, &tmK, smem, L, warp, lane);
+  } else if (warp < WS_MW) {
+    regs_inc<kWsConsRegs>();
+    if (PH == 1) st_consumer_stats<D>(a, smem, L, warp - WS_NP, lane);
+    else st_consumer<D, RND, VAR, PH>(a, smem, L, warp - WS_NP, lane);
+  } else {
+    regs_dec<kWsMmaRegs>();
+    st_tensor_warpgroup<D, PH>(a, &tmV, smem, L, tbase, warp - WS_MW, lane);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WS_MW) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, WS_TMEM_COLS);
+  }
+}
+
+template <int D, int RND, int VAR, int PH>
+cudaError_t st_launch_one(const StArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmV, int grid, cudaStream_t st) {
   auto k = st_kernel<D, RND, VAR, PH>;
-  const size_t smem = (size_t)st_plan<D>().total;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k);
   if (e != cudaSuccess) return e;
-  k<<<grid, WS_NP * 32 + WS_NC * 32, smem, st>>>(a);
+  if (fa.numRegs != kWsLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split assumes this pool
+  const size_t smem = (size_t)st_plan<D>().total + 1024;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, WS_NT, smem, st>>>(a, tmK, tmV);
   return cudaGetLastError();
 }
 
 template <int D, int RND>
-cudaError_t st_launch_var(const StArgs& a, int grid, cudaStream_t st) {
-  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK, 0>(a, grid, st);
-  if (a.p.variant == LAMP_RELAXED) return st_launch_one<D, RND, LAMP_RELAXED, 0>(a, grid, st);
+cudaError_t st_launch_var(const StArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmV, int grid, cudaStream_t st) {
+  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK, 0>(a, tmK, tmV, grid, st);
+  if (a.p.variant == LAMP_RELAXED) return st_launch_one<D, RND, LAMP_RELAXED, 0>(a, tmK, tmV, grid, st);
   // strict: the scores-and-statistics pass, then the selection pass
-  cudaError_t e = st_launch_one<D, RND, LAMP_STRICT, 1>(a, grid, st);
+  cudaError_t e = st_launch_one<D, RND, LAMP_STRICT, 1>(a, tmK, tmV, grid, st);
   if (e != cudaSuccess) return e;
-  return st_launch_one<D, RND, LAMP_STRICT, 2>(a, grid, st);
+  return st_launch_one<D, RND, LAMP_STRICT, 2>(a, tmK, tmV, grid, st);
 }
 
 }  // namespace
 
 size_t stream_slab_ld(int n_k) { return (size_t)((n_k + ST_T - 1) / ST_T) * ST_T; }
 
-size_t stream_smem_bytes(int d) { return d == 64 ? (size_t)st_plan<64>().total : (size_t)st_plan<128>().total; }
+size_t stream_smem_bytes(int d) {  // dynamic shared memory of a launch (with the alignment slack)
+  return (d == 64 ? (size_t)st_plan<64>().total : (size_t)st_plan<128>().total) + 1024;
+}
 
 cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st) {
   StArgs a;
@@ -592,16 +784,20 @@ cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int
   a.slab = reinterpret_cast<float*>(base + ws.st_slab);
   a.ld = stream_slab_ld(p.n_k);
   a.rows = reinterpret_cast<RowStat*>(base + ws.st_rows);
+  CUtensorMap tmK, tmV;
+  cudaError_t e = make_tmap_bf16(&tmK, p.K, p.d, p.n_k, p.B * p.H, WS_DS, WS_UNIT, false);
+  if (e == cudaSuccess) e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, true);
+  if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
   if (p.d == 64) {
-    if (rnd == kRndFast) return st_launch_var<64, kRndFast>(a, grid, st);
-    if (rnd == kRndNone) return st_launch_var<64, kRndNone>(a, grid, st);
-    return st_launch_var<64, kRndExact>(a, grid, st);
+    if (rnd == kRndFast) return st_launch_var<64, kRndFast>(a, tmK, tmV, grid, st);
+    if (rnd == kRndNone) return st_launch_var<64, kRndNone>(a, tmK, tmV, grid, st);
+    return st_launch_var<64, kRndExact>(a, tmK, tmV, grid, st);
   }
-  if (rnd == kRndFast) return st_launch_var<128, kRndFast>(a, grid, st);
-  if (rnd == kRndNone) return st_launch_var<128, kRndNone>(a, grid, st);
-  return st_launch_var<128, kRndExact>(a, grid, st);
+  if (rnd == kRndFast) return st_launch_var<128, kRndFast>(a, tmK, tmV, grid, st);
+  if (rnd == kRndNone) return st_launch_var<128, kRndNone>(a, tmK, tmV, grid, st);
+  return st_launch_var<128, kRndExact>(a, tmK, tmV, grid, st);
 }
 
 }  // namespace lamp

@@ -1,6 +1,7 @@
 // LAMP attention, warp-specialised row kernel (strict, relaxed, given mask) for
 // rows short enough that two blocks of 16 complete score rows fit in shared
-// memory at once (n_k up to about a thousand keys; the GPT-2 XL attention shape).
+// memory at once (n_k up to 1024 keys at d = 64, 960 at d = 128; the GPT-2 XL
+// attention shape).
 //
 // Method ("LAMP: Look-Ahead Mixed-Precision Inference of Large Language Models",
 // technical summary, gist.science paper 2601.21623): section "Implementation
@@ -8,29 +9,40 @@
 // strict test 2 z (1 - z) |y| > tau on the whole probability row); section
 // "Experimental results" (PS(mu), relaxed relative threshold, random control).
 //
-// One persistent CTA of 512 threads per SM works through a fixed sequence of
-// items (b, h, block of 16 query rows), heaviest causal blocks first, in a snake
-// order over the CTAs. Two row buffers alternate between two warp groups:
+// One persistent CTA of 640 threads (5 warpgroups) per SM works through a fixed
+// sequence of items (b, h, block of 16 query rows), heaviest causal blocks first,
+// in a snake order over the CTAs. Two row buffers alternate between three warp
+// roles, each warpgroup with its own register budget (setmaxnreg):
 //
 //   producers (warps 0-7): PS(mu) scores of item k into buffer k & 1. The item's
 //     keys are cut into 64-key units dealt round-robin to the producer warps,
 //     continuing across items. Each warp stages its own K slices (8 head
-//     dimensions x 64 keys, binary32, double buffered) and waits for nothing but
-//     a free buffer. A lane holds 8 rows x 4 keys as sixteen packed binary32
-//     pairs (two rows of one key per 64-bit register): one accumulation step is
-//     fma.rn.f32x2 plus the two-instruction PS(mu) rounding (or the exact
-//     integer rounding), and three shared-memory loads feed 16 packed steps.
+//     dimensions x 64 keys, binary32, double buffered). A lane holds 8 rows x 4
+//     keys as sixteen packed binary32 pairs (two rows of one key per 64-bit
+//     register): one accumulation step is fma.rn.f32x2 plus the two-instruction
+//     PS(mu) rounding (or the exact integer rounding).
 //   consumers (warps 8-15): for item k, two rows per warp, four keys per lane:
-//     row maximum and first argmax, S_rest in double (strict), the criterion
-//     with a double re-evaluation near tau, mask words, warp-compacted FP32
-//     recompute, softmax numerators of the mixed row written in place as bf16
-//     hi/lo pairs; then P.V on tensor cores (mma.sync, V staged by cp.async), the
-//     output, and the staging of Q for item k + 2.
+//     row maximum and first argmax, S_rest in double (strict), the criterion with
+//     a double re-evaluation near tau, mask words, warp-compacted FP32 recompute,
+//     then the softmax numerators of the mixed row written in place as bf16 hi/lo
+//     parts in the tensor-core operand layout (sw_off / p_off), and the staging of
+//     Q for item k + 2.
+//   tensor-core warpgroup (warps 16-19): one thread streams V tiles of 64 keys by
+//     TMA into a ring of shared-memory slots (running ahead across items) and, for
+//     each item once its P is in place, issues O^T = V^T P^T by tcgen05.mma into
+//     one of two TMEM accumulators (lamp_umma.cuh); tcgen05.commit frees each V
+//     slot and signals the item's completion. Then the four warps (one per TMEM
+//     lane quarter) read the accumulator, scale by 1 / l and store the output
+//     with 16-byte stores through a shared-memory tile.
 //
-// Hand-offs use mbarriers: full[b] (256 producer arrivals per item) and empty[b]
-// (256 consumer arrivals: the buffer and its Q are ready for the next item).
+// Hand-offs use mbarriers: full[b] (256 producer arrivals: the scores are in
+// place), pready[b] (256 consumer arrivals: P in place, Q of item k + 2 staged),
+// empty[b] (the item's MMAs have completed), tfree[b] (128 epilogue arrivals:
+// accumulator and row statistics read, so the buffer may be refilled),
+// vfull/vempty per V slot.
 // Every wait is bounded; a wait that gives up records LAMP_ERR_TIMEOUT in the
-// caller's status word (when given) and ends the kernel.
+// caller's status word (when given) and ends the kernel after the tensor-core
+// work in flight has drained and the tensor memory is released.
 #include <cfloat>
 
 #include "lamp_ws_common.cuh"
@@ -38,30 +50,46 @@
 namespace lamp {
 namespace {
 
-struct WsSmem {
-  int bars;   // mbarriers: full[2], empty[2]
-  int q;      // Q [2][D][16] f32
+template <int D>
+__host__ __device__ constexpr int ws_vslots() { return D == 64 ? 6 : 3; }  // V tiles in the ring
+template <int D>
+__host__ __device__ constexpr int ws_vtile_bytes() { return WS_VKEYS * D * 2; }  // 64 keys x D dimensions, bf16
+
+// mbarrier indices
+constexpr int BAR_FULL = 0, BAR_PREADY = 2, BAR_EMPTY = 4, BAR_TFREE = 6, BAR_VFULL = 8;
+template <int D>
+__host__ __device__ constexpr int bar_vempty() { return BAR_VFULL + ws_vslots<D>(); }
+template <int D>
+__host__ __device__ constexpr int bar_drain() { return BAR_VFULL + 2 * ws_vslots<D>(); }
+constexpr int BAR_PROD = 2;  // named barrier of the producer group
+constexpr int BAR_EPI = 3;   // named barrier of the tensor-core warpgroup (output epilogue)
+
+struct WsSmem {  // byte offsets from a 1024-byte aligned base
+  int rows;   // score rows [2][sw_bytes(n_k)] (block layout of lamp_ws_common.cuh)
+  int v;      // V ring [S][D / 64][64 keys][64 dims] bf16, as the TMA leaves it (128-byte swizzle)
   int ks;     // producer K slices [8 warps][2][8][64] f32
-  int v;      // consumer V rings [8 warps][WR][8][72] bf16, later the partial outputs [KQ][16][D] f32
+  int q;      // Q [2][D][16] f32
   int list;   // consumer mask-word buffers [8][2][32] uint32
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
-  int rows;   // score rows [2][16][nkp] f32
+  int otile;  // output tile of an item [16][D] bf16 (epilogue)
+  int bars;   // mbarriers
+  int tmem;   // TMEM base address (written by tcgen05.alloc)
   int total;
 };
 
 template <int D>
-__host__ __device__ inline WsSmem ws_plan(int nkp) {
+__host__ __device__ inline WsSmem ws_plan(int n_k) {
   WsSmem s{};
-  s.bars = 0;
-  s.q = 64;
-  s.ks = s.q + 2 * ws_qfloats<D>() * 4;
-  s.v = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
-  const int vb = WS_NC * ws_vring<D>() * 8 * WS_VSW * 2;  // per-warp V rings
-  const int ob = (WS_NC / (D / 64)) * WS_BM * D * 4;  // per-warp partial outputs
-  s.list = s.v + (vb > ob ? vb : ob);
+  s.rows = 0;
+  s.v = 2 * sw_bytes(n_k);
+  s.ks = s.v + ws_vslots<D>() * ws_vtile_bytes<D>();
+  s.q = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
+  s.list = s.q + 2 * ws_qfloats<D>() * 4;
   s.stats = s.list + WS_NC * 2 * SEL_WMAX * 4;
-  s.rows = s.stats + 2 * WS_BM * 2 * 4;
-  s.total = s.rows + 2 * WS_BM * nkp * 4;
+  s.otile = s.stats + 2 * WS_BM * 2 * 4;
+  s.bars = s.otile + WS_BM * D * 2;
+  s.tmem = s.bars + (bar_drain<D>() + 1) * 8;
+  s.total = s.tmem + 16;
   return s;
 }
 
@@ -69,7 +97,6 @@ struct WsArgs {
   Problem p;
   const int* stats;  // per-(b, h) exponent statistics
   int nchunk;
-  int nkp;           // row stride in floats
   int n_items;
   int n_rb;
 };
@@ -86,41 +113,106 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
   const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
   const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
   const u64 scale2 = pack2(p.scale, p.scale);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);  // full[0], full[1], empty[0], empty[1]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
-  int deal = 0;  // producer warp that takes the next unit
+  float* qbase = reinterpret_cast<float*>(smem + L.q);
+  const int rb = sw_bytes(p.n_k);
+  // Q of the first two items (the consumers stage the later ones)
+  for (int k0 = 0; k0 < 2; ++k0) {
+    const int q0 = ws_item(k0, cta, G, a.n_items);
+    if (q0 < 0) break;
+    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
+  }
+  named_sync(BAR_PROD, WS_NP * 32);
+  const KTma kt{};  // K staged through registers
+  int deal = 0;     // producer warp that takes the next unit
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
     if (q < 0) break;
     const int buf = k & 1;
     const ItemInfo it = ws_decode(q, p, a.n_rb);
-    // one decision per warp: the tile routine synchronises the whole warp
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars + 2 + buf, (k >> 1) & 1))) {  // buffer free, Q staged
+    const uint32_t ph = ((k - 2) >> 1) & 1;
+    // Q of item k is staged (with the consumers' hand-off of item k - 2); one
+    // decision per warp: the tile routine synchronises the whole warp
+    if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + BAR_PREADY + buf, ph))) {
       ws_timeout(p);
       return;
     }
-    const float* sQ = reinterpret_cast<const float*>(smem + L.q) + buf * ws_qfloats<D>();
+    const float* sQ = qbase + buf * ws_qfloats<D>();
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
-    float* rows = reinterpret_cast<float*>(smem + L.rows) + (size_t)buf * WS_BM * a.nkp;
+    float* rows = reinterpret_cast<float*>(smem + L.rows + buf * rb);
     const int U = (it.kv_end + WS_UNIT - 1) / WS_UNIT;
-    ws_produce_tile<D, RND>(p, it, 0, it.kv_end, sQ, rows, a.nkp, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
-                            negc, pow2s, scale2, s);
+    // the buffer itself is free once item k - 2's P.V has completed and its
+    // output has been read (tfree): the tile routine waits for that only before
+    // its first store
+    if (!ws_produce_tile<D, RND, 0>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
+                                    Kh, negc, pow2s, scale2, s, kt, k >= 2 ? bars + BAR_TFREE + buf : nullptr, ph)) {
+      ws_timeout(p);
+      return;
+    }
     deal = (deal + U) % WS_NP;
-    mbar_arrive(bars + buf);  // this thread's scores of item k are in place
+    mbar_arrive(bars + BAR_FULL + buf);  // this thread's scores of item k are in place
   }
 }
 
 // ---------------------------------------------------------------------------
-// Consumers: selection, recompute, softmax, P.V and the output of every item.
+// Output of item k by the tensor-core warpgroup (warp 16 + ew reads TMEM lane
+// quarter ew: head dimensions 32 ew + lane, or 16 ew + lane in lanes 0-15 for the
+// M = 64 shape of d = 64). It waits for the item's MMAs, reads the accumulator
+// (columns P_hi rows, then P_lo rows) and the rows' normalisers l, releases the
+// buffer (tfree), then stores O / l as bf16 through a shared-memory tile with
+// 16-byte stores. False when a bounded wait gave up (agreed by all 128 threads).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ bool ws_epilogue(const Problem& p, const ItemInfo& it, uint64_t* bars, int k, uint32_t tbase,
+                                            const float* stats, uint16_t* otile, int ew, int lane) {
+  const int buf = k & 1;
+  const bool ok = mbar_wait(bars + BAR_EMPTY + buf, (k >> 1) & 1);
+  if (named_or(BAR_EPI, 128, !ok)) return false;
+  tc_fence_after();
+  const float* st = stats + buf * WS_BM * 2;
+  const uint32_t ta = tbase + 32 * buf + ((uint32_t)(32 * ew) << 16);
+  float o[WS_BM];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {  // rows 8h .. 8h + 7
+    float hi[8], lo[8];
+    tmem_ld8(ta + 8 * h, hi);
+    tmem_ld8(ta + 16 + 8 * h, lo);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float lv = st[2 * (8 * h + j) + 1];
+      o[8 * h + j] = lv > 0.f ? __fadd_rn(hi[j], lo[j]) * (1.f / lv) : 0.f;
+    }
+  }
+  tc_fence_before();
+  mbar_arrive(bars + BAR_TFREE + buf);  // accumulator, row statistics and row buffer are free
+  const int dim = D == 128 ? 32 * ew + lane : 16 * ew + lane;
+  if (D == 128 || lane < 16) {
+#pragma unroll
+    for (int r = 0; r < WS_BM; ++r) {
+      otile[r * D + dim] = f32_to_bf16_rne(o[r]);
+      if (p.out_f32 && r < it.rows) p.out_f32[((size_t)it.bh * p.n_q + it.i0 + r) * D + dim] = o[r];
+    }
+  }
+  named_sync(BAR_EPI, 128);
+  for (int c = ew * 32 + lane; c < WS_BM * D / 8; c += 128) {
+    const int r = c / (D / 8), c8 = (c % (D / 8)) * 8;
+    if (r < it.rows)
+      *reinterpret_cast<uint4*>(p.out + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8) =
+          *reinterpret_cast<const uint4*>(otile + r * D + c8);
+  }
+  named_sync(BAR_EPI, 128);  // the tile may be refilled
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Consumers: selection, recompute, softmax and the output of every item.
 // ---------------------------------------------------------------------------
 template <int D, int RND, int VAR>
-__device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int cw,
-                                            int lane) {
-  constexpr int NH = D / 64;
-  constexpr int KQ = WS_NC / NH;
-  constexpr int WR = ws_vring<D>();
+__device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int cw, int lane) {
   constexpr int NCT = WS_NC * 32;  // consumer threads
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
@@ -130,59 +222,24 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   const float band = WS_BAND * p.tau;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
-  uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L.v);
-  float* sO = reinterpret_cast<float*>(smem + L.v);
   float* qbase = reinterpret_cast<float*>(smem + L.q);
+  const int rb = sw_bytes(p.n_k);
   long long nsel = 0;
-  // Q of the first two items, then both buffers are released to the producers
-  for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = ws_item(k0, cta, G, a.n_items);
-    if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), tidc, NCT);
-    mbar_arrive(bars + 2 + k0);
-  }
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
     if (q < 0) break;
     const int buf = k & 1;
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
-    const uint16_t* Vh = p.V + (size_t)it.bh * p.n_k * D;
-    // P.V split: warp (kq, nh) takes the 8-key steps kq, kq + KQ, ... of the row and
-    // the value columns nh*64 .. nh*64 + 63. It stages exactly those V rows in a
-    // ring of WR steps of its own (cp.async, one group per step, empty groups past
-    // the end), so the P.V loop needs no group barrier.
-    const int nh = NH == 2 ? (cw & 1) : 0;
-    const int kq = NH == 2 ? (cw >> 1) : cw;
-    const int ns_all = (it.kv_end + 7) >> 3;
-    const int nsw = ns_all > kq ? (ns_all - kq + KQ - 1) / KQ : 0;  // this warp's steps
-    uint16_t* vring = sV + cw * WR * 8 * WS_VSW;
-    auto load_step = [&](int i) {  // step i of this warp into ring slot i % WR
-      if (i < nsw) {
-        const int key0 = 8 * (kq + KQ * i);
-        uint16_t* dst = vring + (i % WR) * 8 * WS_VSW;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c = lane + 32 * h, key = c >> 3, ch = c & 7;
-          uint16_t* dd = dst + key * WS_VSW + ch * 8;
-          if (key0 + key < p.n_k) cp_async16(dd, Vh + (size_t)(key0 + key) * D + nh * 64 + ch * 8);
-          else *reinterpret_cast<uint4*>(dd) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      cp_async_commit();
-    };
-    for (int i = 0; i < WR - 1; ++i) load_step(i);  // V does not depend on the scores
-
-    const bool ok = mbar_wait(bars + buf, (k >> 1) & 1);
+    const bool ok = mbar_wait(bars + BAR_FULL + buf, (k >> 1) & 1);
     if (named_or(BAR_CONS, NCT, !ok)) {
       ws_timeout(p);
-      cp_async_wait<0>();
       return;
     }
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     float* sQ = qbase + buf * ws_qfloats<D>();
-    float* rows = reinterpret_cast<float*>(smem + L.rows) + (size_t)buf * WS_BM * a.nkp;
+    float* rows = reinterpret_cast<float*>(smem + L.rows + buf * rb);
     float* st = reinterpret_cast<float*>(smem + L.stats) + buf * WS_BM * 2;
     const int written = ((it.kv_end + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
 
@@ -191,28 +248,32 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     // comparison selects, so the hot loops need no validity test.
     int rr_[2], nv[2];
     size_t grow[2];
-    float* row[2];
     SelRows S;
+    S.base = rows;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       rr_[t] = 2 * cw + t;
       nv[t] = rr_[t] < it.rows ? ws_valid_keys(it.i0 + rr_[t], p) : 0;
       grow[t] = (size_t)it.bh * p.n_q + it.i0 + rr_[t];
-      row[t] = rows + (size_t)rr_[t] * a.nkp;
-      S.row[t] = row[t];
+      S.rr[t] = rr_[t];
+      S.off[t] = sw_off(rr_[t], lane);
       S.nv[t] = nv[t];
       S.word0[t] = grow[t] * nwords;
       S.live[t] = rr_[t] < it.rows;
       S.mx[t] = -INFINITY;
       S.mrun[t] = -INFINITY;
     }
+    // keys 128 i4 + 4 lane .. + 3 of row rr_[t]: scores at ob[t] + 2048 i4, P_hi at pbo[t] + 2048 i4
+    const int ob[2] = {sw_off(rr_[0], 4 * lane), sw_off(rr_[1], 4 * lane)};
+    const int pbo[2] = {p_off(rr_[0], 4 * lane), p_off(rr_[1], 4 * lane)};
     const int nvmax = max(nv[0], nv[1]);
     const int nit = (nvmax + 127) >> 7;
     if (p.ps_out) {  // dump of the low-precision scores (before any recompute)
 #pragma unroll
       for (int t = 0; t < 2; ++t)
         if (rr_[t] < it.rows)
-          for (int j = lane; j < p.n_k; j += 32) p.ps_out[grow[t] * p.n_k + j] = j < written ? row[t][j] : -INFINITY;
+          for (int j = lane; j < p.n_k; j += 32)
+            p.ps_out[grow[t] * p.n_k + j] = j < written ? rows[sw_off(rr_[t], j)] : -INFINITY;
     }
     if (VAR == LAMP_STRICT) {
       // A: maximum and first argmax of each row
@@ -222,7 +283,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         const int j0 = 128 * i4 + 4 * lane;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          const float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+          const float4 v = lds4_or_ninf(rows + ob[t] + 2048 * i4, j0 < written);
           if (v.x > m[t]) { m[t] = v.x; am[t] = j0; }
           if (v.y > m[t]) { m[t] = v.y; am[t] = j0 + 1; }
           if (v.z > m[t]) { m[t] = v.z; am[t] = j0 + 2; }
@@ -241,7 +302,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         const int j0 = 128 * i4 + 4 * lane;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          float4 v = lds4_or_ninf(row[t] + j0, j0 < written);
+          float4 v = lds4_or_ninf(rows + ob[t] + 2048 * i4, j0 < written);
           if (j0 == (am[t] & ~3)) {  // the argmax itself is not part of S_rest
             const int e = am[t] & 3;
             if (e == 0) v.x = -INFINITY;
@@ -281,7 +342,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     for (int i4 = 0; i4 < nit; ++i4) sel_step<VAR>(p, S, 128 * i4, written, nwords, tlo, thi, lane, wbuf, nsel);
     sel_finish(p, S, wbuf, 4 * nit, nwords, lane, [&](int t, int j) {
       const float v = ws_recompute<D>(sQ, 2 * cw + t, Kh + (size_t)j * D, p.scale, fast);
-      rows[(size_t)(2 * cw + t) * a.nkp + j] = v;
+      rows[sw_off(2 * cw + t, j)] = v;
       if (t == 0) S.mx[0] = fmaxf(S.mx[0], v);
       else S.mx[1] = fmaxf(S.mx[1], v);
     });
@@ -291,11 +352,12 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
       for (int t = 0; t < 2; ++t)
         if (rr_[t] < it.rows)
           for (int j = lane; j < p.n_k; j += 32)
-            p.mixed_out[grow[t] * p.n_k + j] = j < written ? row[t][j] : -INFINITY;
+            p.mixed_out[grow[t] * p.n_k + j] = j < written ? rows[sw_off(rr_[t], j)] : -INFINITY;
     }
 
-    // D: softmax numerators of the mixed rows, in place; the maximum m' of each
-    // mixed row was tracked through the selection and the recompute
+    // D: softmax numerators of the mixed rows, written in place as the bf16 hi and
+    // lo parts of the P.V operand; the maximum m' of each mixed row was tracked
+    // through the selection and the recompute
     const int nitw = (written + 127) >> 7;
     float mm[2], mL[2], l[2] = {0.f, 0.f};
 #pragma unroll
@@ -305,20 +367,29 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     for (int i4 = 0; i4 < nitw; ++i4) {
       const int j0 = 128 * i4 + 4 * lane;
-      if (j0 >= written) continue;
+      const bool act = j0 < written;
+      float4 v[2];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float4 v = *reinterpret_cast<const float4*>(row[t] + j0);
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-        uint32_t pw[4];
+      for (int t = 0; t < 2; ++t) v[t] = act ? *reinterpret_cast<const float4*>(rows + ob[t] + 2048 * i4)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      __syncwarp();  // the 128 keys of both rows are read before any lane overwrites them
+      if (act) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float pj;  // exp(y - m'), 0 for -inf
-          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(pj) : "f"(fmaf(vv[e], kLog2e, -mL[t])));
-          l[t] += pj;
-          pw[e] = p_pair_cvt(pj);
+        for (int t = 0; t < 2; ++t) {
+          const float vv[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+          uint32_t pw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float pj;  // exp(y - m'), 0 for -inf
+            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(pj) : "f"(fmaf(vv[e], kLog2e, -mL[t])));
+            l[t] += pj;
+            pw[e] = p_pair_cvt(pj);  // low half bf16(P), high half bf16(P - bf16(P))
+          }
+          float* dst = rows + pbo[t] + 2048 * i4;
+          *reinterpret_cast<uint2*>(dst) = make_uint2(__byte_perm(pw[0], pw[1], 0x5410), __byte_perm(pw[2], pw[3], 0x5410));
+          *reinterpret_cast<uint2*>(dst + 512) =
+              make_uint2(__byte_perm(pw[0], pw[1], 0x7632), __byte_perm(pw[2], pw[3], 0x7632));
         }
-        *reinterpret_cast<uint4*>(row[t] + j0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
       }
     }
 #pragma unroll
@@ -330,113 +401,197 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         if (p.lse_out && rr_[t] < it.rows) p.lse_out[grow[t]] = nv[t] > 0 ? mm[t] + logf(l[t]) : -INFINITY;
       }
     }
-    named_sync(BAR_CONS, NCT);  // every P row of the item is in place
-
-    // ---- O = (P.V) / l on tensor cores ----------------------------------------------
-    const int mi = lane >> 3;
-    float acc[8][4];
-#pragma unroll
-    for (int tt = 0; tt < 8; ++tt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[tt][e] = 0.f;
-    const int ra = 8 * (mi & 1) + (lane & 7);
-    const int kl = 4 * (mi & 1) + ((lane & 7) >> 1);  // each V row serves the hi and the lo half of P
-    for (int i = 0; i < nsw; ++i) {
-      cp_async_wait<WR - 2>();  // step i has landed (this lane's copies)
-      __syncwarp();             // ... and every lane's; step i - 1's slot is free
-      load_step(i + WR - 1);
-      const int kb = 8 * (kq + KQ * i);
-      const uint16_t* vb = vring + (i % WR) * 8 * WS_VSW;
-      uint32_t af[4];
-      ldmatrix_x4(smem_u32(rows + (size_t)ra * a.nkp + kb + 4 * (mi >> 1)), af[0], af[1], af[2], af[3]);
-#pragma unroll
-      for (int nb = 0; nb < 4; ++nb) {
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(smem_u32(vb + kl * WS_VSW + 16 * nb + 8 * (mi >> 1)), b0, b1, b2, b3);
-        mma_bf16_16816(acc[2 * nb], af[0], af[1], af[2], af[3], b0, b1);
-        mma_bf16_16816(acc[2 * nb + 1], af[0], af[1], af[2], af[3], b2, b3);
-      }
-    }
-    cp_async_wait<0>();
-    named_sync(BAR_CONS, NCT);  // every warp is done with the V stages (the partial sums reuse them)
-    // each warp's partial sums go to a slot of their own; then one pass adds the KQ
-    // slots of every output in a fixed order (deterministic) and scales by 1 / l
-#pragma unroll
-    for (int tt = 0; tt < 8; ++tt)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int rr = (lane >> 2) + 8 * h;
-        *reinterpret_cast<float2*>(sO + ((size_t)kq * WS_BM + rr) * D + nh * 64 + 8 * tt + 2 * (lane & 3)) =
-            make_float2(acc[tt][2 * h], acc[tt][2 * h + 1]);
-      }
-    named_sync(BAR_CONS, NCT);
-    for (int u = tidc; u < WS_BM * D / 2; u += NCT) {
-      const int rr = u / (D / 2), col = (u % (D / 2)) * 2;
-      if (rr >= it.rows) continue;
-      float2 o = *reinterpret_cast<const float2*>(sO + rr * D + col);
-#pragma unroll
-      for (int g = 1; g < KQ; ++g) {
-        const float2 v = *reinterpret_cast<const float2*>(sO + ((size_t)g * WS_BM + rr) * D + col);
-        o.x += v.x;
-        o.y += v.y;
-      }
-      const float lv = st[2 * rr + 1];
-      const float inv = lv > 0.f ? 1.f / lv : 0.f;
-      const float v0 = o.x * inv, v1 = o.y * inv;
-      const size_t off = ((size_t)it.bh * p.n_q + it.i0 + rr) * D + col;
-      *reinterpret_cast<uint32_t*>(p.out + off) =
-          (uint32_t)f32_to_bf16_rne(v0) | ((uint32_t)f32_to_bf16_rne(v1) << 16);
-      if (p.out_f32) *reinterpret_cast<float2*>(p.out_f32 + off) = make_float2(v0, v1);
-    }
-    named_sync(BAR_CONS, NCT);  // the output sums (V area) and this item's Q are no longer read
+    fence_async_smem();  // P (generic-proxy stores) becomes visible to the tensor core
+    named_sync(BAR_CONS, NCT);  // every P row of the item is in place; Q of the item is no longer read
     const int q2 = ws_item(k + 2, cta, G, a.n_items);
     if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
-    mbar_arrive(bars + 2 + buf);  // buffer free (and Q of item k + 2 staged)
+    mbar_arrive(bars + BAR_PREADY + buf);  // P of item k in place, Q of item k + 2 staged
   }
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
 }
 
-template <int D, int RND, int VAR>
-__global__ void __launch_bounds__(WS_NT, 1) ws_kernel(const WsArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const WsSmem L = ws_plan<D>(a.nkp);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-    mbar_init(bars + 0, WS_NP * 32);  // full[0]
-    mbar_init(bars + 1, WS_NP * 32);  // full[1]
-    mbar_init(bars + 2, WS_NC * 32);  // empty[0]
-    mbar_init(bars + 3, WS_NC * 32);  // empty[1]
-    mbar_fence_init();
+// ---------------------------------------------------------------------------
+// Tensor-core warpgroup (warps 16-19, ew = warp - 16). Per item, lane 0 of warp
+// 16 streams the V tiles by TMA and issues P.V by tcgen05.mma, then the four
+// warps run the item's output epilogue.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUtensorMap* tmV, unsigned char* smem,
+                                                    const WsSmem& L, uint32_t tbase, int ew, int lane) {
+  constexpr int S = ws_vslots<D>();
+  constexpr uint32_t TB = ws_vtile_bytes<D>();
+  const Problem& p = a.p;
+  const int G = gridDim.x, cta = blockIdx.x;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  unsigned char* vring = smem + L.v;
+  const uint32_t vbase = smem_u32(vring), rbase = smem_u32(smem + L.rows);
+  const int rb = sw_bytes(p.n_k);
+  const uint32_t idesc = umma_idesc_bf16(D, 32);
+  const bool issuer = ew == 0 && lane == 0;
+  bool ok = true;
+  // V tiles form one sequence over the CTA's items: tile tl of item kl is number gl
+  int kl = 0, tl = 0, Tl = -1, bhl = 0;
+  int gl = 0, gm = 0;  // next tile to load, next tile to multiply
+  auto next_tile = [&]() -> bool {
+    for (;;) {
+      if (Tl < 0) {
+        const int q = ws_item(kl, cta, G, a.n_items);
+        if (q < 0) return false;
+        const ItemInfo it = ws_decode(q, p, a.n_rb);
+        Tl = (it.kv_end + WS_VKEYS - 1) / WS_VKEYS;
+        bhl = it.bh;
+        tl = 0;
+      }
+      if (tl < Tl) return true;
+      ++kl;
+      Tl = -1;
+    }
+  };
+  auto load_upto = [&](int limit) {  // start the loads of tiles gl .. limit - 1
+    while (ok && gl < limit && next_tile()) {
+      const int slot = gl % S;
+      if (gl >= S && !mbar_wait(bars + bar_vempty<D>() + slot, ((gl / S) - 1) & 1)) {  // its MMAs have read it
+        ok = false;
+        break;
+      }
+      mbar_expect_tx(bars + BAR_VFULL + slot, TB);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tma_load_3d(vring + slot * TB + h * 8192, tmV, 64 * h, WS_VKEYS * tl, bhl, bars + BAR_VFULL + slot);
+      ++tl;
+      ++gl;
+    }
+  };
+  // P.V of item k (the issuing thread only)
+  auto mma_item = [&](int k, const ItemInfo& it) {
+    const int buf = k & 1;
+    const int T = (it.kv_end + WS_VKEYS - 1) / WS_VKEYS;
+    load_upto(gm + S);
+    if (!ok || !mbar_wait(bars + BAR_PREADY + buf, (k >> 1) & 1)) {
+      ok = false;
+      return;
+    }
+    tc_fence_after();
+    const uint32_t dcol = tbase + 32 * buf;
+    const uint32_t pb = rbase + buf * rb;
+    for (int t = 0; t < T; ++t, ++gm) {
+      load_upto(gm + S - 1);  // keep the ring full (waits for the MMAs two tiles back)
+      const int slot = gm % S;
+      if (!ok || !mbar_wait(bars + BAR_VFULL + slot, (gm / S) & 1)) {
+        ok = false;
+        return;
+      }
+      tc_fence_after();
+      const uint32_t va = vbase + slot * TB, pa = pb + t * 4096;
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) {  // 16 keys per MMA
+        const uint64_t ad = umma_desc_sw128(va + s4 * 2048, D == 128 ? 8192u : 0u, 1024);
+        const uint64_t bd = umma_desc_sw128(pa + s4 * 32, 16, 1024);
+        umma_bf16(dcol, ad, bd, idesc, (t | s4) != 0);
+      }
+      umma_commit(bars + bar_vempty<D>() + slot);  // V slot free once these MMAs are done
+    }
+    umma_commit(bars + BAR_EMPTY + buf);  // the item's P.V is complete
+  };
+  const float* stats = reinterpret_cast<const float*>(smem + L.stats);
+  uint16_t* otile = reinterpret_cast<uint16_t*>(smem + L.otile);
+  bool good = true;
+  for (int k = 0;; ++k) {
+    const int q = ws_item(k, cta, G, a.n_items);
+    if (q < 0) break;
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    if (issuer && ok) mma_item(k, it);
+    __syncwarp();
+    // a failed issue leaves the item's accumulator incomplete: the epilogue's
+    // bounded wait then gives up, and all four warps agree on it
+    if (!ws_epilogue<D>(p, it, bars, k, tbase, stats, otile, ew, lane)) {
+      good = false;
+      break;
+    }
   }
-  __syncthreads();
-  if (warp < WS_NP) ws_producer<D, RND>(a, smem, L, warp, lane);
-  else ws_consumer<D, RND, VAR>(a, smem, L, warp - WS_NP, lane);
+  if (issuer) {
+    // drain: every MMA issued and every V load in flight completes before the
+    // tensor memory is released and the CTA exits
+    umma_commit(bars + bar_drain<D>());
+    bool drained = mbar_wait(bars + bar_drain<D>(), 0);
+    for (int g = gm; g < gl; ++g) drained = mbar_wait(bars + BAR_VFULL + g % S, (g / S) & 1) && drained;
+    if (!ok || !drained) good = false;
+  }
+  if (!good && lane == 0) ws_timeout(p);
 }
 
 template <int D, int RND, int VAR>
-cudaError_t ws_launch_one(const WsArgs& a, int grid, size_t smem, cudaStream_t st) {
+__global__ void __launch_bounds__(WS_NT, 1) ws_kernel(const WsArgs a, const __grid_constant__ CUtensorMap tmV) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + smem_align1k_pad(smem_raw);
+  const WsSmem L = ws_plan<D>(a.p.n_k);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.tmem);
+  if (threadIdx.x == 0) {
+    mbar_init(bars + BAR_FULL + 0, WS_NP * 32);
+    mbar_init(bars + BAR_FULL + 1, WS_NP * 32);
+    mbar_init(bars + BAR_PREADY + 0, WS_NC * 32);
+    mbar_init(bars + BAR_PREADY + 1, WS_NC * 32);
+    mbar_init(bars + BAR_EMPTY + 0, 1);
+    mbar_init(bars + BAR_EMPTY + 1, 1);
+    mbar_init(bars + BAR_TFREE + 0, 128);
+    mbar_init(bars + BAR_TFREE + 1, 128);
+    for (int i = 0; i < ws_vslots<D>(); ++i) {
+      mbar_init(bars + BAR_VFULL + i, 1);
+      mbar_init(bars + bar_vempty<D>() + i, 1);
+    }
+    mbar_init(bars + bar_drain<D>(), 1);
+    mbar_fence_init();
+  }
+  if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  if (warp < WS_NP) {
+    regs_inc<kWsProdRegs>();
+    ws_producer<D, RND>(a, smem, L, warp, lane);
+  } else if (warp < WS_MW) {
+    regs_inc<kWsConsRegs>();
+    ws_consumer<D, RND, VAR>(a, smem, L, warp - WS_NP, lane);
+  } else {
+    regs_dec<kWsMmaRegs>();
+    ws_tensor_warpgroup<D>(a, &tmV, smem, L, tbase, warp - WS_MW, lane);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WS_MW) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, WS_TMEM_COLS);
+  }
+}
+
+template <int D, int RND, int VAR>
+cudaError_t ws_launch_one(const WsArgs& a, const CUtensorMap& tmV, int grid, size_t smem, cudaStream_t st) {
   auto k = ws_kernel<D, RND, VAR>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k);
   if (e != cudaSuccess) return e;
-  k<<<grid, WS_NT, smem, st>>>(a);
+  if (fa.numRegs != kWsLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split assumes this pool
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, WS_NT, smem, st>>>(a, tmV);
   return cudaGetLastError();
 }
 
 template <int D, int RND>
-cudaError_t ws_launch_var(const WsArgs& a, int grid, size_t smem, cudaStream_t st) {
-  if (a.p.variant == LAMP_RELAXED) return ws_launch_one<D, RND, LAMP_RELAXED>(a, grid, smem, st);
-  if (a.p.variant == LAMP_GIVEN_MASK) return ws_launch_one<D, RND, LAMP_GIVEN_MASK>(a, grid, smem, st);
-  return ws_launch_one<D, RND, LAMP_STRICT>(a, grid, smem, st);
+cudaError_t ws_launch_var(const WsArgs& a, const CUtensorMap& tmV, int grid, size_t smem, cudaStream_t st) {
+  if (a.p.variant == LAMP_RELAXED) return ws_launch_one<D, RND, LAMP_RELAXED>(a, tmV, grid, smem, st);
+  if (a.p.variant == LAMP_GIVEN_MASK) return ws_launch_one<D, RND, LAMP_GIVEN_MASK>(a, tmV, grid, smem, st);
+  return ws_launch_one<D, RND, LAMP_STRICT>(a, tmV, grid, smem, st);
 }
 
 }  // namespace
 
-int ws_nkp(int n_k) { return ((n_k + 127) / 128) * 128 + 4; }
-
-size_t ws_smem_bytes(int d, int n_k) {
-  const int nkp = ws_nkp(n_k);
-  return d == 64 ? (size_t)ws_plan<64>(nkp).total : (size_t)ws_plan<128>(nkp).total;
+size_t ws_smem_bytes(int d, int n_k) {  // dynamic shared memory of a launch (with the 1024-byte alignment slack)
+  return (d == 64 ? (size_t)ws_plan<64>(n_k).total : (size_t)ws_plan<128>(n_k).total) + 1024;
 }
 
 bool ws_fits(int d, int n_k, size_t smem_optin) {
@@ -448,20 +603,22 @@ cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num
   a.p = p;
   a.stats = reinterpret_cast<const int*>(base + ws.stats);
   a.nchunk = ws.nchunk;
-  a.nkp = ws_nkp(p.n_k);
   a.n_rb = (p.n_q + WS_BM - 1) / WS_BM;
   a.n_items = a.n_rb * p.B * p.H;
+  CUtensorMap tmV;
+  cudaError_t e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, true);
+  if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   const size_t smem = ws_smem_bytes(p.d, p.n_k);
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
   if (p.d == 64) {
-    if (rnd == kRndFast) return ws_launch_var<64, kRndFast>(a, grid, smem, st);
-    if (rnd == kRndNone) return ws_launch_var<64, kRndNone>(a, grid, smem, st);
-    return ws_launch_var<64, kRndExact>(a, grid, smem, st);
+    if (rnd == kRndFast) return ws_launch_var<64, kRndFast>(a, tmV, grid, smem, st);
+    if (rnd == kRndNone) return ws_launch_var<64, kRndNone>(a, tmV, grid, smem, st);
+    return ws_launch_var<64, kRndExact>(a, tmV, grid, smem, st);
   }
-  if (rnd == kRndFast) return ws_launch_var<128, kRndFast>(a, grid, smem, st);
-  if (rnd == kRndNone) return ws_launch_var<128, kRndNone>(a, grid, smem, st);
-  return ws_launch_var<128, kRndExact>(a, grid, smem, st);
+  if (rnd == kRndFast) return ws_launch_var<128, kRndFast>(a, tmV, grid, smem, st);
+  if (rnd == kRndNone) return ws_launch_var<128, kRndNone>(a, tmV, grid, smem, st);
+  return ws_launch_var<128, kRndExact>(a, tmV, grid, smem, st);
 }
 
 }  // namespace lamp

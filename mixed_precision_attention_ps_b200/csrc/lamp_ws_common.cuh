@@ -1,6 +1,6 @@
 // Device pieces shared by the warp-specialised LAMP kernels (whole-row and
-// streamed): work order, Q staging, the producer's score tile and the FP32
-// recompute. Method: "LAMP: Look-Ahead Mixed-Precision Inference of Large
+// streamed): work order, Q staging, the layout of the score rows in shared
+// memory, the producer's score tile and the FP32 recompute. Method: "LAMP: Look-Ahead Mixed-Precision Inference of Large
 // Language Models" (technical summary, gist.science paper 2601.21623), sections
 // "Implementation strategy" (steps 1 and 3) and "Experimental results" (PS(mu)).
 #pragma once
@@ -8,25 +8,63 @@
 #include "lamp.h"
 #include "lamp_device.cuh"
 #include "lamp_kernels.h"
+#include "lamp_umma.cuh"
 
 namespace lamp {
 namespace {
 
 constexpr int WS_BM = 16;              // query rows per item
-constexpr int WS_NT = kWsThreads;      // 512
+constexpr int WS_NT = kWsThreads;      // 640
 constexpr int WS_NP = 8;               // producer warps
 constexpr int WS_NC = 8;               // consumer warps
+constexpr int WS_MW = WS_NP + WS_NC;   // the tensor-core warp (V tiles by TMA, P.V by tcgen05.mma), first of its warpgroup
 constexpr int WS_UNIT = 64;            // keys per producer unit
 constexpr int WS_DS = 8;               // head dimensions per K slice
 constexpr float WS_BAND = 8e-6f;       // relative band around tau re-evaluated in double
 constexpr int BAR_CONS = 1;            // named barrier of the consumer group
-constexpr int WS_VSW = 72;             // row stride (bf16) of a consumer warp's V ring: 64 columns + pad
-template <int D>
-__host__ __device__ constexpr int ws_vring() { return D == 64 ? 6 : 4; }  // V steps in a consumer warp's ring
+constexpr int WS_VKEYS = 64;           // keys per V tile (one TMA box of 64 keys x 64 dimensions per half)
+constexpr int WS_TMEM_COLS = 64;       // two P.V accumulators of N = 32 columns (P_hi rows, P_lo rows)
+// Per-warpgroup register budgets (setmaxnreg; every warp of a warpgroup executes
+// the same one).
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
 // Q of an item in shared memory: [D][16 rows] f32 (dimension-major, so a 16-byte
 // load gives four rows of one dimension: the packed pairs of two row pairs)
 template <int D>
 __host__ __device__ constexpr int ws_qfloats() { return D * WS_BM; }
+
+// ---------------------------------------------------------------------------
+// Score rows of an item (16 query rows) in shared memory: blocks of 64 keys, 4096
+// bytes each, laid out so that the softmax numerators can be written in place as
+// the B operand of the P.V tensor-core product (K-major, 128-byte swizzle; see
+// lamp_umma.cuh):
+//   block b = j / 64 at 4096 b; half h = (j / 32) % 2 at 2048 h holds the fp32
+//   scores of keys 32h .. 32h + 31 of the block; row r is the 128-byte line at
+//   1024 (r / 8) + 128 (r % 8) of the half, and its 16-byte chunk c = (j % 32) / 4
+//   sits at position c ^ (r % 8).
+// After the softmax pass the same two lines of row r hold the block's 64 P_hi
+// values (half 0) and P_lo values (half 1) as bf16, chunk (j % 64) / 8 at position
+// ((j % 64) / 8) ^ (r % 8): a row's P overwrites only that row's own scores. A
+// warp reading one row touches 32 consecutive keys per 128-byte line (no bank
+// conflicts), and 4 consecutive keys are one 16-byte chunk.
+// ---------------------------------------------------------------------------
+constexpr int SW_BLOCK_FLOATS = 1024;  // one 64-key block of 16 rows
+
+// Float index of score (r, j).
+__device__ __forceinline__ int sw_off(int r, int j) {
+  return ((j >> 6) << 10) | (((j >> 5) & 1) << 9) | ((r >> 3) << 8) | ((r & 7) << 5) |
+         ((((j >> 2) & 7) ^ (r & 7)) << 2) | (j & 3);
+}
+// Float index of the 8 bytes that hold P_hi of keys j .. j + 3 (j a multiple of
+// 4) of row r; P_lo follows at + 512 floats (2048 bytes).
+__device__ __forceinline__ int p_off(int r, int j) {
+  return ((j >> 6) << 10) | ((r >> 3) << 8) | ((r & 7) << 5) | ((((j >> 3) & 7) ^ (r & 7)) << 2) | ((j & 4) >> 1);
+}
+// Bytes of the score rows of an item with n keys.
+__host__ __device__ constexpr int sw_bytes(int n) { return ((n + 63) / 64) * 4096; }
 
 // The k-th item of CTA b (snake order over heaviest-first items), or -1.
 __device__ __forceinline__ int ws_item(int k, int b, int G, int n_items) {
@@ -59,10 +97,12 @@ __device__ __forceinline__ void ws_timeout(const Problem& p) {
 }
 
 // Q rows of an item as binary32 [D][16] (rows past the problem are zero).
+// Thread u takes row u % 16 of the 8-dimension group u / 16, so that the 16
+// lanes of a half-warp write 16 consecutive floats of each dimension.
 template <int D>
 __device__ __forceinline__ void ws_stage_q(float* sQ, const Problem& p, const ItemInfo& it, int t, int nthreads) {
   for (int u = t; u < WS_BM * D / 8; u += nthreads) {
-    const int r = u / (D / 8), c8 = (u % (D / 8)) * 8;
+    const int r = u % WS_BM, c8 = (u / WS_BM) * 8;
     uint4 w = make_uint4(0u, 0u, 0u, 0u);
     if (r < it.rows) w = __ldg(reinterpret_cast<const uint4*>(p.Q + ((size_t)it.bh * p.n_q + it.i0 + r) * D + c8));
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -95,101 +135,184 @@ __device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, con
   }
 }
 
+// K staging of a producer warp.
+//   KT = 0: K slices travel global -> registers -> shared memory (binary32) two
+//           stream positions ahead of their use, so an L2 round trip hides behind
+//           two slices of arithmetic.
+//   KT = 1: a TMA load brings each bf16 slice (64 keys x 8 dimensions, 1 KB) into a
+//           ring of KRING stages of the warp, completing on the stage's mbarrier,
+//           three positions ahead; the warp widens the landed slice to binary32
+//           into the slice buffer one position ahead of its use.
+constexpr int KRING = 3;
+struct KTma {
+  const CUtensorMap* map;  // K as [B*H][n_k][d] bf16, box {8 dims, 64 keys, 1}
+  uint16_t* ring;          // this warp's KRING stages of [64 keys][8 dims] bf16 (1024-byte aligned)
+  uint64_t* bar;           // this warp's KRING mbarriers (one arrival + 1024 bytes each)
+  uint32_t* count;         // slices this warp has loaded so far (stage = n % KRING, phase = n / KRING)
+};
+
 // Scores of one tile of an item, keys t0 .. t0 + tlen - 1, by one producer warp:
 // the tile's 64-key units j = first, first + 8, ... (the others belong to the other
-// producer warps). Unit j's scores go to rows[r * stride + 64 j + c] for the 16
-// rows r of the item; keys past a row's valid range hold -inf.
-template <int D, int RND>
-__device__ __forceinline__ void ws_produce_tile(const Problem& p, const ItemInfo& it, int t0, int tlen,
-                                                const float* sQ, float* rows, int stride, float* ksw, int lane,
-                                                int first, bool fast, const uint16_t* Kh, u64 negc, u64 pow2s,
-                                                u64 scale2, int s) {
+// producer warps). The scores of key t0 + c go to rows[sw_off(r, c)] for the 16
+// rows r of the item (the block layout above); keys past a row's valid range hold
+// -inf.
+// The buffer may still be read by the tensor core when the call starts: the
+// warp waits for free_bar's phase free_phase (when free_bar is not null) only
+// before its first store, one unit of arithmetic later. Returns false when a
+// bounded wait gave up (the warp's copies in flight have then landed).
+template <int D, int RND, int KT>
+__device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo& it, int t0, int tlen,
+                                                const float* sQ, float* rows, float* ksw, int lane, int first,
+                                                bool fast, const uint16_t* Kh, u64 negc, u64 pow2s, u64 scale2,
+                                                int s, const KTma& kt, uint64_t* free_bar, uint32_t free_phase) {
   constexpr int NSL = D / WS_DS;  // K slices per unit
   const int gr = lane & 1, gk = lane >> 1;  // rows 8gr..8gr+7, keys 4gk..4gk+3 of a unit
   const int qoff = 8 * gr, koff = 4 * gk;
   const int U = (tlen + WS_UNIT - 1) / WS_UNIT;
   const int mine = first < U ? (U - first + WS_NP - 1) / WS_NP : 0;
   const int total = mine * NSL;
-    // K slices travel global -> registers -> shared two stream positions ahead of
-    // their use, so an L2 round trip hides behind two slices of arithmetic.
-    uint4 kra[2], krb[2];
-    auto load = [&](int pos, uint4 (&kr)[2]) {  // keys lane and lane + 32 of the slice at pos
+  uint4 kra[2], krb[2];
+  auto load = [&](int pos, uint4 (&kr)[2]) {  // KT 0: keys lane and lane + 32 of the slice at pos
+    const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int key = t0 + j * WS_UNIT + lane + 32 * h;
+      kr[h] = make_uint4(0u, 0u, 0u, 0u);
+      if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
+    }
+  };
+  auto issue = [&](int pos) {  // KT 1: TMA of the slice at pos into its ring stage
+    if (lane == 0) {
+      const uint32_t n = *kt.count + pos;
       const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
+      fence_async_smem();  // the stage's earlier reads (generic proxy) precede the copy
+      mbar_expect_tx(kt.bar + n % KRING, WS_UNIT * WS_DS * 2);
+      tma_load_3d(kt.ring + (n % KRING) * WS_UNIT * WS_DS, kt.map, sl * WS_DS, t0 + j * WS_UNIT, it.bh,
+                  kt.bar + n % KRING);
+    }
+  };
+  auto widen = [&](int b2, const uint4 (&kr)[2]) {  // binary32 [8 dims][64 keys] into slice buffer b2
+    float* dst = ksw + b2 * WS_DS * WS_UNIT + lane;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int key = t0 + j * WS_UNIT + lane + 32 * h;
-        kr[h] = make_uint4(0u, 0u, 0u, 0u);
-        if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t ws[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dst[(2 * e) * WS_UNIT + 32 * h] = bf16_lo(ws[e]);
+        dst[(2 * e + 1) * WS_UNIT + 32 * h] = bf16_hi(ws[e]);
       }
-    };
-    auto store = [&](int b2, const uint4 (&kr)[2]) {
-      float* dst = ksw + b2 * WS_DS * WS_UNIT + lane;
+    }
+  };
+  bool failed = false;
+  int fpos = 0;  // the stream position during which a wait gave up
+  auto landed = [&](int pos, uint4 (&kr)[2]) -> bool {  // KT 1: the slice at pos from its ring stage
+    const uint32_t n = *kt.count + pos;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(kt.bar + n % KRING, (n / KRING) & 1))) return false;
+    const uint16_t* src = kt.ring + (n % KRING) * WS_UNIT * WS_DS;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t ws[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w};
+    for (int h = 0; h < 2; ++h) kr[h] = *reinterpret_cast<const uint4*>(src + (lane + 32 * h) * WS_DS);
+    return true;
+  };
+  u64 acc[4][4];
+  // one stream position: compute slice pos, then stage slice pos + 1 into the free
+  // binary32 buffer and start the load of slice pos + 3 (KT 0: into `cur`, the
+  // register set of pos + 1, two sets alternating; KT 1: into the ring stage pos
+  // has released)
+  auto body = [&](int pos, uint4 (&cur)[2]) {
+    const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
+    if (sl == 0) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          dst[(2 * e) * WS_UNIT + 32 * h] = bf16_lo(ws[e]);
-          dst[(2 * e + 1) * WS_UNIT + 32 * h] = bf16_hi(ws[e]);
+      for (int rp = 0; rp < 4; ++rp)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[rp][i] = 0ull;
+    }
+    const float* qs = sQ + sl * WS_DS * WS_BM;
+    const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
+    if (RND == kRndFast && fast) ws_score_slice<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+    else if (RND == kRndNone && fast) ws_score_slice<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+    else ws_score_slice<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+    if (sl == NSL - 1) {
+      if (free_bar) {  // first store of the call: the buffer's previous contents are no longer read
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(free_bar, free_phase))) {
+          failed = true;
+          fpos = pos;
+          return;
         }
+        free_bar = nullptr;
       }
-    };
-    u64 acc[4][4];
-    // one stream position: compute slice pos, move the slice held in `cur` (loaded
-    // two positions ago) into the free shared buffer, then reuse `cur` for the load
-    // of position pos + 3; two register sets alternate, so no load is waited on early
-    auto body = [&](int pos, uint4 (&cur)[2]) {
-      const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
-      if (sl == 0) {
+      const int c0 = j * WS_UNIT + koff;  // lane's first column, relative to the tile
+      const int j0 = t0 + c0;             // ... and as an absolute key
 #pragma unroll
-        for (int rp = 0; rp < 4; ++rp)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[rp][i] = 0ull;
+      for (int rp = 0; rp < 4; ++rp) {
+        const int r0 = 8 * gr + 2 * rp;
+        const int nv0 = r0 < it.rows ? ws_valid_keys(it.i0 + r0, p) : 0;
+        const int nv1 = r0 + 1 < it.rows ? ws_valid_keys(it.i0 + r0 + 1, p) : 0;
+        float4 y0, y1;
+        const u64 a0 = mul2u(acc[rp][0], scale2), a1 = mul2u(acc[rp][1], scale2);
+        const u64 a2 = mul2u(acc[rp][2], scale2), a3 = mul2u(acc[rp][3], scale2);
+        y0.x = j0 < nv0 ? lo_f(a0) : -INFINITY;
+        y0.y = j0 + 1 < nv0 ? lo_f(a1) : -INFINITY;
+        y0.z = j0 + 2 < nv0 ? lo_f(a2) : -INFINITY;
+        y0.w = j0 + 3 < nv0 ? lo_f(a3) : -INFINITY;
+        y1.x = j0 < nv1 ? hi_f(a0) : -INFINITY;
+        y1.y = j0 + 1 < nv1 ? hi_f(a1) : -INFINITY;
+        y1.z = j0 + 2 < nv1 ? hi_f(a2) : -INFINITY;
+        y1.w = j0 + 3 < nv1 ? hi_f(a3) : -INFINITY;
+        *reinterpret_cast<float4*>(rows + sw_off(r0, c0)) = y0;
+        *reinterpret_cast<float4*>(rows + sw_off(r0 + 1, c0)) = y1;
       }
-      const float* qs = sQ + sl * WS_DS * WS_BM;
-      const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
-      if (RND == kRndFast && fast) ws_score_slice<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      else if (RND == kRndNone && fast) ws_score_slice<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      else ws_score_slice<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-      if (sl == NSL - 1) {
-        const int j0 = t0 + j * WS_UNIT + koff;  // absolute key of the lane's first column
-        float* dst = rows + j * WS_UNIT + koff;
-#pragma unroll
-        for (int rp = 0; rp < 4; ++rp) {
-          const int r0 = 8 * gr + 2 * rp;
-          const int nv0 = r0 < it.rows ? ws_valid_keys(it.i0 + r0, p) : 0;
-          const int nv1 = r0 + 1 < it.rows ? ws_valid_keys(it.i0 + r0 + 1, p) : 0;
-          float4 y0, y1;
-          const u64 a0 = mul2u(acc[rp][0], scale2), a1 = mul2u(acc[rp][1], scale2);
-          const u64 a2 = mul2u(acc[rp][2], scale2), a3 = mul2u(acc[rp][3], scale2);
-          y0.x = j0 < nv0 ? lo_f(a0) : -INFINITY;
-          y0.y = j0 + 1 < nv0 ? lo_f(a1) : -INFINITY;
-          y0.z = j0 + 2 < nv0 ? lo_f(a2) : -INFINITY;
-          y0.w = j0 + 3 < nv0 ? lo_f(a3) : -INFINITY;
-          y1.x = j0 < nv1 ? hi_f(a0) : -INFINITY;
-          y1.y = j0 + 1 < nv1 ? hi_f(a1) : -INFINITY;
-          y1.z = j0 + 2 < nv1 ? hi_f(a2) : -INFINITY;
-          y1.w = j0 + 3 < nv1 ? hi_f(a3) : -INFINITY;
-          *reinterpret_cast<float4*>(dst + (size_t)r0 * stride) = y0;
-          *reinterpret_cast<float4*>(dst + (size_t)(r0 + 1) * stride) = y1;
-        }
-      }
-      __syncwarp();  // every lane is done reading slice pos - 1's buffer
-      if (pos + 1 < total) store((pos + 1) & 1, cur);
+    }
+    __syncwarp();  // every lane is done reading slice pos - 1's buffer
+    if (KT == 0) {
+      if (pos + 1 < total) widen((pos + 1) & 1, cur);
       if (pos + 3 < total) load(pos + 3, cur);
-      __syncwarp();
-    };
+    } else {
+      if (pos + 1 < total) {
+        if (!landed(pos + 1, cur)) {
+          failed = true;
+          fpos = pos;
+          return;
+        }
+        widen((pos + 1) & 1, cur);
+      }
+      __syncwarp();  // every lane has read the stage of pos + 1 (and of pos, before)
+      if (pos + 3 < total) issue(pos + 3);
+    }
+    __syncwarp();
+  };
+  if (KT == 0) {
     if (total > 0) {
       load(0, kra);
-      store(0, kra);
+      widen(0, kra);
     }
     if (total > 1) load(1, kra);
     if (total > 2) load(2, krb);
-    __syncwarp();
-    for (int pos = 0; pos < total; pos += 2) {
-      body(pos, kra);
-      if (pos + 1 < total) body(pos + 1, krb);
+  } else {
+    for (int i = 0; i < 3 && i < total; ++i) issue(i);
+    if (total > 0) {
+      if (landed(0, kra)) {
+        widen(0, kra);
+      } else {
+        failed = true;
+        fpos = -1;
+      }
     }
+  }
+  __syncwarp();
+  for (int pos = 0; pos < total && !failed; pos += 2) {
+    body(pos, kra);
+    if (pos + 1 < total && !failed) body(pos + 1, krb);
+  }
+  if (KT == 1) {
+    if (failed) {  // the slices requested but not yet landed must land before the warp gives up
+      for (int q = fpos + 1; q <= fpos + 2 && q < total; ++q) {
+        const uint32_t n = *kt.count + q;
+        mbar_wait(kt.bar + n % KRING, (n / KRING) & 1);
+      }
+    }
+    *kt.count += total;
+  }
+  return !failed;  // (a warp with no unit of its own writes nothing and so needs no wait)
 }
 
 // FP32 recompute of score (row r, key j): the sequential binary32 sum over
@@ -233,7 +356,9 @@ __device__ __forceinline__ float4 lds4_or_ninf(const float* ptr, bool ok) {
 constexpr int SEL_WMAX = 32;  // mask words per row a pass holds (1024 keys)
 
 struct SelRows {
-  float* row[2];     // the two score rows (key j of the pass at row[t][j])
+  float* base;       // the item's score rows (block layout, sw_off)
+  int rr[2];         // the warp's two rows (key j of the pass at base[sw_off(rr[t], j)])
+  int off[2];        // sw_off(rr[t], lane): key kb + 32 m + lane (kb a multiple of 128) is at off + 16 kb + 512 m
   int nv[2];         // valid keys of each row, counted from the pass's key 0
   size_t word0[2];   // mask word of the pass's key 0 in mask_out / mask_in
   bool live[2];      // the row exists (only live rows write mask words)
@@ -258,7 +383,7 @@ __device__ __forceinline__ void sel_step(const Problem& p, SelRows& S, int kb, i
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) y[t][m] = kb + 32 * m < written ? S.row[t][kb + 32 * m + lane] : -INFINITY;
+    for (int m = 0; m < 4; ++m) y[t][m] = kb + 32 * m < written ? S.base[S.off[t] + 16 * kb + 512 * m] : -INFINITY;
     if (VAR == LAMP_GIVEN_MASK) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
