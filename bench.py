@@ -84,12 +84,14 @@ DEFAULTS = {  # workload -> (variant, rate)
 
 
 def lookup_tau(workload: str, variant: int, mu: int, rate: float | None) -> tuple[float, float | None]:
+    """The calibrated tau as the binary32 value the C ABI receives (the value the
+    GPU parity tests pass to both the kernels and the oracle)."""
     if workload == "single_head_128" and rate is None:
-        return 0.05, None
+        return float(np.float32(0.05)), None
     doc = json.load(open(TAU_FILE))
     for e in doc["entries"]:
         if e["workload"] == workload and e["variant"] == variant and e["mu"] == mu and abs(e["rate"] - rate) < 1e-12:
-            return float(e["tau"]), float(e["rate"])
+            return float(np.float32(e["tau"])), float(e["rate"])
     raise SystemExit(f"no tau for {workload} variant={variant} mu={mu} rate={rate} in {TAU_FILE}")
 
 

@@ -151,7 +151,15 @@ typedef struct {
   int *status_out;             /* device status word, may be NULL: set to LAMP_ERR_TIMEOUT when
                                   a bounded wait inside a kernel gave up (the outputs of the
                                   call are then undefined); never cleared by the library */
+  int debug_stall;             /* 0 in normal use. LAMP_DEBUG_STALL_PRODUCERS (tests of the
+                                  failure path only): in the whole-row kernel the score
+                                  producers hand over nothing, so every other warp's bounded
+                                  wait (about 2 s) runs out; the kernel then writes
+                                  LAMP_ERR_TIMEOUT to status_out and returns, its outputs
+                                  undefined. Other kernels ignore the field. */
 } lamp_args;
+
+#define LAMP_DEBUG_STALL_PRODUCERS 1
 
 LAMP_API int lamp_attention_ex(const lamp_args *args);
 
@@ -165,10 +173,14 @@ LAMP_API int lamp_attention_ex(const lamp_args *args);
  *              workspace_bytes 0 (LAMP_ERR_ARG otherwise).
  *   scratch    a fixed array of LAMP_NOALLOC_SCRATCH_BYTES in the memory of every
  *              GPU that loads the library, held until the process exits. A problem
- *              that needs more (strict rows too long for shared memory) is rejected
- *              with LAMP_ERR_WORKSPACE before anything is launched.
+ *              is rejected with LAMP_ERR_WORKSPACE before anything is launched when
+ *              lamp_workspace_size() for it exceeds LAMP_NOALLOC_SCRATCH_BYTES; the
+ *              usual causes are the score slab of strict rows longer than the
+ *              whole-row kernel takes (B*H*n_q*ceil(n_k/512)*512*4 bytes) and the
+ *              per-chunk partials of long decode rows.
  *   first call on a device: looks up the device address of that array (no
- *              allocation); make it before capturing a stream into a graph.
+ *              allocation; a failed lookup is retried by the next call); make it
+ *              before capturing a stream into a graph.
  *   sharing    every call on a device uses the same array, and keeps nothing in it
  *              from one call to the next (the call clears what must start at zero).
  *              Calls whose kernels overlap on the GPU (work on two streams without

@@ -15,7 +15,7 @@ from __future__ import annotations
 from dataclasses import dataclass
 
 from ._native import (LAMP_ERR_ARG, LAMP_ERR_CHECK, LAMP_ERR_CUDA, LAMP_ERR_TIMEOUT,  # noqa: F401
-                      LAMP_ERR_UNSUPPORTED, LAMP_ERR_WORKSPACE, LAMP_GIVEN_MASK, LAMP_MAX_SCORE_SLAB_BYTES,
+                      LAMP_DEBUG_STALL_PRODUCERS, LAMP_ERR_UNSUPPORTED, LAMP_ERR_WORKSPACE, LAMP_GIVEN_MASK, LAMP_MAX_SCORE_SLAB_BYTES,
                       LAMP_NOALLOC_SCRATCH_BYTES, LAMP_OK, LAMP_RELAXED, LAMP_STRICT, LampError, lamp_args,
                       lamp_args_size, lamp_attention, lamp_attention_ex, lamp_attention_noalloc, lamp_dims,
                       lamp_gelu_args, lamp_gelu_args_size, lamp_last_error, lamp_linear_gelu,

@@ -25,6 +25,7 @@ LAMP_ERR_TIMEOUT = -5
 LAMP_ERR_CHECK = -6
 LAMP_MAX_SCORE_SLAB_BYTES = 64 << 30
 LAMP_NOALLOC_SCRATCH_BYTES = 4 << 20
+LAMP_DEBUG_STALL_PRODUCERS = 1
 
 STATUS_NAMES = {
     LAMP_OK: "LAMP_OK", LAMP_ERR_ARG: "LAMP_ERR_ARG", LAMP_ERR_UNSUPPORTED: "LAMP_ERR_UNSUPPORTED",
@@ -70,6 +71,7 @@ class lamp_args(ctypes.Structure):
         ("workspace", _P),
         ("workspace_bytes", ctypes.c_size_t),
         ("status_out", _P),
+        ("debug_stall", ctypes.c_int),
     ]
 
 
@@ -211,11 +213,12 @@ def lamp_attention(dims, Q, K, V, out, mask_out, mu: int, tau: float, variant: i
 def make_args(dims, Q, K, V, out, *, mask_out=None, mu=4, tau=0.0, variant=LAMP_STRICT, causal=1,
               stream=None, scale=0.0, mask_in=None, out_f32=None, ps_scores_out=None,
               mixed_scores_out=None, lse_out=None, n_selected_out=None, workspace=None,
-              workspace_bytes=0, status_out=None) -> lamp_args:
+              workspace_bytes=0, status_out=None, debug_stall=0) -> lamp_args:
     return lamp_args(lamp_dims(*dims), _ptr(Q), _ptr(K), _ptr(V), _ptr(out), _ptr(mask_out), int(mu),
                      float(tau), int(variant), int(causal), _stream(stream), float(scale), _ptr(mask_in),
                      _ptr(out_f32), _ptr(ps_scores_out), _ptr(mixed_scores_out), _ptr(lse_out),
-                     _ptr(n_selected_out), _ptr(workspace), int(workspace_bytes), _ptr(status_out))
+                     _ptr(n_selected_out), _ptr(workspace), int(workspace_bytes), _ptr(status_out),
+                     int(debug_stall))
 
 
 def lamp_attention_ex(args: lamp_args | None = None, check: bool = True, **kw) -> int:

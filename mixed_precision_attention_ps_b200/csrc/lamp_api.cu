@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "lamp.h"
@@ -107,6 +108,8 @@ int check_args(const lamp_args* a) {
   if (a->causal != 0 && a->causal != 1) return fail(LAMP_ERR_ARG, "causal must be 0 or 1");
   if (std::isnan(a->scale) || a->scale < 0.f || std::isinf(a->scale))
     return fail(LAMP_ERR_ARG, "scale must be 0 (default) or a positive finite value");
+  if (a->debug_stall != 0 && a->debug_stall != LAMP_DEBUG_STALL_PRODUCERS)
+    return fail(LAMP_ERR_ARG, "debug_stall must be 0 or LAMP_DEBUG_STALL_PRODUCERS");
   if (d.d != 64 && d.d != 128) return fail(LAMP_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d.d);
   const long long rows = (long long)d.B * d.H * d.n_q;
   if ((long long)d.B * d.H > 65535 || rows > (1LL << 40))
@@ -141,6 +144,7 @@ lamp::Problem make_problem(const lamp_args* a) {
   p.lse_out = a->lse_out;
   p.nsel_out = a->n_selected_out;
   p.status_out = a->status_out;
+  p.debug_stall = a->debug_stall;
   p.emax_sum_limit = emax_sum_limit(a->mu, a->dims.d);
   return p;
 }
@@ -164,20 +168,28 @@ cudaError_t run_kernels(const lamp::Problem& p, const lamp::Workspace& ws, char*
 // the name stands for a host-side shadow, not for a device address: kernels get
 // the address that cudaGetSymbolAddress returns for the current device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LAMP_NOALLOC_SCRATCH_BYTES];
-char* g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
+std::atomic<char*> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on device dev (the current device),
-// looked up on the first call for that device.
+// Device address of the scratch array on device dev (the current device). Only a
+// successful lookup is kept: a failed one (for instance while another thread
+// holds a stream capture open) is retried on the next call, and its error is
+// cleared from the runtime's last-error state.
 cudaError_t noalloc_scratch(int dev, char*& ptr) {
-  std::call_once(g_noalloc_once[dev], [&]() {
-    void* addr = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
-    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? static_cast<char*>(addr) : nullptr;
-  });
-  ptr = g_noalloc_ptr[dev];
-  return g_noalloc_err[dev];
+  ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (ptr) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  ptr = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+  if (ptr) return cudaSuccess;
+  void* addr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+  if (e != cudaSuccess || !addr) {
+    (void)cudaGetLastError();
+    return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+  }
+  ptr = static_cast<char*>(addr);
+  g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -37,6 +37,7 @@ struct Problem {
   float* lse_out;
   unsigned long long* nsel_out;
   int* status_out;       // optional device status word (LAMP_ERR_TIMEOUT on a bounded wait that gave up)
+  int debug_stall;       // LAMP_DEBUG_STALL_PRODUCERS: the whole-row producers hand over nothing (failure-path tests)
   int emax_sum_limit;  // largest e_q + e_k for which the fast score path is exact
 };
 

@@ -117,6 +117,8 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
   float* qbase = reinterpret_cast<float*>(smem + L.q);
   const int rb = sw_bytes(p.n_k);
+  // failure-path tests: hand over nothing, so that every other warp's bounded wait runs out
+  if (p.debug_stall == LAMP_DEBUG_STALL_PRODUCERS) return;
   // Q of the first two items (the consumers stage the later ones)
   for (int k0 = 0; k0 < 2; ++k0) {
     const int q0 = ws_item(k0, cta, G, a.n_items);

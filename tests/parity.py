@@ -26,6 +26,10 @@ KL_TOL = 1e-6
 TIE_REL = 1e-6
 TIE_FRAC = 1e-5
 
+# (label, near-tie mask differences, valid entries compared) of the calibrated-tau
+# cases, summarised at the end of the test session (tests/conftest.py)
+TIE_LOG: list = []
+
 
 def to_device(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)

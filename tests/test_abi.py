@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_struct_layout_matches(lib):
-    assert lamp.lamp_args_size() == ctypes.sizeof(_native.lamp_args) == 168
+    assert lamp.lamp_args_size() == ctypes.sizeof(_native.lamp_args) == 176
     assert lamp.lamp_gelu_args_size() == ctypes.sizeof(_native.lamp_gelu_args) == 112
     assert lamp.lamp_ln_args_size() == ctypes.sizeof(_native.lamp_ln_args) == 136
     assert lamp.lamp_version().startswith("lamp-b200")
@@ -70,6 +70,7 @@ def call_ex(**kw):
     (dict(Q=FAKE + 8), lamp.LAMP_ERR_UNSUPPORTED, "16-byte"),
     (dict(out_f32=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
     (dict(n_selected_out=FAKE + 4), lamp.LAMP_ERR_UNSUPPORTED, "aligned"),
+    (dict(debug_stall=7), lamp.LAMP_ERR_ARG, "debug_stall"),
 ])
 def test_argument_checks(lib, kw, code, msg):
     rc = call_ex(**kw)
