@@ -17,9 +17,7 @@
 // 640 threads per SM, items (b, h, 16 query rows) in a snake order, two tile
 // buffers in the block layout of lamp_ws_common.cuh.
 //   producers (warps 0-7): 64-key units dealt round-robin, PS(mu) steps as packed
-//     binary32 pairs; each warp's K slices arrive by TMA (bf16, 64 keys x 8
-//     dimensions) in a ring of three stages and are widened on the way to the
-//     binary32 slice buffer.
+//     binary32 pairs, K slices staged through registers as binary32.
 //   consumers (warps 8-15): per tile the criterion (double re-evaluation near
 //     tau), mask words, warp-compacted FP32 recompute, then the online softmax
 //     (running maximum m and normaliser l per row, rescale factor
@@ -55,16 +53,13 @@ __host__ __device__ constexpr int sb_vempty() { return SB_VFULL + st_vslots<D>()
 template <int D>
 __host__ __device__ constexpr int sb_drain() { return SB_VFULL + 2 * st_vslots<D>(); }
 template <int D>
-__host__ __device__ constexpr int sb_kring() { return sb_drain<D>() + 1; }  // [8 warps][KRING]
-template <int D>
-__host__ __device__ constexpr int sb_count() { return sb_kring<D>() + WS_NP * KRING; }
+__host__ __device__ constexpr int sb_count() { return sb_drain<D>() + 1; }
 constexpr int BAR_PROD = 2;  // named barrier of the producer group
 constexpr int BAR_EPI = 3;   // named barrier of the tensor-core warpgroup (output epilogue)
 
 struct StSmem {  // byte offsets from a 1024-byte aligned base
   int tiles;  // score tiles [2][sw_bytes(512)] (block layout)
   int v;      // V ring [S][D / 64][64 keys][64 dims] bf16 (128-byte swizzle)
-  int kring;  // producer K stages [8 warps][KRING][64 keys][8 dims] bf16
   int ks;     // producer K slices [8 warps][2][8][64] f32
   int q;      // Q [2][D][16] f32, by item parity
   int list;   // consumer mask-word buffers [8][2][32] uint32
@@ -80,8 +75,7 @@ __host__ __device__ inline StSmem st_plan() {
   StSmem s{};
   s.tiles = 0;
   s.v = 2 * sw_bytes(ST_T);
-  s.kring = s.v + st_vslots<D>() * st_vtile_bytes<D>();
-  s.ks = s.kring + WS_NP * KRING * WS_UNIT * WS_DS * 2;
+  s.ks = s.v + st_vslots<D>() * st_vtile_bytes<D>();
   s.q = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
   s.list = s.q + 2 * ws_qfloats<D>() * 4;
   s.rstat = s.list + WS_NC * 2 * SEL_WMAX * 4;
@@ -125,8 +119,8 @@ __device__ __forceinline__ int st_ntiles(int kv_end) { return kv_end > 0 ? (kv_e
 // Producers: every tile of every item, in the order the consumers take them.
 // ---------------------------------------------------------------------------
 template <int D, int RND, int PH>
-__device__ __forceinline__ void st_producer(const StArgs& a, const CUtensorMap* tmK, unsigned char* smem,
-                                            const StSmem& L, int warp, int lane) {
+__device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem, const StSmem& L, int warp,
+                                            int lane) {
   const Problem& p = a.p;
   const int G = gridDim.x, cta = blockIdx.x;
   const int s = 23 - p.mu;
@@ -136,12 +130,6 @@ __device__ __forceinline__ void st_producer(const StArgs& a, const CUtensorMap* 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
   float* qbase = reinterpret_cast<float*>(smem + L.q);
-  uint32_t kcount = 0;
-  KTma kt;
-  kt.map = tmK;
-  kt.ring = reinterpret_cast<uint16_t*>(smem + L.kring) + warp * KRING * WS_UNIT * WS_DS;
-  kt.bar = bars + sb_kring<D>() + warp * KRING;
-  kt.count = &kcount;
   // Q of the first two items (the consumers stage the later ones)
   for (int k0 = 0; k0 < 2; ++k0) {
     const int q0 = ws_item(k0, cta, G, a.n_items);
@@ -195,9 +183,8 @@ __device__ __forceinline__ void st_producer(const StArgs& a, const CUtensorMap* 
       } else {
         // the tile buffer is free once tile k - 2's P.V has completed and been read
         // (tfree): the tile routine waits for that only before its first store
-        if (!ws_produce_tile<D, RND, 1>(p, it, t0, tlen, sQ, tile, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
-                                        Kh, negc, pow2s, scale2, s, kt, k >= 2 ? bars + SB_TFREE + buf : nullptr,
-                                        ph)) {
+        if (!ws_produce_tile<D, RND>(p, it, t0, tlen, sQ, tile, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
+                                     negc, pow2s, scale2, s, k >= 2 ? bars + SB_TFREE + buf : nullptr, ph)) {
           ws_timeout(p);
           return;
         }
@@ -692,8 +679,7 @@ __device__ __forceinline__ void st_tensor_warpgroup(const StArgs& a, const CUten
 }
 
 template <int D, int RND, int VAR, int PH>
-__global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __grid_constant__ CUtensorMap tmK,
-                                                     const __grid_constant__ CUtensorMap tmV) {
+__global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __grid_constant__ CUtensorMap tmV) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + smem_align1k_pad(smem_raw);
   const StSmem L = st_plan<D>();
@@ -714,7 +700,6 @@ __global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __gr
       mbar_init(bars + sb_vempty<D>() + i, 1);
     }
     mbar_init(bars + sb_drain<D>(), 1);
-    for (int i = 0; i < WS_NP * KRING; ++i) mbar_init(bars + sb_kring<D>() + i, 1);
     mbar_fence_init();
   }
   if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
@@ -724,7 +709,7 @@ __global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __gr
   const uint32_t tbase = *tslot;
   if (warp < WS_NP) {
     regs_inc<kWsProdRegs>();
-    st_producer<D, RND, PH>(a, &tmK, smem, L, warp, lane);
+    st_producer<D, RND, PH>(a, smem, L, warp, lane);
   } else if (warp < WS_MW) {
     regs_inc<kWsConsRegs>();
     if (PH == 1) st_consumer_stats<D>(a, smem, L, warp - WS_NP, lane);
@@ -743,7 +728,7 @@ __global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __gr
 }
 
 template <int D, int RND, int VAR, int PH>
-cudaError_t st_launch_one(const StArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmV, int grid, cudaStream_t st) {
+cudaError_t st_launch_one(const StArgs& a, const CUtensorMap& tmV, int grid, cudaStream_t st) {
   auto k = st_kernel<D, RND, VAR, PH>;
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, k);
@@ -752,18 +737,18 @@ cudaError_t st_launch_one(const StArgs& a, const CUtensorMap& tmK, const CUtenso
   const size_t smem = (size_t)st_plan<D>().total + 1024;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, WS_NT, smem, st>>>(a, tmK, tmV);
+  k<<<grid, WS_NT, smem, st>>>(a, tmV);
   return cudaGetLastError();
 }
 
 template <int D, int RND>
-cudaError_t st_launch_var(const StArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmV, int grid, cudaStream_t st) {
-  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK, 0>(a, tmK, tmV, grid, st);
-  if (a.p.variant == LAMP_RELAXED) return st_launch_one<D, RND, LAMP_RELAXED, 0>(a, tmK, tmV, grid, st);
+cudaError_t st_launch_var(const StArgs& a, const CUtensorMap& tmV, int grid, cudaStream_t st) {
+  if (a.p.variant == LAMP_GIVEN_MASK) return st_launch_one<D, RND, LAMP_GIVEN_MASK, 0>(a, tmV, grid, st);
+  if (a.p.variant == LAMP_RELAXED) return st_launch_one<D, RND, LAMP_RELAXED, 0>(a, tmV, grid, st);
   // strict: the scores-and-statistics pass, then the selection pass
-  cudaError_t e = st_launch_one<D, RND, LAMP_STRICT, 1>(a, tmK, tmV, grid, st);
+  cudaError_t e = st_launch_one<D, RND, LAMP_STRICT, 1>(a, tmV, grid, st);
   if (e != cudaSuccess) return e;
-  return st_launch_one<D, RND, LAMP_STRICT, 2>(a, tmK, tmV, grid, st);
+  return st_launch_one<D, RND, LAMP_STRICT, 2>(a, tmV, grid, st);
 }
 
 }  // namespace
@@ -784,20 +769,19 @@ cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int
   a.slab = reinterpret_cast<float*>(base + ws.st_slab);
   a.ld = stream_slab_ld(p.n_k);
   a.rows = reinterpret_cast<RowStat*>(base + ws.st_rows);
-  CUtensorMap tmK, tmV;
-  cudaError_t e = make_tmap_bf16(&tmK, p.K, p.d, p.n_k, p.B * p.H, WS_DS, WS_UNIT, false);
-  if (e == cudaSuccess) e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, true);
+  CUtensorMap tmV;
+  const cudaError_t e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, true);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);
   if (p.d == 64) {
-    if (rnd == kRndFast) return st_launch_var<64, kRndFast>(a, tmK, tmV, grid, st);
-    if (rnd == kRndNone) return st_launch_var<64, kRndNone>(a, tmK, tmV, grid, st);
-    return st_launch_var<64, kRndExact>(a, tmK, tmV, grid, st);
+    if (rnd == kRndFast) return st_launch_var<64, kRndFast>(a, tmV, grid, st);
+    if (rnd == kRndNone) return st_launch_var<64, kRndNone>(a, tmV, grid, st);
+    return st_launch_var<64, kRndExact>(a, tmV, grid, st);
   }
-  if (rnd == kRndFast) return st_launch_var<128, kRndFast>(a, tmK, tmV, grid, st);
-  if (rnd == kRndNone) return st_launch_var<128, kRndNone>(a, tmK, tmV, grid, st);
-  return st_launch_var<128, kRndExact>(a, tmK, tmV, grid, st);
+  if (rnd == kRndFast) return st_launch_var<128, kRndFast>(a, tmV, grid, st);
+  if (rnd == kRndNone) return st_launch_var<128, kRndNone>(a, tmV, grid, st);
+  return st_launch_var<128, kRndExact>(a, tmV, grid, st);
 }
 
 }  // namespace lamp

@@ -126,7 +126,6 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
     ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
   }
   named_sync(BAR_PROD, WS_NP * 32);
-  const KTma kt{};  // K staged through registers
   int deal = 0;     // producer warp that takes the next unit
   for (int k = 0;; ++k) {
     const int q = ws_item(k, cta, G, a.n_items);
@@ -149,8 +148,8 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
     // the buffer itself is free once item k - 2's P.V has completed and its
     // output has been read (tfree): the tile routine waits for that only before
     // its first store
-    if (!ws_produce_tile<D, RND, 0>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast,
-                                    Kh, negc, pow2s, scale2, s, kt, k >= 2 ? bars + BAR_TFREE + buf : nullptr, ph)) {
+    if (!ws_produce_tile<D, RND>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
+                                 negc, pow2s, scale2, s, k >= 2 ? bars + BAR_TFREE + buf : nullptr, ph)) {
       ws_timeout(p);
       return;
     }

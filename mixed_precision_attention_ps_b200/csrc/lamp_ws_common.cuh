@@ -135,36 +135,24 @@ __device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, con
   }
 }
 
-// K staging of a producer warp.
-//   KT = 0: K slices travel global -> registers -> shared memory (binary32) two
-//           stream positions ahead of their use, so an L2 round trip hides behind
-//           two slices of arithmetic.
-//   KT = 1: a TMA load brings each bf16 slice (64 keys x 8 dimensions, 1 KB) into a
-//           ring of KRING stages of the warp, completing on the stage's mbarrier,
-//           three positions ahead; the warp widens the landed slice to binary32
-//           into the slice buffer one position ahead of its use.
-constexpr int KRING = 3;
-struct KTma {
-  const CUtensorMap* map;  // K as [B*H][n_k][d] bf16, box {8 dims, 64 keys, 1}
-  uint16_t* ring;          // this warp's KRING stages of [64 keys][8 dims] bf16 (1024-byte aligned)
-  uint64_t* bar;           // this warp's KRING mbarriers (one arrival + 1024 bytes each)
-  uint32_t* count;         // slices this warp has loaded so far (stage = n % KRING, phase = n / KRING)
-};
-
 // Scores of one tile of an item, keys t0 .. t0 + tlen - 1, by one producer warp:
 // the tile's 64-key units j = first, first + 8, ... (the others belong to the other
 // producer warps). The scores of key t0 + c go to rows[sw_off(r, c)] for the 16
 // rows r of the item (the block layout above); keys past a row's valid range hold
 // -inf.
-// The buffer may still be read by the tensor core when the call starts: the
-// warp waits for free_bar's phase free_phase (when free_bar is not null) only
-// before its first store, one unit of arithmetic later. Returns false when a
-// bounded wait gave up (the warp's copies in flight have then landed).
-template <int D, int RND, int KT>
+// K slices travel global -> registers -> shared memory (binary32) two stream
+// positions ahead of their use, so an L2 round trip hides behind two slices of
+// arithmetic. (A TMA load of each bf16 slice, a box of 64 rows of 16 bytes, into
+// a ring that the warp then widens was measured 15 % slower on the streamed
+// kernel.) The buffer may still be read by the tensor core when the call
+// starts: the warp waits for free_bar's phase free_phase (when free_bar is not
+// null) only before its first store, one unit of arithmetic later. Returns false
+// when that bounded wait gave up.
+template <int D, int RND>
 __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo& it, int t0, int tlen,
                                                 const float* sQ, float* rows, float* ksw, int lane, int first,
                                                 bool fast, const uint16_t* Kh, u64 negc, u64 pow2s, u64 scale2,
-                                                int s, const KTma& kt, uint64_t* free_bar, uint32_t free_phase) {
+                                                int s, uint64_t* free_bar, uint32_t free_phase) {
   constexpr int NSL = D / WS_DS;  // K slices per unit
   const int gr = lane & 1, gk = lane >> 1;  // rows 8gr..8gr+7, keys 4gk..4gk+3 of a unit
   const int qoff = 8 * gr, koff = 4 * gk;
@@ -172,23 +160,13 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
   const int mine = first < U ? (U - first + WS_NP - 1) / WS_NP : 0;
   const int total = mine * NSL;
   uint4 kra[2], krb[2];
-  auto load = [&](int pos, uint4 (&kr)[2]) {  // KT 0: keys lane and lane + 32 of the slice at pos
+  auto load = [&](int pos, uint4 (&kr)[2]) {  // keys lane and lane + 32 of the slice at pos
     const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int key = t0 + j * WS_UNIT + lane + 32 * h;
       kr[h] = make_uint4(0u, 0u, 0u, 0u);
       if (key < it.kv_end) kr[h] = __ldg(reinterpret_cast<const uint4*>(Kh + (size_t)key * D + sl * WS_DS));
-    }
-  };
-  auto issue = [&](int pos) {  // KT 1: TMA of the slice at pos into its ring stage
-    if (lane == 0) {
-      const uint32_t n = *kt.count + pos;
-      const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
-      fence_async_smem();  // the stage's earlier reads (generic proxy) precede the copy
-      mbar_expect_tx(kt.bar + n % KRING, WS_UNIT * WS_DS * 2);
-      tma_load_3d(kt.ring + (n % KRING) * WS_UNIT * WS_DS, kt.map, sl * WS_DS, t0 + j * WS_UNIT, it.bh,
-                  kt.bar + n % KRING);
     }
   };
   auto widen = [&](int b2, const uint4 (&kr)[2]) {  // binary32 [8 dims][64 keys] into slice buffer b2
@@ -204,20 +182,10 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
     }
   };
   bool failed = false;
-  int fpos = 0;  // the stream position during which a wait gave up
-  auto landed = [&](int pos, uint4 (&kr)[2]) -> bool {  // KT 1: the slice at pos from its ring stage
-    const uint32_t n = *kt.count + pos;
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(kt.bar + n % KRING, (n / KRING) & 1))) return false;
-    const uint16_t* src = kt.ring + (n % KRING) * WS_UNIT * WS_DS;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) kr[h] = *reinterpret_cast<const uint4*>(src + (lane + 32 * h) * WS_DS);
-    return true;
-  };
   u64 acc[4][4];
   // one stream position: compute slice pos, then stage slice pos + 1 into the free
-  // binary32 buffer and start the load of slice pos + 3 (KT 0: into `cur`, the
-  // register set of pos + 1, two sets alternating; KT 1: into the ring stage pos
-  // has released)
+  // binary32 buffer and start the load of slice pos + 3 into `cur` (the register
+  // set of pos + 1; two sets alternate, so no load is waited on early)
   auto body = [&](int pos, uint4 (&cur)[2]) {
     const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
     if (sl == 0) {
@@ -235,7 +203,6 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
       if (free_bar) {  // first store of the call: the buffer's previous contents are no longer read
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(free_bar, free_phase))) {
           failed = true;
-          fpos = pos;
           return;
         }
         free_bar = nullptr;
@@ -263,54 +230,20 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
       }
     }
     __syncwarp();  // every lane is done reading slice pos - 1's buffer
-    if (KT == 0) {
-      if (pos + 1 < total) widen((pos + 1) & 1, cur);
-      if (pos + 3 < total) load(pos + 3, cur);
-    } else {
-      if (pos + 1 < total) {
-        if (!landed(pos + 1, cur)) {
-          failed = true;
-          fpos = pos;
-          return;
-        }
-        widen((pos + 1) & 1, cur);
-      }
-      __syncwarp();  // every lane has read the stage of pos + 1 (and of pos, before)
-      if (pos + 3 < total) issue(pos + 3);
-    }
+    if (pos + 1 < total) widen((pos + 1) & 1, cur);
+    if (pos + 3 < total) load(pos + 3, cur);
     __syncwarp();
   };
-  if (KT == 0) {
-    if (total > 0) {
-      load(0, kra);
-      widen(0, kra);
-    }
-    if (total > 1) load(1, kra);
-    if (total > 2) load(2, krb);
-  } else {
-    for (int i = 0; i < 3 && i < total; ++i) issue(i);
-    if (total > 0) {
-      if (landed(0, kra)) {
-        widen(0, kra);
-      } else {
-        failed = true;
-        fpos = -1;
-      }
-    }
+  if (total > 0) {
+    load(0, kra);
+    widen(0, kra);
   }
+  if (total > 1) load(1, kra);
+  if (total > 2) load(2, krb);
   __syncwarp();
   for (int pos = 0; pos < total && !failed; pos += 2) {
     body(pos, kra);
     if (pos + 1 < total && !failed) body(pos + 1, krb);
-  }
-  if (KT == 1) {
-    if (failed) {  // the slices requested but not yet landed must land before the warp gives up
-      for (int q = fpos + 1; q <= fpos + 2 && q < total; ++q) {
-        const uint32_t n = *kt.count + q;
-        mbar_wait(kt.bar + n % KRING, (n / KRING) & 1);
-      }
-    }
-    *kt.count += total;
   }
   return !failed;  // (a warp with no unit of its own writes nothing and so needs no wait)
 }
