@@ -73,6 +73,7 @@ struct WsSmem {  // byte offsets from a 1024-byte aligned base
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
   int otile;  // output tile of an item [16][D] bf16 (epilogue)
   int bars;   // mbarriers
+  int sched;  // item ring [8] (the CTA's k-th item at k % 8; -1 = no more) and the published count
   int tmem;   // TMEM base address (written by tcgen05.alloc)
   int total;
 };
@@ -88,18 +89,51 @@ __host__ __device__ inline WsSmem ws_plan(int n_k) {
   s.stats = s.list + WS_NC * 2 * SEL_WMAX * 4;
   s.otile = s.stats + 2 * WS_BM * 2 * 4;
   s.bars = s.otile + WS_BM * D * 2;
-  s.tmem = s.bars + (bar_drain<D>() + 1) * 8;
+  s.sched = s.bars + (bar_drain<D>() + 1) * 8;
+  s.tmem = s.sched + 16 * 4;
   s.total = s.tmem + 16;
   return s;
 }
 
 struct WsArgs {
   Problem p;
-  const int* stats;  // per-(b, h) exponent statistics
+  const int* stats;   // per-(b, h) exponent statistics
+  unsigned* counter;  // next item to hand out (zeroed by the preparation kernel)
   int nchunk;
   int n_items;
   int n_rb;
 };
+
+// Items are handed out at run time, heaviest first, from a global counter, so
+// that CTAs which run slower (two SMs share a TPC's resources) take fewer. The
+// CTA's k-th item is claimed two items ahead: items 0 and 1 by the producers at
+// the start, item k + 2 by the consumers when they begin item k. Its number
+// (-1: none left) goes to ring[k % 8], then the published count rises to k + 1.
+// The producers read it after pready of item k - 2, the consumers after their
+// own barrier, the tensor-core warpgroup after seeing the count pass k.
+constexpr int kRing = 8;
+__device__ __forceinline__ int claim_item(unsigned* counter, int n_items) {
+  const unsigned q = atomicAdd(counter, 1u);
+  return q < (unsigned)n_items ? (int)q : -1;
+}
+__device__ __forceinline__ void publish_item(volatile int* sched, int k, int q) {
+  sched[k % kRing] = q;
+  __threadfence_block();
+  sched[kRing] = k + 1;
+}
+// Bounded wait until the CTA's k-th item is published: its number (-1: none),
+// or -2 when the wait gave up.
+__device__ __forceinline__ int wait_published(const volatile int* sched, int k) {
+  if (sched[kRing] <= k) {
+    const uint64_t t0 = global_ns();
+    while (sched[kRing] <= k) {
+      if (global_ns() - t0 > kWaitLimitNs) return -2;
+      __nanosleep(32);
+    }
+  }
+  __threadfence_block();
+  return sched[k % kRing];
+}
 
 // ---------------------------------------------------------------------------
 // Producers: PS(mu) scores of every item into the item's row buffer.
@@ -108,7 +142,6 @@ template <int D, int RND>
 __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int warp,
                                             int lane) {
   const Problem& p = a.p;
-  const int G = gridDim.x, cta = blockIdx.x;
   const int s = 23 - p.mu;
   const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
   const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
@@ -119,26 +152,33 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
   const int rb = sw_bytes(p.n_k);
   // failure-path tests: hand over nothing, so that every other warp's bounded wait runs out
   if (p.debug_stall == LAMP_DEBUG_STALL_PRODUCERS) return;
-  // Q of the first two items (the consumers stage the later ones)
+  volatile int* sched = reinterpret_cast<volatile int*>(smem + L.sched);
+  // claim the first two items and stage their Q (the consumers do the later ones)
+  if (warp == 0 && lane == 0) {
+    const int q0 = claim_item(a.counter, a.n_items);
+    sched[0] = q0;
+    publish_item(sched, 1, q0 < 0 ? -1 : claim_item(a.counter, a.n_items));
+  }
+  named_sync(BAR_PROD, WS_NP * 32);
   for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = ws_item(k0, cta, G, a.n_items);
+    const int q0 = sched[k0];
     if (q0 < 0) break;
     ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
   }
   named_sync(BAR_PROD, WS_NP * 32);
   int deal = 0;     // producer warp that takes the next unit
   for (int k = 0;; ++k) {
-    const int q = ws_item(k, cta, G, a.n_items);
-    if (q < 0) break;
     const int buf = k & 1;
-    const ItemInfo it = ws_decode(q, p, a.n_rb);
     const uint32_t ph = ((k - 2) >> 1) & 1;
-    // Q of item k is staged (with the consumers' hand-off of item k - 2); one
-    // decision per warp: the tile routine synchronises the whole warp
+    // item k is claimed and its Q staged (with the consumers' hand-off of item
+    // k - 2); one decision per warp: the tile routine synchronises the whole warp
     if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + BAR_PREADY + buf, ph))) {
       ws_timeout(p);
       return;
     }
+    const int q = sched[k % kRing];
+    if (q < 0) break;
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
     const float* sQ = qbase + buf * ws_qfloats<D>();
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
@@ -217,7 +257,6 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   constexpr int NCT = WS_NC * 32;  // consumer threads
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
-  const int G = gridDim.x, cta = blockIdx.x;
   const int nwords = (p.n_k + 31) >> 5;
   const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = WS_BAND * p.tau;
@@ -225,18 +264,32 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
   float* qbase = reinterpret_cast<float*>(smem + L.q);
   const int rb = sw_bytes(p.n_k);
+  volatile int* sched = reinterpret_cast<volatile int*>(smem + L.sched);
   long long nsel = 0;
   for (int k = 0;; ++k) {
-    const int q = ws_item(k, cta, G, a.n_items);
+    // items 0 and 1 come from the producers (all threads agree on whether the
+    // wait for them gave up), later ones from this warpgroup
+    int q;
+    if (k < 2) {
+      q = wait_published(sched, k);
+      if (named_or(BAR_CONS, NCT, q == -2)) {
+        ws_timeout(p);
+        return;
+      }
+    } else {
+      q = sched[k % kRing];
+    }
     if (q < 0) break;
     const int buf = k & 1;
-    const ItemInfo it = ws_decode(q, p, a.n_rb);
-    const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
+    // claim item k + 2 now, so that the tensor-core warpgroup can prefetch its V
+    if (tidc == 0) publish_item(sched, k + 2, claim_item(a.counter, a.n_items));
     const bool ok = mbar_wait(bars + BAR_FULL + buf, (k >> 1) & 1);
-    if (named_or(BAR_CONS, NCT, !ok)) {
+    if (named_or(BAR_CONS, NCT, !ok)) {  // also makes item k + 2's number visible to every consumer
       ws_timeout(p);
       return;
     }
+    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
                                                           p.emax_sum_limit);
     float* sQ = qbase + buf * ws_qfloats<D>();
@@ -404,7 +457,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     fence_async_smem();  // P (generic-proxy stores) becomes visible to the tensor core
     named_sync(BAR_CONS, NCT);  // every P row of the item is in place; Q of the item is no longer read
-    const int q2 = ws_item(k + 2, cta, G, a.n_items);
+    const int q2 = sched[(k + 2) % kRing];
     if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
     mbar_arrive(bars + BAR_PREADY + buf);  // P of item k in place, Q of item k + 2 staged
   }
@@ -422,7 +475,6 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
   constexpr int S = ws_vslots<D>();
   constexpr uint32_t TB = ws_vtile_bytes<D>();
   const Problem& p = a.p;
-  const int G = gridDim.x, cta = blockIdx.x;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   unsigned char* vring = smem + L.v;
   const uint32_t vbase = smem_u32(vring), rbase = smem_u32(smem + L.rows);
@@ -433,10 +485,13 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
   // V tiles form one sequence over the CTA's items: tile tl of item kl is number gl
   int kl = 0, tl = 0, Tl = -1, bhl = 0;
   int gl = 0, gm = 0;  // next tile to load, next tile to multiply
-  auto next_tile = [&]() -> bool {
+  const volatile int* sched = reinterpret_cast<const volatile int*>(smem + L.sched);
+  auto next_tile = [&]() -> bool {  // false: no further tile known yet (or none left)
     for (;;) {
       if (Tl < 0) {
-        const int q = ws_item(kl, cta, G, a.n_items);
+        if (sched[kRing] <= kl) return false;  // item kl is not claimed yet
+        __threadfence_block();
+        const int q = sched[kl % kRing];
         if (q < 0) return false;
         const ItemInfo it = ws_decode(q, p, a.n_rb);
         Tl = (it.kv_end + WS_VKEYS - 1) / WS_VKEYS;
@@ -498,8 +553,12 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
   uint16_t* otile = reinterpret_cast<uint16_t*>(smem + L.otile);
   bool good = true;
   for (int k = 0;; ++k) {
-    const int q = ws_item(k, cta, G, a.n_items);
-    if (q < 0) break;
+    const int q = wait_published(sched, k);
+    if (q == -1) break;
+    if (q < 0) {  // the wait gave up (agreed: every thread polls the same count)
+      good = false;
+      break;
+    }
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     if (issuer && ok) mma_item(k, it);
     __syncwarp();
@@ -544,6 +603,7 @@ __global__ void __launch_bounds__(WS_NT, 1) ws_kernel(const WsArgs a, const __gr
     }
     mbar_init(bars + bar_drain<D>(), 1);
     mbar_fence_init();
+    reinterpret_cast<volatile int*>(smem + L.sched)[kRing] = 0;  // no item published yet
   }
   if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
   tc_fence_before();
@@ -603,6 +663,7 @@ cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num
   WsArgs a;
   a.p = p;
   a.stats = reinterpret_cast<const int*>(base + ws.stats);
+  a.counter = reinterpret_cast<unsigned*>(base + ws.counters);
   a.nchunk = ws.nchunk;
   a.n_rb = (p.n_q + WS_BM - 1) / WS_BM;
   a.n_items = a.n_rb * p.B * p.H;
