@@ -14,8 +14,8 @@
 // it, FP32 recompute of the selection before the softmax.
 //
 // Same organisation as the whole-row kernel (lamp_ws.cu): one persistent CTA of
-// 640 threads per SM, items (b, h, 16 query rows) in a snake order, two tile
-// buffers in the block layout of lamp_ws_common.cuh.
+// 640 threads per SM, items (b, h, 16 query rows) handed out at run time from a
+// global counter, two tile buffers in the block layout of lamp_ws_common.cuh.
 //   producers (warps 0-7): 64-key units dealt round-robin, PS(mu) steps as packed
 //     binary32 pairs, K slices staged through registers as binary32.
 //   consumers (warps 8-15): per tile the criterion (double re-evaluation near
@@ -66,6 +66,7 @@ struct StSmem {  // byte offsets from a 1024-byte aligned base
   int rstat;  // per tile parity and row: m, l, alpha, spare [2][16][4] f32
   int otile;  // output tile of an item [16][D] bf16 (epilogue)
   int bars;   // mbarriers
+  int sched;  // item ring [8] and published count (lamp_ws_common.cuh)
   int tmem;   // TMEM base address
   int total;
 };
@@ -81,7 +82,8 @@ __host__ __device__ inline StSmem st_plan() {
   s.rstat = s.list + WS_NC * 2 * SEL_WMAX * 4;
   s.otile = s.rstat + 2 * WS_BM * 4 * 4;
   s.bars = s.otile + WS_BM * D * 2;
-  s.tmem = s.bars + sb_count<D>() * 8;
+  s.sched = s.bars + sb_count<D>() * 8;
+  s.tmem = s.sched + 16 * 4;
   s.total = s.tmem + 16;
   return s;
 }
@@ -104,7 +106,8 @@ struct RowStat {
 
 struct StArgs {
   Problem p;
-  const int* stats;  // per-(b, h) exponent statistics
+  const int* stats;   // per-(b, h) exponent statistics
+  unsigned* counter;  // next item to hand out (zeroed by the preparation kernel; one per pass)
   int nchunk;
   int n_items;
   int n_rb;
@@ -115,6 +118,22 @@ struct StArgs {
 
 __device__ __forceinline__ int st_ntiles(int kv_end) { return kv_end > 0 ? (kv_end + ST_T - 1) / ST_T : 1; }
 
+// The consumers' item ii (-1: none left, -2: the wait for it gave up, agreed by
+// every consumer thread). Items 0 and 1 come from the producers; at each item
+// thread 0 claims item ii + 2, which the consumers' next barrier (the first
+// tile's hand-off) makes visible to all of them.
+__device__ __forceinline__ int st_next_item(const StArgs& a, ItemRing sched, int ii, int tidc) {
+  int q;
+  if (ii < 2) {
+    q = wait_published(sched, ii);
+    if (named_or(BAR_CONS, WS_NC * 32, q == -2)) return -2;
+  } else {
+    q = sched.get(ii);
+  }
+  if (q >= 0 && tidc == 0) publish_item(sched, ii + 2, claim_item(a.counter, a.n_items));
+  return q;
+}
+
 // ---------------------------------------------------------------------------
 // Producers: every tile of every item, in the order the consumers take them.
 // ---------------------------------------------------------------------------
@@ -122,7 +141,6 @@ template <int D, int RND, int PH>
 __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem, const StSmem& L, int warp,
                                             int lane) {
   const Problem& p = a.p;
-  const int G = gridDim.x, cta = blockIdx.x;
   const int s = 23 - p.mu;
   const u64 negc = pack2(-(float)((1u << s) - 1u), -(float)((1u << s) - 1u));
   const u64 pow2s = pack2((float)(1u << s), (float)(1u << s));
@@ -130,9 +148,16 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* ksw = reinterpret_cast<float*>(smem + L.ks) + warp * 2 * WS_DS * WS_UNIT;
   float* qbase = reinterpret_cast<float*>(smem + L.q);
-  // Q of the first two items (the consumers stage the later ones)
+  const ItemRing sched{smem_u32(smem + L.sched)};
+  // claim the first two items and stage their Q (the consumers do the later ones)
+  if (warp == 0 && lane == 0) {
+    const int q0 = claim_item(a.counter, a.n_items);
+    sched.put(0, q0);
+    publish_item(sched, 1, q0 < 0 ? -1 : claim_item(a.counter, a.n_items));
+  }
+  named_sync(BAR_PROD, WS_NP * 32);
   for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = ws_item(k0, cta, G, a.n_items);
+    const int q0 = sched.get(k0);
     if (q0 < 0) break;
     ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
   }
@@ -140,7 +165,14 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
   int deal = 0;  // producer warp that takes the next unit
   int k = 0;     // tile counter: buffer k & 1, phase k >> 1
   for (int ii = 0;; ++ii) {
-    const int q = ws_item(ii, cta, G, a.n_items);
+    // the consumers' hand-off of tile k - 2, which follows their claim of item ii
+    // (made when they began item ii - 2, whose first tile is k - 2 or earlier);
+    // one decision per warp: the tile routine synchronises the warp
+    if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + SB_PREADY + (k & 1), ((k - 2) >> 1) & 1))) {
+      ws_timeout(p);
+      return;
+    }
+    const int q = sched.get(ii);
     if (q < 0) break;
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
@@ -153,9 +185,9 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
       const int t0 = t * ST_T;
       const int tlen = max(0, min(ST_T, it.kv_end - t0));
       const uint32_t ph = ((k - 2) >> 1) & 1;
-      // the consumers' hand-off of tile k - 2 (and, at an item's first tile, its Q
-      // staged); one decision per warp: the tile routine synchronises the warp
-      if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + SB_PREADY + buf, ph))) {
+      // the consumers' hand-off of tile k - 2 (waited above for an item's first
+      // tile, whose Q it also brings)
+      if (t > 0 && k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + SB_PREADY + buf, ph))) {
         ws_timeout(p);
         return;
       }
@@ -203,7 +235,6 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   constexpr int NCT = WS_NC * 32;
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
-  const int G = gridDim.x, cta = blockIdx.x;
   const int nwords = (p.n_k + 31) >> 5;
   const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = WS_BAND * p.tau;
@@ -213,10 +244,15 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
   uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
   float* qbase = reinterpret_cast<float*>(smem + L.q);
   float* rst = reinterpret_cast<float*>(smem + L.rstat);
+  const ItemRing sched{smem_u32(smem + L.sched)};
   long long nsel = 0;
   int k = 0;
   for (int ii = 0;; ++ii) {
-    const int q = ws_item(ii, cta, G, a.n_items);
+    const int q = st_next_item(a, sched, ii, tidc);
+    if (q == -2) {
+      ws_timeout(p);
+      return;
+    }
     if (q < 0) break;
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
@@ -359,7 +395,7 @@ __device__ __forceinline__ void st_consumer(const StArgs& a, unsigned char* smem
       fence_async_smem();  // P (generic-proxy stores) becomes visible to the tensor core
       named_sync(BAR_CONS, NCT);  // P and every row's m, l, alpha of the tile are in place
       if (t == nt - 1) {   // Q of the item is no longer read: stage item + 2's
-        const int q2 = ws_item(ii + 2, cta, G, a.n_items);
+        const int q2 = sched.get(ii + 2);
         if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
       }
       mbar_arrive(bars + SB_PREADY + buf);  // P of the tile in place (and at an item's end, Q of item + 2)
@@ -396,12 +432,16 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
   constexpr int NCT = WS_NC * 32;
   const Problem& p = a.p;
   const int tidc = cw * 32 + lane;
-  const int G = gridDim.x, cta = blockIdx.x;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* qbase = reinterpret_cast<float*>(smem + L.q);
+  const ItemRing sched{smem_u32(smem + L.sched)};
   int k = 0;
   for (int ii = 0;; ++ii) {
-    const int q = ws_item(ii, cta, G, a.n_items);
+    const int q = st_next_item(a, sched, ii, tidc);
+    if (q == -2) {
+      ws_timeout(p);
+      return;
+    }
     if (q < 0) break;
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     float* sQ = qbase + (ii & 1) * ws_qfloats<D>();
@@ -484,7 +524,7 @@ __device__ __forceinline__ void st_consumer_stats(const StArgs& a, unsigned char
             a.rows[grow[tt]] = rs;
           }
         // this pass reads no Q, and the producers are done with the item's
-        const int q2 = ws_item(ii + 2, cta, G, a.n_items);
+        const int q2 = sched.get(ii + 2);
         if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
       }
       mbar_arrive(bars + SB_PREADY + buf);  // tile buffer read (and, after an item's last tile, Q of item + 2 staged)
@@ -508,10 +548,10 @@ __device__ __forceinline__ void st_tensor_warpgroup(const StArgs& a, const CUten
   constexpr int S = st_vslots<D>();
   constexpr uint32_t TB = st_vtile_bytes<D>();
   const Problem& p = a.p;
-  const int G = gridDim.x, cta = blockIdx.x;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   unsigned char* vring = smem + L.v;
   const uint32_t vbase = smem_u32(vring), tiles = smem_u32(smem + L.tiles);
+  const ItemRing sched{smem_u32(smem + L.sched)};
   const uint32_t idesc = umma_idesc_bf16(D, 32);
   const float* rst = reinterpret_cast<const float*>(smem + L.rstat);
   uint16_t* otile = reinterpret_cast<uint16_t*>(smem + L.otile);
@@ -521,10 +561,12 @@ __device__ __forceinline__ void st_tensor_warpgroup(const StArgs& a, const CUten
   // (item il, tile tl) is number gl
   int il = 0, tl = 0, ntl = -1, bhl = 0, kvl = 0, vt = 0, nvl = -1;
   int gl = 0, gm = 0;  // next V tile to load, next V tile to multiply
-  auto next_v = [&]() -> bool {
+  auto next_v = [&]() -> bool {  // false: no further V tile known yet (or none left)
     for (;;) {
       if (ntl < 0) {  // enter item il
-        const int q = ws_item(il, cta, G, a.n_items);
+        if (sched.count() <= il) return false;  // item il is not claimed yet
+        __threadfence_block();
+        const int q = sched.get(il);
         if (q < 0) return false;
         const ItemInfo it = ws_decode(q, p, a.n_rb);
         ntl = st_ntiles(it.kv_end);
@@ -604,8 +646,12 @@ __device__ __forceinline__ void st_tensor_warpgroup(const StArgs& a, const CUten
   bool good = true;
   int k = 0;
   for (int ii = 0; good; ++ii) {
-    const int q = ws_item(ii, cta, G, a.n_items);
-    if (q < 0) break;
+    const int q = wait_published(sched, ii);
+    if (q == -1) break;
+    if (q < 0) {  // the wait gave up (agreed: every thread polls the same count)
+      good = false;
+      break;
+    }
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const int nt = st_ntiles(it.kv_end);
     float o[WS_BM];  // this thread's head dimension of the item's 16 rows
@@ -701,6 +747,7 @@ __global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __gr
     }
     mbar_init(bars + sb_drain<D>(), 1);
     mbar_fence_init();
+    ItemRing{smem_u32(smem + L.sched)}.set_count(0);  // no item published yet
   }
   if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
   tc_fence_before();
@@ -730,6 +777,8 @@ __global__ void __launch_bounds__(WS_NT, 1) st_kernel(const StArgs a, const __gr
 template <int D, int RND, int VAR, int PH>
 cudaError_t st_launch_one(const StArgs& a, const CUtensorMap& tmV, int grid, cudaStream_t st) {
   auto k = st_kernel<D, RND, VAR, PH>;
+  StArgs b = a;
+  b.counter += PH == 2 ? 1 : 0;  // the selection pass hands out the items afresh
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, k);
   if (e != cudaSuccess) return e;
@@ -737,7 +786,7 @@ cudaError_t st_launch_one(const StArgs& a, const CUtensorMap& tmV, int grid, cud
   const size_t smem = (size_t)st_plan<D>().total + 1024;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, WS_NT, smem, st>>>(a, tmV);
+  k<<<grid, WS_NT, smem, st>>>(b, tmV);
   return cudaGetLastError();
 }
 
@@ -763,6 +812,7 @@ cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int
   StArgs a;
   a.p = p;
   a.stats = reinterpret_cast<const int*>(base + ws.stats);
+  a.counter = reinterpret_cast<unsigned*>(base + ws.counters);
   a.nchunk = ws.nchunk;
   a.n_rb = (p.n_q + WS_BM - 1) / WS_BM;
   a.n_items = a.n_rb * p.B * p.H;

@@ -104,36 +104,6 @@ struct WsArgs {
   int n_rb;
 };
 
-// Items are handed out at run time, heaviest first, from a global counter, so
-// that CTAs which run slower (two SMs share a TPC's resources) take fewer. The
-// CTA's k-th item is claimed two items ahead: items 0 and 1 by the producers at
-// the start, item k + 2 by the consumers when they begin item k. Its number
-// (-1: none left) goes to ring[k % 8], then the published count rises to k + 1.
-// The producers read it after pready of item k - 2, the consumers after their
-// own barrier, the tensor-core warpgroup after seeing the count pass k.
-constexpr int kRing = 8;
-__device__ __forceinline__ int claim_item(unsigned* counter, int n_items) {
-  const unsigned q = atomicAdd(counter, 1u);
-  return q < (unsigned)n_items ? (int)q : -1;
-}
-__device__ __forceinline__ void publish_item(volatile int* sched, int k, int q) {
-  sched[k % kRing] = q;
-  __threadfence_block();
-  sched[kRing] = k + 1;
-}
-// Bounded wait until the CTA's k-th item is published: its number (-1: none),
-// or -2 when the wait gave up.
-__device__ __forceinline__ int wait_published(const volatile int* sched, int k) {
-  if (sched[kRing] <= k) {
-    const uint64_t t0 = global_ns();
-    while (sched[kRing] <= k) {
-      if (global_ns() - t0 > kWaitLimitNs) return -2;
-      __nanosleep(32);
-    }
-  }
-  __threadfence_block();
-  return sched[k % kRing];
-}
 
 // ---------------------------------------------------------------------------
 // Producers: PS(mu) scores of every item into the item's row buffer.
@@ -152,16 +122,16 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
   const int rb = sw_bytes(p.n_k);
   // failure-path tests: hand over nothing, so that every other warp's bounded wait runs out
   if (p.debug_stall == LAMP_DEBUG_STALL_PRODUCERS) return;
-  volatile int* sched = reinterpret_cast<volatile int*>(smem + L.sched);
+  const ItemRing sched{smem_u32(smem + L.sched)};
   // claim the first two items and stage their Q (the consumers do the later ones)
   if (warp == 0 && lane == 0) {
     const int q0 = claim_item(a.counter, a.n_items);
-    sched[0] = q0;
+    sched.put(0, q0);
     publish_item(sched, 1, q0 < 0 ? -1 : claim_item(a.counter, a.n_items));
   }
   named_sync(BAR_PROD, WS_NP * 32);
   for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = sched[k0];
+    const int q0 = sched.get(k0);
     if (q0 < 0) break;
     ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
   }
@@ -176,7 +146,7 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
       ws_timeout(p);
       return;
     }
-    const int q = sched[k % kRing];
+    const int q = sched.get(k);
     if (q < 0) break;
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const float* sQ = qbase + buf * ws_qfloats<D>();
@@ -264,7 +234,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + L.list) + cw * 2 * SEL_WMAX;
   float* qbase = reinterpret_cast<float*>(smem + L.q);
   const int rb = sw_bytes(p.n_k);
-  volatile int* sched = reinterpret_cast<volatile int*>(smem + L.sched);
+  const ItemRing sched{smem_u32(smem + L.sched)};
   long long nsel = 0;
   for (int k = 0;; ++k) {
     // items 0 and 1 come from the producers (all threads agree on whether the
@@ -277,7 +247,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
         return;
       }
     } else {
-      q = sched[k % kRing];
+      q = sched.get(k);
     }
     if (q < 0) break;
     const int buf = k & 1;
@@ -457,7 +427,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     fence_async_smem();  // P (generic-proxy stores) becomes visible to the tensor core
     named_sync(BAR_CONS, NCT);  // every P row of the item is in place; Q of the item is no longer read
-    const int q2 = sched[(k + 2) % kRing];
+    const int q2 = sched.get(k + 2);
     if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
     mbar_arrive(bars + BAR_PREADY + buf);  // P of item k in place, Q of item k + 2 staged
   }
@@ -485,13 +455,13 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
   // V tiles form one sequence over the CTA's items: tile tl of item kl is number gl
   int kl = 0, tl = 0, Tl = -1, bhl = 0;
   int gl = 0, gm = 0;  // next tile to load, next tile to multiply
-  const volatile int* sched = reinterpret_cast<const volatile int*>(smem + L.sched);
+  const ItemRing sched{smem_u32(smem + L.sched)};
   auto next_tile = [&]() -> bool {  // false: no further tile known yet (or none left)
     for (;;) {
       if (Tl < 0) {
-        if (sched[kRing] <= kl) return false;  // item kl is not claimed yet
+        if (sched.count() <= kl) return false;  // item kl is not claimed yet
         __threadfence_block();
-        const int q = sched[kl % kRing];
+        const int q = sched.get(kl);
         if (q < 0) return false;
         const ItemInfo it = ws_decode(q, p, a.n_rb);
         Tl = (it.kv_end + WS_VKEYS - 1) / WS_VKEYS;
@@ -603,7 +573,7 @@ __global__ void __launch_bounds__(WS_NT, 1) ws_kernel(const WsArgs a, const __gr
     }
     mbar_init(bars + bar_drain<D>(), 1);
     mbar_fence_init();
-    reinterpret_cast<volatile int*>(smem + L.sched)[kRing] = 0;  // no item published yet
+    ItemRing{smem_u32(smem + L.sched)}.set_count(0);  // no item published yet
   }
   if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
   tc_fence_before();

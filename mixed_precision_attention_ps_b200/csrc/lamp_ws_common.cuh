@@ -66,10 +66,44 @@ __device__ __forceinline__ int p_off(int r, int j) {
 // Bytes of the score rows of an item with n keys.
 __host__ __device__ constexpr int sw_bytes(int n) { return ((n + 63) / 64) * 4096; }
 
-// The k-th item of CTA b (snake order over heaviest-first items), or -1.
-__device__ __forceinline__ int ws_item(int k, int b, int G, int n_items) {
-  const int q = (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
-  return q < n_items ? q : -1;
+// Items are handed out at run time, heaviest first, from a global counter, so
+// that CTAs which run slower (two SMs share a TPC's resources) take fewer. A
+// CTA claims its k-th item two items ahead: items 0 and 1 by the producers at
+// the start, item k + 2 by the consumers when they begin item k. The number
+// (-1: none left) goes to ring[k % 8] in shared memory, then the published count
+// ring[8] (zeroed at kernel start) rises to k + 1. The producers read it after
+// the consumers' hand-off of an earlier tile, the consumers after their own
+// barrier, the tensor-core warpgroup after seeing the count pass k.
+constexpr int kRing = 8;
+// The ring, addressed through its 32-bit shared-window address.
+struct ItemRing {
+  uint32_t a;  // address of ring[0]
+  __device__ __forceinline__ int get(int k) const { return ld_volatile_shared(a + 4 * (k & (kRing - 1))); }
+  __device__ __forceinline__ int count() const { return ld_volatile_shared(a + 4 * kRing); }
+  __device__ __forceinline__ void put(int k, int q) const { st_volatile_shared(a + 4 * (k & (kRing - 1)), q); }
+  __device__ __forceinline__ void set_count(int n) const { st_volatile_shared(a + 4 * kRing, n); }
+};
+__device__ __forceinline__ int claim_item(unsigned* counter, int n_items) {
+  const unsigned q = atomicAdd(counter, 1u);
+  return q < (unsigned)n_items ? (int)q : -1;
+}
+__device__ __forceinline__ void publish_item(ItemRing r, int k, int q) {
+  r.put(k, q);
+  __threadfence_block();
+  r.set_count(k + 1);
+}
+// Bounded wait until the CTA's k-th item is published: its number (-1: none),
+// or -2 when the wait gave up.
+__device__ __forceinline__ int wait_published(ItemRing r, int k) {
+  if (r.count() <= k) {
+    const uint64_t t0 = global_ns();
+    while (r.count() <= k) {
+      if (global_ns() - t0 > kWaitLimitNs) return -2;
+      __nanosleep(32);
+    }
+  }
+  __threadfence_block();
+  return r.get(k);
 }
 
 struct ItemInfo {
