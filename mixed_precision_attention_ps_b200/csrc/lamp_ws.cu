@@ -9,9 +9,9 @@
 // strict test 2 z (1 - z) |y| > tau on the whole probability row); section
 // "Experimental results" (PS(mu), relaxed relative threshold, random control).
 //
-// One persistent CTA of 640 threads (5 warpgroups) per SM works through a fixed
-// sequence of items (b, h, block of 16 query rows), heaviest causal blocks first,
-// in a snake order over the CTAs. Two row buffers alternate between three warp
+// One persistent CTA of 640 threads (5 warpgroups) per SM works through items
+// (b, h, block of 16 query rows) that it claims at run time from a work counter,
+// heaviest causal blocks first. Two row buffers alternate between three warp
 // roles, each warpgroup with its own register budget (setmaxnreg):
 //
 //   producers (warps 0-7): PS(mu) scores of item k into buffer k & 1. The item's
@@ -25,21 +25,23 @@
 //     row maximum and first argmax, S_rest in double (strict), the criterion with
 //     a double re-evaluation near tau, mask words, warp-compacted FP32 recompute,
 //     then the softmax numerators of the mixed row written in place as bf16 hi/lo
-//     parts in the tensor-core operand layout (sw_off / p_off), and the staging of
-//     Q for item k + 2.
+//     parts in the tensor-core operand layout (sw_off / p_off).
 //   tensor-core warpgroup (warps 16-19): one thread streams V tiles of 64 keys by
 //     TMA into a ring of shared-memory slots (running ahead across items) and, for
 //     each item once its P is in place, issues O^T = V^T P^T by tcgen05.mma into
 //     one of two TMEM accumulators (lamp_umma.cuh); tcgen05.commit frees each V
 //     slot and signals the item's completion. Then the four warps (one per TMEM
 //     lane quarter) read the accumulator, scale by 1 / l and store the output
-//     with 16-byte stores through a shared-memory tile.
+//     with 16-byte stores through a shared-memory tile. Warp 17 also hands out
+//     the items: it claims item k + 3, reads its head's exponent statistics,
+//     stages its Q into slot k % 3 and publishes it in a ring in shared memory
+//     once the output of item k is stored.
 //
 // Hand-offs use mbarriers: full[b] (256 producer arrivals: the scores are in
-// place), pready[b] (256 consumer arrivals: P in place, Q of item k + 2 staged),
-// empty[b] (the item's MMAs have completed), tfree[b] (128 epilogue arrivals:
-// accumulator and row statistics read, so the buffer may be refilled),
-// vfull/vempty per V slot.
+// place), pready[b] (256 consumer arrivals: P in place), empty[b] (the item's
+// MMAs have completed), tfree[b] (128 epilogue arrivals: accumulator and row
+// statistics read, so the buffer may be refilled), vfull/vempty per V slot; and
+// the ring's published count (polled).
 // Every wait is bounded; a wait that gives up records LAMP_ERR_TIMEOUT in the
 // caller's status word (when given) and ends the kernel after the tensor-core
 // work in flight has drained and the tensor memory is released.
@@ -61,19 +63,18 @@ template <int D>
 __host__ __device__ constexpr int bar_vempty() { return BAR_VFULL + ws_vslots<D>(); }
 template <int D>
 __host__ __device__ constexpr int bar_drain() { return BAR_VFULL + 2 * ws_vslots<D>(); }
-constexpr int BAR_PROD = 2;  // named barrier of the producer group
 constexpr int BAR_EPI = 3;   // named barrier of the tensor-core warpgroup (output epilogue)
 
 struct WsSmem {  // byte offsets from a 1024-byte aligned base
   int rows;   // score rows [2][sw_bytes(n_k)] (block layout of lamp_ws_common.cuh)
   int v;      // V ring [S][D / 64][64 keys][64 dims] bf16, as the TMA leaves it (128-byte swizzle)
   int ks;     // producer K slices [8 warps][2][8][64] f32
-  int q;      // Q [2][D][16] f32
+  int q;      // Q [3][D][16] f32 (item k in slot k % 3)
   int list;   // consumer mask-word buffers [8][2][32] uint32
   int stats;  // per buffer and row: softmax max, normaliser [2][16][2] f32
   int otile;  // output tile of an item [16][D] bf16 (epilogue)
   int bars;   // mbarriers
-  int sched;  // item ring [8] (the CTA's k-th item at k % 8; -1 = no more) and the published count
+  int sched;  // item ring [8] and its published count (ItemRing)
   int tmem;   // TMEM base address (written by tcgen05.alloc)
   int total;
 };
@@ -85,7 +86,7 @@ __host__ __device__ inline WsSmem ws_plan(int n_k) {
   s.v = 2 * sw_bytes(n_k);
   s.ks = s.v + ws_vslots<D>() * ws_vtile_bytes<D>();
   s.q = s.ks + WS_NP * 2 * WS_DS * WS_UNIT * 4;
-  s.list = s.q + 2 * ws_qfloats<D>() * 4;
+  s.list = s.q + 3 * ws_qfloats<D>() * 4;
   s.stats = s.list + WS_NC * 2 * SEL_WMAX * 4;
   s.otile = s.stats + 2 * WS_BM * 2 * 4;
   s.bars = s.otile + WS_BM * D * 2;
@@ -105,6 +106,40 @@ struct WsArgs {
 };
 
 
+// Ring entries of this kernel: 2 q + f for item q (f = 1: the head's products
+// admit the two-instruction rounding and the fused recompute), -1 for none left.
+__device__ __forceinline__ int ring_q(int v) { return v >> 1; }
+__device__ __forceinline__ bool ring_fast(int v) { return (v & 1) != 0; }
+
+// ---------------------------------------------------------------------------
+// Hand-out of the CTA's k-th item, by one warp of the tensor-core warpgroup:
+// claims it from the work counter (heaviest first), reads its head's exponent
+// statistics, stages its Q into slot k % 3 and publishes it in the ring. Items
+// 0-2 go out at the start, item k + 3 after the output of item k, when every
+// role is done with item k and so with slot k % 3; that is still an item ahead of
+// the producers (they cannot store item k + 2 before that output is read). None
+// of the global-memory latency of a hand-out sits on the path of the roles that
+// wait for it. Returns false once no item is left (-1 published).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ bool ws_hand_out(const WsArgs& a, unsigned char* smem, const WsSmem& L, int k, int lane) {
+  const Problem& p = a.p;
+  const ItemRing sched{smem_u32(smem + L.sched)};
+  int q = lane == 0 ? claim_item(a.counter, a.n_items) : 0;
+  q = __shfl_sync(0xFFFFFFFFu, q, 0);
+  if (q < 0) {
+    if (lane == 0) publish_item(sched, k, -1);
+    return false;
+  }
+  const ItemInfo it = ws_decode(q, p, a.n_rb);
+  const bool fast = head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk, p.emax_sum_limit);
+  ws_stage_q<D>(reinterpret_cast<float*>(smem + L.q) + (k % 3) * ws_qfloats<D>(), p, it, lane, 32);
+  __threadfence_block();
+  __syncwarp();
+  if (lane == 0) publish_item(sched, k, 2 * q + (fast ? 1 : 0));
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // Producers: PS(mu) scores of every item into the item's row buffer.
 // ---------------------------------------------------------------------------
@@ -123,43 +158,33 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
   // failure-path tests: hand over nothing, so that every other warp's bounded wait runs out
   if (p.debug_stall == LAMP_DEBUG_STALL_PRODUCERS) return;
   const ItemRing sched{smem_u32(smem + L.sched)};
-  // claim the first two items and stage their Q (the consumers do the later ones)
-  if (warp == 0 && lane == 0) {
-    const int q0 = claim_item(a.counter, a.n_items);
-    sched.put(0, q0);
-    publish_item(sched, 1, q0 < 0 ? -1 : claim_item(a.counter, a.n_items));
-  }
-  named_sync(BAR_PROD, WS_NP * 32);
-  for (int k0 = 0; k0 < 2; ++k0) {
-    const int q0 = sched.get(k0);
-    if (q0 < 0) break;
-    ws_stage_q<D>(qbase + k0 * ws_qfloats<D>(), p, ws_decode(q0, p, a.n_rb), warp * 32 + lane, WS_NP * 32);
-  }
-  named_sync(BAR_PROD, WS_NP * 32);
   int deal = 0;     // producer warp that takes the next unit
   for (int k = 0;; ++k) {
     const int buf = k & 1;
     const uint32_t ph = ((k - 2) >> 1) & 1;
-    // item k is claimed and its Q staged (with the consumers' hand-off of item
-    // k - 2); one decision per warp: the tile routine synchronises the whole warp
-    if (k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + BAR_PREADY + buf, ph))) {
+    // item k, published with its Q staged by the hand-out (one decision per
+    // warp: the tile routine synchronises the whole warp)
+    int v = lane == 0 ? wait_published(sched, k) : 0;
+    v = __shfl_sync(0xFFFFFFFFu, v, 0);
+    if (v == -2) {
       ws_timeout(p);
       return;
     }
-    const int q = sched.get(k);
-    if (q < 0) break;
-    const ItemInfo it = ws_decode(q, p, a.n_rb);
-    const float* sQ = qbase + buf * ws_qfloats<D>();
-    const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
-                                                          p.emax_sum_limit);
+    if (v < 0) break;
+    const ItemInfo it = ws_decode(ring_q(v), p, a.n_rb);
+    const float* sQ = qbase + (k % 3) * ws_qfloats<D>();
+    const bool fast = (RND != kRndExact) && ring_fast(v);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
     float* rows = reinterpret_cast<float*>(smem + L.rows + buf * rb);
     const int U = (it.kv_end + WS_UNIT - 1) / WS_UNIT;
     // the buffer itself is free once item k - 2's P.V has completed and its
     // output has been read (tfree): the tile routine waits for that only before
-    // its first store
-    if (!ws_produce_tile<D, RND>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
-                                 negc, pow2s, scale2, s, k >= 2 ? bars + BAR_TFREE + buf : nullptr, ph)) {
+    // its first store. A warp without a unit in this item waits for it before its
+    // arrival, so that no arrival on full[b] runs two items ahead of another's.
+    const int first = (warp - deal + WS_NP) % WS_NP;
+    if (!ws_produce_tile<D, RND>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, first, fast, Kh, negc, pow2s, scale2, s,
+                                 k >= 2 ? bars + BAR_TFREE + buf : nullptr, ph) ||
+        (first >= U && k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + BAR_TFREE + buf, ph)))) {
       ws_timeout(p);
       return;
     }
@@ -226,7 +251,6 @@ template <int D, int RND, int VAR>
 __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem, const WsSmem& L, int cw, int lane) {
   constexpr int NCT = WS_NC * 32;  // consumer threads
   const Problem& p = a.p;
-  const int tidc = cw * 32 + lane;
   const int nwords = (p.n_k + 31) >> 5;
   const bool refine_ok = VAR != LAMP_GIVEN_MASK && isfinite(p.tau) && p.tau >= 0.f;
   const float band = WS_BAND * p.tau;
@@ -237,32 +261,21 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
   const ItemRing sched{smem_u32(smem + L.sched)};
   long long nsel = 0;
   for (int k = 0;; ++k) {
-    // items 0 and 1 come from the producers (all threads agree on whether the
-    // wait for them gave up), later ones from this warpgroup
-    int q;
-    if (k < 2) {
-      q = wait_published(sched, k);
-      if (named_or(BAR_CONS, NCT, q == -2)) {
-        ws_timeout(p);
-        return;
-      }
-    } else {
-      q = sched.get(k);
-    }
-    if (q < 0) break;
+    // item k (published before the producers started it), then its scores; the
+    // barrier also makes all threads agree on a wait that gave up
+    const int v = wait_published(sched, k);
     const int buf = k & 1;
-    // claim item k + 2 now, so that the tensor-core warpgroup can prefetch its V
-    if (tidc == 0) publish_item(sched, k + 2, claim_item(a.counter, a.n_items));
-    const bool ok = mbar_wait(bars + BAR_FULL + buf, (k >> 1) & 1);
-    if (named_or(BAR_CONS, NCT, !ok)) {  // also makes item k + 2's number visible to every consumer
+    const bool ok = v != -2 && (v == -1 || mbar_wait(bars + BAR_FULL + buf, (k >> 1) & 1));
+    if (named_or(BAR_CONS, NCT, !ok)) {
       ws_timeout(p);
       return;
     }
+    if (v < 0) break;
+    const int q = ring_q(v);
     const ItemInfo it = ws_decode(q, p, a.n_rb);
     const uint16_t* Kh = p.K + (size_t)it.bh * p.n_k * D;
-    const bool fast = (RND != kRndExact) && head_fast_ok(a.stats + (size_t)it.bh * a.nchunk * 4, a.nchunk,
-                                                          p.emax_sum_limit);
-    float* sQ = qbase + buf * ws_qfloats<D>();
+    const bool fast = (RND != kRndExact) && ring_fast(v);
+    const float* sQ = qbase + (k % 3) * ws_qfloats<D>();
     float* rows = reinterpret_cast<float*>(smem + L.rows + buf * rb);
     float* st = reinterpret_cast<float*>(smem + L.stats) + buf * WS_BM * 2;
     const int written = ((it.kv_end + WS_UNIT - 1) / WS_UNIT) * WS_UNIT;  // keys the producers wrote
@@ -427,9 +440,7 @@ __device__ __forceinline__ void ws_consumer(const WsArgs& a, unsigned char* smem
     }
     fence_async_smem();  // P (generic-proxy stores) becomes visible to the tensor core
     named_sync(BAR_CONS, NCT);  // every P row of the item is in place; Q of the item is no longer read
-    const int q2 = sched.get(k + 2);
-    if (q2 >= 0) ws_stage_q<D>(sQ, p, ws_decode(q2, p, a.n_rb), tidc, NCT);
-    mbar_arrive(bars + BAR_PREADY + buf);  // P of item k in place, Q of item k + 2 staged
+    mbar_arrive(bars + BAR_PREADY + buf);  // P of item k in place
   }
   if (lane == 0 && nsel && p.nsel_out) atomicAdd(p.nsel_out, (unsigned long long)nsel);
 }
@@ -461,9 +472,9 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
       if (Tl < 0) {
         if (sched.count() <= kl) return false;  // item kl is not claimed yet
         __threadfence_block();
-        const int q = sched.get(kl);
-        if (q < 0) return false;
-        const ItemInfo it = ws_decode(q, p, a.n_rb);
+        const int v = sched.get(kl);
+        if (v < 0) return false;
+        const ItemInfo it = ws_decode(ring_q(v), p, a.n_rb);
         Tl = (it.kv_end + WS_VKEYS - 1) / WS_VKEYS;
         bhl = it.bh;
         tl = 0;
@@ -522,14 +533,18 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
   const float* stats = reinterpret_cast<const float*>(smem + L.stats);
   uint16_t* otile = reinterpret_cast<uint16_t*>(smem + L.otile);
   bool good = true;
+  // items 0-2 at the start, item k + 3 after item k's output
+  const bool handler = ew == 1;
+  bool more = true;
+  for (int k0 = 0; handler && more && k0 < 3; ++k0) more = ws_hand_out<D>(a, smem, L, k0, lane);
   for (int k = 0;; ++k) {
-    const int q = wait_published(sched, k);
-    if (q == -1) break;
-    if (q < 0) {  // the wait gave up (agreed: every thread polls the same count)
+    const int v = wait_published(sched, k);
+    if (named_or(BAR_EPI, 128, v == -2)) {  // the wait gave up (all four warps agree)
       good = false;
       break;
     }
-    const ItemInfo it = ws_decode(q, p, a.n_rb);
+    if (v < 0) break;
+    const ItemInfo it = ws_decode(ring_q(v), p, a.n_rb);
     if (issuer && ok) mma_item(k, it);
     __syncwarp();
     // a failed issue leaves the item's accumulator incomplete: the epilogue's
@@ -538,6 +553,7 @@ __device__ __forceinline__ void ws_tensor_warpgroup(const WsArgs& a, const CUten
       good = false;
       break;
     }
+    if (handler && more) more = ws_hand_out<D>(a, smem, L, k + 3, lane);
   }
   if (issuer) {
     // drain: every MMA issued and every V load in flight completes before the
@@ -573,7 +589,8 @@ __global__ void __launch_bounds__(WS_NT, 1) ws_kernel(const WsArgs a, const __gr
     }
     mbar_init(bars + bar_drain<D>(), 1);
     mbar_fence_init();
-    ItemRing{smem_u32(smem + L.sched)}.set_count(0);  // no item published yet
+    const ItemRing sched{smem_u32(smem + L.sched)};
+    sched.set_count(0);  // no item published yet
   }
   if (warp == WS_MW) tmem_alloc(tslot, WS_TMEM_COLS);
   tc_fence_before();
@@ -605,7 +622,8 @@ cudaError_t ws_launch_one(const WsArgs& a, const CUtensorMap& tmV, int grid, siz
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, k);
   if (e != cudaSuccess) return e;
-  if (fa.numRegs != kWsLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split assumes this pool
+  // the register split assumes this pool, and the block must be launchable with it
+  if (fa.numRegs != kWsLaunchRegs || fa.maxThreadsPerBlock < WS_NT) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, WS_NT, smem, st>>>(a, tmV);

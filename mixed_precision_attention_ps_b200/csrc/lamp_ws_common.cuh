@@ -75,7 +75,8 @@ __host__ __device__ constexpr int sw_bytes(int n) { return ((n + 63) / 64) * 409
 // the consumers' hand-off of an earlier tile, the consumers after their own
 // barrier, the tensor-core warpgroup after seeing the count pass k.
 constexpr int kRing = 8;
-// The ring, addressed through its 32-bit shared-window address.
+// The ring, addressed through its 32-bit shared-window address: ring[0..7] and
+// the published count at [8].
 struct ItemRing {
   uint32_t a;  // address of ring[0]
   __device__ __forceinline__ int get(int k) const { return ld_volatile_shared(a + 4 * (k & (kRing - 1))); }
