@@ -9,9 +9,10 @@
 // the same as in the whole-row kernels; only the work is split differently.
 //
 // A row is cut into 512-key chunks, one CTA of 256 threads per (chunk, b, h):
-//   1. scores: the chunk's K rows go to shared memory by cp.async (16-byte pieces
-//      swizzled against bank conflicts); a thread computes two keys as one packed
-//      pair per PS(mu) step. The low-precision scores go to a scratch buffer (L2
+//   1. scores: the chunk's K rows go to shared memory by TMA, 16 dimensions of
+//      the 512 keys per load (two boxes of 256 keys x 32 bytes, 32-byte swizzle, so
+//      that a thread's two 16-byte reads of a key hit all 32 banks across a
+//      quarter warp); a thread computes two keys as one packed pair per PS(mu) step. The low-precision scores go to a scratch buffer (L2
 //      resident), with per (row, chunk) statistics: maximum, first argmax and
 //      S = sum of exp(y - max) over the chunk's other keys (binary32 expf summed in
 //      double).
@@ -33,6 +34,7 @@
 #include "lamp.h"
 #include "lamp_device.cuh"
 #include "lamp_kernels.h"
+#include "lamp_umma.cuh"
 
 namespace lamp {
 namespace {
@@ -112,20 +114,22 @@ __device__ __forceinline__ float block_sum_f(float v, float* red) {
 // ---------------------------------------------------------------------------
 // 1. Scores and chunk statistics. grid (n_ch, B*H).
 // K comes in slices of 16 dimensions of all 512 keys through a ring of DC_NR
-// slots (cp.async, [2 pieces][512 keys] uint4 per slot, so the 16-byte loads of
-// consecutive threads are consecutive). Thread t computes keys t and t + 256 for
-// the NQ query rows at once; a slice's 16 values of each Q row sit in registers.
-// The two-instruction rounding is taken optimistically: the largest and smallest
-// magnitudes of the chunk's K values are folded on the way (binary32 max / min of
-// the widened values; padding keys hold 1.0), and a chunk outside the rounding's
-// domain (or holding an exact zero, conservatively) is computed again with the
-// exact rounding.
+// slots, one TMA load of two boxes (keys k0 .. k0 + 255 and k0 + 256 .. + 511, 32
+// bytes of each) per slice, completing on the slot's mbarrier. Thread t computes
+// keys t and t + 256 for the NQ query rows at once; a slice's 16 values of each Q
+// row sit in registers. Keys past the row read as zero from the TMA and are
+// replaced by 1.0 (their scores are masked; 1.0 leaves the magnitude test below
+// unchanged). The two-instruction rounding is taken optimistically: the largest
+// and smallest magnitudes of the chunk's K values are folded on the way (binary32
+// max / min of the widened values), and a chunk outside the rounding's domain (or
+// holding an exact zero, conservatively) is computed again with the exact rounding.
 // ---------------------------------------------------------------------------
-constexpr int DC_NR = 4;  // K slices in the ring
+constexpr int DC_NR = 4;                           // K slices in the ring
+constexpr uint32_t DC_SLICE = DC_CK * 16 * 2;      // bytes of a slice (16 dimensions of 512 keys)
 
 template <int D>
-__host__ __device__ constexpr size_t dec_scores_smem() {
-  return (size_t)DC_MAXQ * D * 4 + (size_t)DC_NR * 2 * DC_CK * 16;
+__host__ __device__ constexpr size_t dec_scores_smem() {  // ring, Q rows, 1024-byte alignment slack
+  return (size_t)DC_NR * DC_SLICE + (size_t)DC_MAXQ * D * 4 + 1024;
 }
 
 __device__ __forceinline__ int f32_exp(float v) { return (int)((__float_as_uint(v) >> 23) & 0xFFu); }
@@ -141,33 +145,44 @@ __device__ __forceinline__ bool dec_fast_ok(float qmax, float qmin, float kmax, 
   return (eq + ek <= emax_sum_limit) && (lq + lk >= -126);
 }
 
+// The slices of one pass over the chunk. g counts the slices this CTA has taken
+// through the ring (slot g % DC_NR, phase (g / DC_NR) & 1) across passes; ok turns
+// false when a wait gave up (the pass then skips the waits that follow).
 template <int D, int NQ, int MODE, bool FOLD>
-__device__ __forceinline__ void dec_slices(const uint16_t* Kh, int k0, int n_k, const float* sQf, uint4* ring,
-                                           u64 (&acc)[NQ], float& kmax, float& kmin, u64 negc, u64 pow2s, int s) {
+__device__ __forceinline__ void dec_slices(const CUtensorMap* tmK, int bh, int k0, int n_k, const float* sQf,
+                                           unsigned char* ring, uint64_t* bars, int& g, u64 (&acc)[NQ],
+                                           float& kmax, float& kmin, u64 negc, u64 pow2s, int s, bool& ok) {
   constexpr int NSL = D / 16;
   const int t = threadIdx.x;
-  auto issue = [&](int sl) {
+  auto issue = [&](int sl) {  // thread 0
     if (sl < NSL) {
-      uint4* slot = ring + (sl % DC_NR) * 2 * DC_CK;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int u = t + DC_T * r, j = u >> 1, pc = u & 1;
-        uint4* dst = slot + pc * DC_CK + j;
-        if (k0 + j < n_k) cp_async16(dst, Kh + (size_t)(k0 + j) * D + sl * 16 + pc * 8);
-        else *dst = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // 1.0: no effect on the test
-      }
+      const int gs = g + sl;
+      unsigned char* slot = ring + (gs % DC_NR) * DC_SLICE;
+      uint64_t* bar = bars + gs % DC_NR;
+      mbar_expect_tx(bar, DC_SLICE);
+      tma_load_3d(slot, tmK, 16 * sl, k0, bh, bar);
+      tma_load_3d(slot + DC_SLICE / 2, tmK, 16 * sl, k0 + DC_T, bh, bar);
     }
-    cp_async_commit();
   };
+  const bool va = k0 + t < n_k, vb = k0 + t + DC_T < n_k;
+  const int sw = 16 * ((t >> 2) & 1);  // the 32-byte swizzle: 16-byte half c of row t sits at 16 c ^ sw
+  const uint4 one = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
 #pragma unroll
   for (int i = 0; i < NQ; ++i) acc[i] = 0ull;
-  for (int sl = 0; sl < DC_NR - 1; ++sl) issue(sl);
+  if (t == 0)
+    for (int sl = 0; sl < DC_NR - 1; ++sl) issue(sl);
   for (int sl = 0; sl < NSL; ++sl) {
-    cp_async_wait<DC_NR - 2>();
-    __syncthreads();  // slice sl has landed everywhere; every thread is done with slice sl - 1
-    issue(sl + DC_NR - 1);
-    const uint4* slot = ring + (sl % DC_NR) * 2 * DC_CK;
-    const uint4 a0 = slot[t], a1 = slot[DC_CK + t], b0 = slot[t + DC_T], b1 = slot[DC_CK + t + DC_T];
+    const int gs = g + sl;
+    if (ok) ok = mbar_wait(bars + gs % DC_NR, (gs / DC_NR) & 1);
+    __syncthreads();  // slice sl has landed; every thread is done with slice sl - 1, whose slot is refilled
+    if (t == 0) issue(sl + DC_NR - 1);
+    const unsigned char* slot = ring + (gs % DC_NR) * DC_SLICE;
+    uint4 a0 = *reinterpret_cast<const uint4*>(slot + 32 * t + sw);
+    uint4 a1 = *reinterpret_cast<const uint4*>(slot + 32 * t + (16 ^ sw));
+    uint4 b0 = *reinterpret_cast<const uint4*>(slot + DC_SLICE / 2 + 32 * t + sw);
+    uint4 b1 = *reinterpret_cast<const uint4*>(slot + DC_SLICE / 2 + 32 * t + (16 ^ sw));
+    if (!va) a0 = a1 = one;
+    if (!vb) b0 = b1 = one;
     const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     float q[NQ][16];
@@ -192,15 +207,16 @@ __device__ __forceinline__ void dec_slices(const uint16_t* Kh, int k0, int n_k, 
       for (int i = 0; i < NQ; ++i) acc[i] = ps_step<MODE>(pack2(q[i][e], q[i][e]), kp, acc[i], negc, pow2s, s);
     }
   }
-  cp_async_wait<0>();
   __syncthreads();  // the ring may be refilled
+  g += NSL;
 }
 
 template <int D, int RND, int NQ>
-__global__ void __launch_bounds__(DC_T) dec_scores_kernel(const DecArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  float* sQf = reinterpret_cast<float*>(smem);
-  uint4* ring = reinterpret_cast<uint4*>(smem + (size_t)DC_MAXQ * D * 4);
+__global__ void __launch_bounds__(DC_T) dec_scores_kernel(const DecArgs a, const __grid_constant__ CUtensorMap tmK) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* ring = smem_raw + smem_align1k_pad(smem_raw);
+  float* sQf = reinterpret_cast<float*>(ring + DC_NR * DC_SLICE);
+  __shared__ __align__(8) uint64_t bars[DC_NR];
   __shared__ float redf[DC_T / 32];
   __shared__ int redi[DC_T / 32];
   __shared__ double redd[DC_T / 32];
@@ -211,6 +227,8 @@ __global__ void __launch_bounds__(DC_T) dec_scores_kernel(const DecArgs a) {
   if (t == 0) {  // the whole chunk of K towards L2 at once; the ring then reads it from there
     const int nk = min(DC_CK, p.n_k - k0);
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(Kh + (size_t)k0 * D), "r"(nk * D * 2) : "memory");
+    for (int i = 0; i < DC_NR; ++i) mbar_init(bars + i, 1);
+    mbar_fence_init();
   }
   if (c == 0 && t < NQ) a.rowdone[(size_t)bh * NQ + t] = 0;  // the selection kernel counts finished chunks
   if (c == 0 && bh == 0 && t == 0 && p.nsel_out) *p.nsel_out = 0ull;
@@ -229,19 +247,24 @@ __global__ void __launch_bounds__(DC_T) dec_scores_kernel(const DecArgs a) {
   u64 acc[NQ];
   float kmax = 0.f, kmin = INFINITY;
   int fast = 0;
+  int g = 0;       // slices taken through the ring
+  bool ok = true;  // no wait gave up
+  __syncthreads();  // the barriers are initialised, Q is in place
   if (RND == kRndExact) {
-    dec_slices<D, NQ, kStepExact, false>(Kh, k0, p.n_k, sQf, ring, acc, kmax, kmin, negc, pow2s, s);
+    dec_slices<D, NQ, kStepExact, false>(&tmK, bh, k0, p.n_k, sQf, ring, bars, g, acc, kmax, kmin, negc, pow2s, s, ok);
   } else {
-    dec_slices<D, NQ, RND == kRndFast ? kStepFast : kStepF32, true>(Kh, k0, p.n_k, sQf, ring, acc, kmax, kmin, negc,
-                                                                    pow2s, s);
+    dec_slices<D, NQ, RND == kRndFast ? kStepFast : kStepF32, true>(&tmK, bh, k0, p.n_k, sQf, ring, bars, g, acc,
+                                                                    kmax, kmin, negc, pow2s, s, ok);
     qmax = block_max(qmax, redf);
     qmin = -block_max(-qmin, redf);
     kmax = block_max(kmax, redf);
     kmin = -block_max(-kmin, redf);
     fast = dec_fast_ok(qmax, qmin, kmax, kmin, p.emax_sum_limit) ? 1 : 0;
     if (!fast)  // outside the two-instruction rounding's domain: the exact rounding
-      dec_slices<D, NQ, kStepExact, false>(Kh, k0, p.n_k, sQf, ring, acc, kmax, kmin, negc, pow2s, s);
+      dec_slices<D, NQ, kStepExact, false>(&tmK, bh, k0, p.n_k, sQf, ring, bars, g, acc, kmax, kmin, negc, pow2s, s,
+                                           ok);
   }
+  if (!ok && p.status_out) atomicExch(p.status_out, LAMP_ERR_TIMEOUT);
   if (t == 0) a.cfast[(size_t)bh * a.n_ch + c] = fast;
 #pragma unroll
   for (int i = 0; i < NQ; ++i) {
@@ -528,32 +551,35 @@ __global__ void __launch_bounds__(DC_T) dec_select_kernel(const DecArgs a) {
 }
 
 template <int D, int RND, int NQ>
-cudaError_t dec_launch_scores(const DecArgs& a, dim3 grid, cudaStream_t st) {
+cudaError_t dec_launch_scores(const DecArgs& a, const CUtensorMap& tmK, dim3 grid, cudaStream_t st) {
   const size_t smem = dec_scores_smem<D>();
   cudaError_t e = cudaFuncSetAttribute(dec_scores_kernel<D, RND, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  dec_scores_kernel<D, RND, NQ><<<grid, DC_T, smem, st>>>(a);
+  dec_scores_kernel<D, RND, NQ><<<grid, DC_T, smem, st>>>(a, tmK);
   return cudaGetLastError();
 }
 
 template <int D, int RND>
-cudaError_t dec_launch_rnd(const DecArgs& a, dim3 grid, cudaStream_t st) {
+cudaError_t dec_launch_rnd(const DecArgs& a, const CUtensorMap& tmK, dim3 grid, cudaStream_t st) {
   switch (a.p.n_q) {
-    case 1: return dec_launch_scores<D, RND, 1>(a, grid, st);
-    case 2: return dec_launch_scores<D, RND, 2>(a, grid, st);
-    case 3: return dec_launch_scores<D, RND, 3>(a, grid, st);
-    default: return dec_launch_scores<D, RND, 4>(a, grid, st);
+    case 1: return dec_launch_scores<D, RND, 1>(a, tmK, grid, st);
+    case 2: return dec_launch_scores<D, RND, 2>(a, tmK, grid, st);
+    case 3: return dec_launch_scores<D, RND, 3>(a, tmK, grid, st);
+    default: return dec_launch_scores<D, RND, 4>(a, tmK, grid, st);
   }
 }
 
 template <int D>
 cudaError_t dec_launch(const DecArgs& a, int rnd, cudaStream_t st) {
   const dim3 grid((unsigned)a.n_ch, (unsigned)(a.p.B * a.p.H));
-  cudaError_t e;
-  if (rnd == kRndFast) e = dec_launch_rnd<D, kRndFast>(a, grid, st);
-  else if (rnd == kRndNone) e = dec_launch_rnd<D, kRndNone>(a, grid, st);
-  else e = dec_launch_rnd<D, kRndExact>(a, grid, st);
+  // K slices: boxes of 16 dimensions x 256 keys of one (b, h), 32-byte swizzle
+  CUtensorMap tmK;
+  cudaError_t e = make_tmap_bf16(&tmK, a.p.K, D, a.p.n_k, a.p.B * a.p.H, 16, DC_T, 32);
+  if (e != cudaSuccess) return e;
+  if (rnd == kRndFast) e = dec_launch_rnd<D, kRndFast>(a, tmK, grid, st);
+  else if (rnd == kRndNone) e = dec_launch_rnd<D, kRndNone>(a, tmK, grid, st);
+  else e = dec_launch_rnd<D, kRndExact>(a, tmK, grid, st);
   if (e != cudaSuccess) return e;
   if (a.p.variant == LAMP_STRICT) dec_select_kernel<D, LAMP_STRICT><<<grid, DC_T, 0, st>>>(a);
   else if (a.p.variant == LAMP_RELAXED) dec_select_kernel<D, LAMP_RELAXED><<<grid, DC_T, 0, st>>>(a);

@@ -85,8 +85,9 @@ constexpr size_t kStaticSmemReserve = 256;
 Workspace plan_workspace(const Problem& p, int num_sms, size_t smem_optin);
 // Tensor map of a [bh][n][d] bf16 tensor (row-major, this GPU's memory) for TMA
 // boxes of box_x dimensions x box_y rows of one (b, h); rows past n read as zero.
+// swizzle: 0, 32 or 128 (bytes of the shared-memory swizzle pattern).
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n, int bh, int box_x, int box_y,
-                           bool swizzle128);
+                           int swizzle);
 cudaError_t launch_prep(const Problem& p, const Workspace& ws, char* base, cudaStream_t st);
 cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num_sms, cudaStream_t st);
 bool ws_fits(int d, int n_k, size_t smem_optin);

@@ -820,7 +820,7 @@ cudaError_t launch_stream(const Problem& p, const Workspace& ws, char* base, int
   a.ld = stream_slab_ld(p.n_k);
   a.rows = reinterpret_cast<RowStat*>(base + ws.st_rows);
   CUtensorMap tmV;
-  const cudaError_t e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, true);
+  const cudaError_t e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, 128);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   const int rnd = p.mu == 23 ? kRndNone : (p.mu <= 10 ? kRndFast : kRndExact);

@@ -32,7 +32,7 @@ cudaError_t encoder(PFN_cuTensorMapEncodeTiled_v12000& fn) {
 }  // namespace
 
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n, int bh, int box_x, int box_y,
-                           bool swizzle128) {
+                           int swizzle) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   cudaError_t e = encoder(fn);
   if (e != cudaSuccess) return e;
@@ -42,7 +42,8 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n, int
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : (swizzle == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE),
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

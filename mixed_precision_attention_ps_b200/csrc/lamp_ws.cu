@@ -656,7 +656,7 @@ cudaError_t launch_ws(const Problem& p, const Workspace& ws, char* base, int num
   a.n_rb = (p.n_q + WS_BM - 1) / WS_BM;
   a.n_items = a.n_rb * p.B * p.H;
   CUtensorMap tmV;
-  cudaError_t e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, true);
+  cudaError_t e = make_tmap_bf16(&tmV, p.V, p.d, p.n_k, p.B * p.H, 64, WS_VKEYS, 128);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   const size_t smem = ws_smem_bytes(p.d, p.n_k);
