@@ -75,6 +75,16 @@ __host__ __device__ constexpr int sw_bytes(int n) { return ((n + 63) / 64) * 409
 // the consumers' hand-off of an earlier tile, the consumers after their own
 // barrier, the tensor-core warpgroup after seeing the count pass k.
 constexpr int kRing = 8;
+// Volatile 32-bit shared-memory accesses by shared-window address (the ring is
+// polled by other warps of the CTA).
+__device__ __forceinline__ int ld_volatile_shared(uint32_t addr) {
+  int v;
+  asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_volatile_shared(uint32_t addr, int v) {
+  asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 // The ring, addressed through its 32-bit shared-window address: ring[0..7] and
 // the published count at [8].
 struct ItemRing {
