@@ -5,6 +5,8 @@
 // "Implementation strategy" (steps 1 and 3) and "Experimental results" (PS(mu)).
 #pragma once
 
+#include <type_traits>
+
 #include "lamp.h"
 #include "lamp_device.cuh"
 #include "lamp_kernels.h"
@@ -231,7 +233,7 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
   // one stream position: compute slice pos, then stage slice pos + 1 into the free
   // binary32 buffer and start the load of slice pos + 3 into `cur` (the register
   // set of pos + 1; two sets alternate, so no load is waited on early)
-  auto body = [&](int pos, uint4 (&cur)[2]) {
+  auto body = [&](auto mode, int pos, uint4 (&cur)[2]) {
     const int j = first + WS_NP * (pos / NSL), sl = pos % NSL;
     if (sl == 0) {
 #pragma unroll
@@ -241,9 +243,7 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
     }
     const float* qs = sQ + sl * WS_DS * WS_BM;
     const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
-    if (RND == kRndFast && fast) ws_score_slice<kStepFast>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-    else if (RND == kRndNone && fast) ws_score_slice<kStepF32>(qs, ks, qoff, koff, acc, negc, pow2s, s);
-    else ws_score_slice<kStepExact>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+    ws_score_slice<decltype(mode)::value>(qs, ks, qoff, koff, acc, negc, pow2s, s);
     if (sl == NSL - 1) {
       if (free_bar) {  // first store of the call: the buffer's previous contents are no longer read
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(free_bar, free_phase))) {
@@ -286,10 +286,18 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
   if (total > 1) load(1, kra);
   if (total > 2) load(2, krb);
   __syncwarp();
-  for (int pos = 0; pos < total && !failed; pos += 2) {
-    body(pos, kra);
-    if (pos + 1 < total && !failed) body(pos + 1, krb);
-  }
+  // one step form for the whole tile: the exact rounding's loop is a separate
+  // copy, so that its code does not sit inside the fast loop (with the branch in
+  // the loop, 3 % of a GPT-2 XL call went to the instruction fetch of the other
+  // warp roles)
+  auto run = [&](auto mode) {
+    for (int pos = 0; pos < total && !failed; pos += 2) {
+      body(mode, pos, kra);
+      if (pos + 1 < total && !failed) body(mode, pos + 1, krb);
+    }
+  };
+  if (RND != kRndExact && fast) run(std::integral_constant<int, RND == kRndFast ? kStepFast : kStepF32>{});
+  else run(std::integral_constant<int, kStepExact>{});
   return !failed;  // (a warp with no unit of its own writes nothing and so needs no wait)
 }
 
