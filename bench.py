@@ -100,6 +100,17 @@ def is_decode(w) -> bool:
     return w.n_q <= 4 and w.n_k >= 512
 
 
+def library_launches_per_call(w, variant: int) -> int:
+    """The library's kernels in one attention call, by its routing: decode shapes run
+    the scores and the selection kernels; the others the exponent-statistics kernel
+    and one row kernel, and strict rows too long for the whole-row kernel (more than
+    1024 keys at d = 64, 896 at d = 128) its two streamed passes."""
+    if is_decode(w):
+        return 2
+    whole_row = w.n_k <= (1024 if w.d == 64 else 896)
+    return 3 if (variant == 0 and not whole_row) else 2
+
+
 def rank_workload(w, rank: int):
     """Weak scaling: every rank runs the same shape on its own inputs (seed + rank)."""
     return S.Workload(w.B, w.H, w.n_q, w.n_k, w.d, w.causal, w.outlier_frac, w.outlier_scale, seed=w.seed + rank)
@@ -362,7 +373,7 @@ def run_ours(a, w, variant, mu, tau, cfg):
     clk = clocks.stop()
     times = [s.elapsed_time(e) for s, e in evs]
     ms = max_over_ranks([statistics.mean(times)], dev)[0]
-    launches_per_step = 4 if is_decode(w) else 2  # exponent statistics + row kernel (decode: + 3)
+    launches_per_step = library_launches_per_call(w, variant)
 
     # ---- end to end through the C ABI with host buffers ---------------------------------
     # Every step copies its inputs from pinned host memory and reads its output and

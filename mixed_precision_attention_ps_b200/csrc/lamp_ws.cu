@@ -1,6 +1,6 @@
 // LAMP attention, warp-specialised row kernel (strict, relaxed, given mask) for
 // rows short enough that two blocks of 16 complete score rows fit in shared
-// memory at once (n_k up to 1024 keys at d = 64, 960 at d = 128; the GPT-2 XL
+// memory at once (n_k up to 1024 keys at d = 64, 896 at d = 128; the GPT-2 XL
 // attention shape).
 //
 // Method ("LAMP: Look-Ahead Mixed-Precision Inference of Large Language Models",
