@@ -215,7 +215,7 @@ __device__ __forceinline__ void st_producer(const StArgs& a, unsigned char* smem
       } else {
         // the tile buffer is free once tile k - 2's P.V has completed and been read
         // (tfree): the tile routine waits for that only before its first store
-        if (!ws_produce_tile<D, RND>(p, it, t0, tlen, sQ, tile, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
+        if (!ws_produce_tile<D, RND, WS_DS>(p, it, t0, tlen, sQ, tile, ksw, lane, (warp - deal + WS_NP) % WS_NP, fast, Kh,
                                      negc, pow2s, scale2, s, k >= 2 ? bars + SB_TFREE + buf : nullptr, ph)) {
           ws_timeout(p);
           return;

@@ -182,7 +182,7 @@ __device__ __forceinline__ void ws_producer(const WsArgs& a, unsigned char* smem
     // its first store. A warp without a unit in this item waits for it before its
     // arrival, so that no arrival on full[b] runs two items ahead of another's.
     const int first = (warp - deal + WS_NP) % WS_NP;
-    if (!ws_produce_tile<D, RND>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, first, fast, Kh, negc, pow2s, scale2, s,
+    if (!ws_produce_tile<D, RND, 2>(p, it, 0, it.kv_end, sQ, rows, ksw, lane, first, fast, Kh, negc, pow2s, scale2, s,
                                  k >= 2 ? bars + BAR_TFREE + buf : nullptr, ph) ||
         (first >= U && k >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bars + BAR_TFREE + buf, ph)))) {
       ws_timeout(p);

@@ -165,10 +165,14 @@ __device__ __forceinline__ void ws_stage_q(float* sQ, const Problem& p, const It
 // over rows: acc[rp][i] holds rows 8gr + 2rp, 8gr + 2rp + 1 at key 4gk + i.
 //   qs: Q of this slice, [WS_DS][16] f32 (lane rows 8gr..8gr+7 at qoff = 8gr);
 //   ks: warp's K slice, [WS_DS][64] f32 (lane keys at koff = 4gk).
-template <int MODE>
+// KU: steps unrolled together. The whole-row kernel takes 2: its producer loop
+// then fits the instruction cache that the five warp roles of an SM share
+// (GPT-2 XL strict 0.219 -> 0.211 ms, batch 8 relaxed 1.62 -> 1.39 ms against
+// all 8); the streamed kernel at d = 128 keeps all 8 (2 was 1.5 % slower there).
+template <int MODE, int KU>
 __device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, const float* __restrict__ ks, int qoff,
                                                int koff, u64 (&acc)[4][4], u64 negc, u64 pow2s, int s) {
-#pragma unroll
+#pragma unroll KU
   for (int dd = 0; dd < WS_DS; ++dd) {
     const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff);
     const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(qs + dd * WS_BM + qoff + 4);
@@ -195,7 +199,7 @@ __device__ __forceinline__ void ws_score_slice(const float* __restrict__ qs, con
 // starts: the warp waits for free_bar's phase free_phase (when free_bar is not
 // null) only before its first store, one unit of arithmetic later. Returns false
 // when that bounded wait gave up.
-template <int D, int RND>
+template <int D, int RND, int KU>
 __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo& it, int t0, int tlen,
                                                 const float* sQ, float* rows, float* ksw, int lane, int first,
                                                 bool fast, const uint16_t* Kh, u64 negc, u64 pow2s, u64 scale2,
@@ -243,7 +247,7 @@ __device__ __forceinline__ bool ws_produce_tile(const Problem& p, const ItemInfo
     }
     const float* qs = sQ + sl * WS_DS * WS_BM;
     const float* ks = ksw + (pos & 1) * WS_DS * WS_UNIT;
-    ws_score_slice<decltype(mode)::value>(qs, ks, qoff, koff, acc, negc, pow2s, s);
+    ws_score_slice<decltype(mode)::value, KU>(qs, ks, qoff, koff, acc, negc, pow2s, s);
     if (sl == NSL - 1) {
       if (free_bar) {  // first store of the call: the buffer's previous contents are no longer read
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(free_bar, free_phase))) {
