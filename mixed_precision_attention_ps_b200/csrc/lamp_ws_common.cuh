@@ -70,12 +70,12 @@ __host__ __device__ constexpr int sw_bytes(int n) { return ((n + 63) / 64) * 409
 
 // Items are handed out at run time, heaviest first, from a global counter, so
 // that CTAs which run slower (two SMs share a TPC's resources) take fewer. A
-// CTA claims its k-th item two items ahead: items 0 and 1 by the producers at
-// the start, item k + 2 by the consumers when they begin item k. The number
-// (-1: none left) goes to ring[k % 8] in shared memory, then the published count
-// ring[8] (zeroed at kernel start) rises to k + 1. The producers read it after
-// the consumers' hand-off of an earlier tile, the consumers after their own
-// barrier, the tensor-core warpgroup after seeing the count pass k.
+// CTA's k-th item goes to ring[k % 8] in shared memory (-1: none left), then the
+// published count ring[8] (zeroed at kernel start) rises to k + 1; readers poll
+// the count (bounded) or follow a barrier that orders them after the write.
+// Who claims: in the streamed kernel items 0 and 1 by the producers at the start
+// and item k + 2 by the consumers when they begin item k; in the whole-row
+// kernel one warp of the tensor-core warpgroup, three items ahead (lamp_ws.cu).
 constexpr int kRing = 8;
 // Volatile 32-bit shared-memory accesses by shared-window address (the ring is
 // polled by other warps of the CTA).
